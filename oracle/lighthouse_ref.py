@@ -248,7 +248,7 @@ def attn_bwd(qs, ks, vs, os_, lse, dos):
                 i1 = min(S, i0 + _ROW_BLOCK)
                 s = (qs[b, h, i0:i1] @ ks[b, h, :i1].T) * sigma
                 visible = np.arange(i1)[None, :] <= np.arange(i0, i1)[:, None]
-                P = np.where(visible, np.exp(s - lse[b, h, i0:i1, None]), 0.0)
+                P = np.exp(np.where(visible, s - lse[b, h, i0:i1, None], -np.inf))
                 dP = dos[b, h, i0:i1] @ vs[b, h, :i1].T
                 dS = P * (dP - D[i0:i1, None])
                 dv[b, h, :i1] += P.T @ dos[b, h, i0:i1]
@@ -308,30 +308,49 @@ def gather_bwd(idx, dx_sub, geo: Geometry):
 
 
 # ---------------------------------------------------------------------------------------
+# Storage rounding (SPEC section 9): the layer stores the pyramid, O_sub and dO_sub in its
+# dtype. Round to nearest, ties to even, from the exact value.
+# ---------------------------------------------------------------------------------------
+def round_to(x, store):
+    """Exact value -> nearest value of the storage type ("bf16", "f32" or None = keep)."""
+    x = np.asarray(x, dtype=np.float64)
+    if store is None:
+        return x
+    if store == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if store == "bf16":  # 8 significant bits: scale the frexp mantissa to [128, 256), round
+        m, e = np.frexp(x)
+        return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+    raise ValueError(store)
+
+
+# ---------------------------------------------------------------------------------------
 # Whole layer
 # ---------------------------------------------------------------------------------------
-def layer_fwd(q, k, v, geo: Geometry, g, idx=None):
+def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
     """Forward of the layer. g is the score group size (8 for bf16 inputs, 4 for fp32).
 
-    idx may be given to force a selection (used for the dense recovery identity).
+    idx may be given to force a selection (used for the dense recovery identity). store names
+    the storage type of the stored intermediates (pyramid cells and O_sub), SPEC section 9.
     Returns (O [B,H,N,d] float64, saved dict for layer_bwd).
     """
     geo.check()
-    pq, pk, pv = (build_pyramid(x, geo) for x in (q, k, v))
+    pq, pk, pv = (round_to(build_pyramid(x, geo), store) for x in (q, k, v))
     r = None
     if idx is None:
         r = score(q, k, geo, g)
         idx = select_topk(r, geo)
     qs, ks, vs = gather(q, pq, idx), gather(k, pk, idx), gather(v, pv, idx)
     os_, lse = attn_fwd(qs, ks, vs)
+    os_ = round_to(os_, store)
     o = scatter(idx, os_, geo)
-    saved = dict(idx=idx, score=r, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, geo=geo)
+    saved = dict(idx=idx, score=r, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, geo=geo, store=store)
     return o, saved
 
 
 def layer_bwd(saved, d_o):
     """Backward of the layer: returns (dQ, dK, dV) [B,H,N,d] float64."""
     geo, idx = saved["geo"], saved["idx"]
-    dos = scatter_bwd(idx, d_o, geo)
+    dos = round_to(scatter_bwd(idx, d_o, geo), saved.get("store"))
     dqs, dks, dvs = attn_bwd(saved["qs"], saved["ks"], saved["vs"], saved["os"], saved["lse"], dos)
     return gather_bwd(idx, dqs, geo), gather_bwd(idx, dks, geo), gather_bwd(idx, dvs, geo)

@@ -326,3 +326,16 @@ def test_gradients_finite_differences(N, p, L, S):
             args[which][pos] -= 2 * eps
             num[pos] = (up - loss(*args)) / (2 * eps)
         np.testing.assert_allclose(gr, num, rtol=1e-6, atol=1e-7)
+
+
+# ---------------------------------------------------------------- storage rounding (SPEC 9)
+def test_bf16_rounding_matches_library_conversion():
+    """Round-to-nearest-even to bf16 equals torch's fp32 -> bf16 conversion on fp32 values."""
+    x = np.concatenate([rand(100000, scale=10.0), np.float32([1 + 2 ** -8, 1 + 3 * 2 ** -8,
+                                                              -(1 + 2 ** -8), 0.0, 2 ** -20])])
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_to(x.astype(np.float64), "bf16"), want)
+    assert O.round_to(np.float64(1 + 2 ** -8), "bf16") == 1.0  # tie goes to even
+    assert O.round_to(np.float64(1 + 3 * 2 ** -8), "bf16") == 1 + 2 ** -6
+    y = rand(1000).astype(np.float64) / 3
+    np.testing.assert_array_equal(O.round_to(y, "f32"), y.astype(np.float32).astype(np.float64))
