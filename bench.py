@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Throughput of the Lighthouse selection layer, forward + backward, on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input: the pyramid and
+scores, the stratified top-K, the gather, the causal attention on the S rows and the
+scatter-back, then the backward through all of them. Every stage runs in liblh.so. Inputs are
+resident in HBM before the timed region; each input tensor (1 GiB at 128K) is larger than the
+126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 128k] [--impl reference]
+
+Under torchrun each rank runs its own copy of the workload (heads are independent problems),
+there is no data-path collective, and rank 0 prints one JSON line with the whole-job tokens/s.
+`--impl reference` times the CPU oracle (test infrastructure) on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_hierarchical_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Lighthouse layer fwd+bwd tokens/s at N=128K, 1 B200; % of HBM / tensor roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- process group
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.file.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.file.read())) if len(r) >= 9]
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], None, set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(nm)
+        load = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def stage_work(w, geo):
+    """Algorithmic bytes (HBM-bound stages) or FLOPs (attention) per launch of each stage."""
+    B, H, N, d, S = w.B, w.H, w.N, w.d, w.S
+    e = torch.tensor([], dtype=w.dtype).element_size()
+    R = geo["R"]
+    BH = B * H
+    return {
+        "pyramid_score": ("hbm", 3 * BH * N * d * e + 3 * BH * R * d * e + BH * (N + R) * 4),
+        "select": ("hbm", BH * (N + R) * 4 + BH * S * 4),
+        "gather": ("hbm", 2 * 3 * BH * S * d * e + BH * S * 4),
+        "attn_fwd": ("tensor", 2 * BH * S * S * d),
+        "scatter": ("hbm", BH * S * d * e + BH * N * d * e + BH * S * 4),
+        "scatter_bwd": ("hbm", BH * N * d * e + BH * S * d * e + BH * S * 4),
+        "attn_bwd": ("tensor", 5 * BH * S * S * d),
+        "gather_bwd": ("hbm", 3 * BH * S * d * 4 + 3 * BH * N * d * e + BH * S * 4),
+    }
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import sparse_hierarchical_attention_b200 as lh
+    from sparse_hierarchical_attention_b200 import Shape
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    shape = Shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S, w.dtype)
+    geo = lh.lh_validate(shape)
+    B, H, N, d, S, dt = w.B, w.H, w.N, w.d, w.S, w.dtype
+    R = geo["R"]
+    q, k, v, d_o = make_inputs(w, dev, seed=1000 * rank)
+    E = lambda *s, t=dt: torch.empty(*s, dtype=t, device=dev)  # noqa: E731
+    pq, pk, pv = E(B, H, max(R, 1), d), E(B, H, max(R, 1), d), E(B, H, max(R, 1), d)
+    score = E(B, H, N + R, t=torch.float32)
+    idx = E(B, H, S, t=torch.int32)
+    qs, ks, vs, os_ = (E(B, H, S, d) for _ in range(4))
+    lse = E(B, H, S, t=torch.float32)
+    o = E(B, H, N, d)
+    dos = E(B, H, S, d)
+    dqs, dks, dvs = (E(B, H, S, d, t=torch.float32) for _ in range(3))
+    dq, dk, dv = (E(B, H, N, d) for _ in range(3))
+    ws = torch.zeros(lh.lh_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+
+    stages = [
+        ("pyramid_score", lambda: lh.lh_build_pyramid(shape, q, k, v, pq, pk, pv, score, ws)),
+        ("select", lambda: lh.lh_select_topk(shape, score, idx)),
+        ("gather", lambda: lh.lh_gather(shape, q, k, v, pq, pk, pv, idx, qs, ks, vs, ws)),
+        ("attn_fwd", lambda: lh.lh_attn_fwd(shape, qs, ks, vs, os_, lse, ws)),
+        ("scatter", lambda: lh.lh_scatter(shape, idx, os_, o)),
+        ("scatter_bwd", lambda: lh.lh_scatter_bwd(shape, idx, d_o, dos, ws)),
+        ("attn_bwd", lambda: lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, dqs, dks, dvs, ws)),
+        ("gather_bwd", lambda: lh.lh_gather_bwd(shape, idx, dqs, dks, dvs, dq, dk, dv)),
+    ]
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        for _, fn in stages:
+            fn()
+    torch.cuda.synchronize()
+    rc, flags = lh.lh_check(ws)
+    if rc:
+        raise RuntimeError(f"device fault flags {flags:#x} during warm-up")
+
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = Clocks(local)
+    time.sleep(0.3)
+    t_wall = time.perf_counter()
+    for s in range(K):
+        ev[s][0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            ev[s][i + 1].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = sum(ev[s][0].elapsed_time(ev[s][-1]) for s in range(K))
+    per_stage = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)) / K
+                 for i, (name, _) in enumerate(stages)}
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / K
+    tokens = B * N * world
+    value = tokens / (ms_step / 1e3)
+
+    pk_, src = peaks()
+    work = stage_work(w, geo)
+    stage_report = {}
+    for name, ms in per_stage.items():
+        kind, amount = work[name]
+        if kind == "hbm":
+            ach, peak, unit = amount / (ms / 1e3) / 1e9, pk_["hbm_gbs"], "GB/s"
+        else:
+            ach, peak, unit = amount / (ms / 1e3) / 1e12, pk_["bf16_tflops"], "TFLOP/s"
+        stage_report[name] = {"ms": round(ms, 4), "achieved": round(ach, 2), "unit": unit,
+                              "frac": round(ach / peak, 4), "bound": kind}
+    dom = max(per_stage, key=per_stage.get)
+    kind, amount = work[dom]
+    rf = stage_report[dom]
+    roofline = {"kernel": dom, "bound": "hbm" if kind == "hbm" else "tensor",
+                "achieved": rf["achieved"], "peak": pk_["hbm_gbs"] if kind == "hbm" else pk_["bf16_tflops"],
+                "unit": rf["unit"], "frac": rf["frac"], "traffic": None,
+                "peak_source": f"{src} ({'hbm_gbs' if kind == 'hbm' else 'bf16_tflops'})",
+                "units_per_launch": amount}
+    nf, nb = lh.lh_launches(shape)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world)
+    for t in (pq, pk, pv, score, qs, ks, vs, os_, dos, dqs, dks, dvs, dq, dk, dv, o):
+        del t
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) Q/K/V with the workload's row-scale recipe; dO N(0,1))",
+        "config": {"workload": w.name, "describe": w.describe, "B": B, "H": H, "N": N, "d": d,
+                   "p": w.p, "L": w.L, "S": S, "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"replicas x{world} (independent heads, no collective)",
+                   "l2": "inputs larger than L2 (each input tensor > 126 MB); no flush"},
+        "stages": stage_report, "roofline": roofline, "gpu_launches": (nf + nb) * K,
+        "clocks": clk, "wall_s_timed": round(wall, 3),
+    }
+    if e2e:
+        out["e2e"] = e2e
+    return out
+
+
+def run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world):
+    """Same metric through the public layer API from pinned host buffers: per step, copy Q,K,V,dO
+    in, run lh_layer_fwd + lh_layer_bwd, copy O, dQ, dK, dV out."""
+    from sparse_hierarchical_attention_b200 import LighthouseLayer
+    layer = LighthouseLayer(shape, dev)
+    h_in = [t.cpu().pin_memory() for t in (q, k, v, d_o)]
+    h_out = [torch.empty_like(h_in[0]).pin_memory() for _ in range(4)]
+    d_in = [torch.empty_like(q) for _ in range(4)]
+    d_out = [torch.empty_like(q) for _ in range(4)]
+    saved = layer.new_saved()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for h, dbuf in zip(h_in, d_in):
+            dbuf.copy_(h, non_blocking=True)
+        layer.forward(d_in[0], d_in[1], d_in[2], o=d_out[0], saved=saved)
+        layer.backward(saved, d_in[3], dq=d_out[1], dk=d_out[2], dv=d_out[3])
+        for h, dbuf in zip(h_out, d_out):
+            h.copy_(dbuf, non_blocking=True)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world) / K
+    layer.check()
+    nbytes = sum(t.numel() * t.element_size() for t in h_in)
+    return {"value": round(w.B * w.N * world / (ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
+            "api": "LighthouseLayer.forward/backward -> lh_layer_fwd/lh_layer_bwd"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, frac, seed=0):
+    """One head, the first N/frac tokens (same p, L and rows per chunk), on the host."""
+    N, S = w.N // frac, w.S // frac
+    q, k, v, d_o = make_inputs(w, "cpu", seed=seed, B=1, H=1, N=N)
+    return [t.to(torch.float64).numpy() for t in (q, k, v, d_o)], N, S
+
+
+def time_oracle(w, frac, steps=1):
+    import oracle as O
+    (q, k, v, d_o), N, S = oracle_sample(w, frac)
+    geo = O.Geometry(N, w.p, w.L, S).check()
+    store = "bf16" if w.dtype == torch.bfloat16 else "f32"
+    g = 8 if w.dtype == torch.bfloat16 else 4
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        o, sv = O.layer_fwd(q, k, v, geo, g, store=store)
+        O.layer_bwd(sv, d_o)
+    dt = (time.perf_counter() - t0) / steps
+    # layer tokens/s: this head's N tokens took dt; the layer runs B*H such heads
+    value = N / (dt * w.H * w.B)
+    return value, dt, N, S
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w):
+    frac = 4
+    value, dt, N, S = time_oracle(w, frac)
+    return {"value": round(value, 2), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"head 0 of {w.B * w.H}, first {N} of {w.N} tokens (S={S}, same p, L, "
+                      f"rows per chunk), fwd+bwd in {dt:.2f}s; tokens/s = {N}/({dt:.2f}s x "
+                      f"{w.B * w.H} heads). A prefix has cheaper attention per token than the "
+                      "whole sequence, so this overstates the oracle's full-workload rate."}
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    frac = 16
+    for _ in range(args.warmup):
+        time_oracle(w, frac)
+    t0 = time.perf_counter()
+    vals = [time_oracle(w, frac)[1] for _ in range(args.steps)]
+    total = time.perf_counter() - t0
+    dt = sum(vals) / len(vals)
+    N = w.N // frac
+    value = N / (dt * w.H * w.B)
+    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+          "sample": f"each step: head 0 of {w.B * w.H}, first {N} of {w.N} tokens, fwd+bwd"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * dt, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe as our arm)",
+            "config": {"workload": w.name, "describe": w.describe, "sample_tokens": N},
+            "cpu_baseline": cb, "wall_s": round(total, 2),
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    out = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(WORKLOADS[args.workload])
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * lh.h - C ABI of the Lighthouse selection layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer wraps causal scaled-dot-product attention in five steps. It builds a symmetric
+ * average-pooling pyramid over Q, K and V. It scores every cell with the l2 norms of its query
+ * and key, max-pooled up the levels. It picks a stratified top-K that always keeps the coarsest
+ * level. It gathers the picks into one short causal subsequence and runs dense causal attention
+ * on it. Finally it scatters the outputs back to token positions. The backward pass sends
+ * gradients to Q, K and V through the scatter, the attention and the gather; the selection gets
+ * none.
+ *
+ * Sources: "Long Context Pre-Training with Lighthouse Attention" (gist.science summary),
+ * technical summary sections 2.A (pyramid), 2.B (scoring, selection, no gradient through the
+ * selection), 2.C (gather, dense attention, scatter-back), 2.D (recovery phase = dense SDPA);
+ * and the Nous Research article on edge.aivizor.me, the paragraph listing the four stages
+ * ("two scalar scores per cell", "the coarsest level is always kept").
+ *
+ * Conventions common to every entry point:
+ *  - Tensors are contiguous [B, H, rows, d] with d fastest. They live in device memory that the
+ *    caller allocates and frees. The library never allocates, frees or synchronises, except for
+ *    lh_check, which synchronises the stream it is given.
+ *  - The element type of Q, K, V, pyramid, subsequence and output tensors is shape.dtype (fp32
+ *    or bf16). Score, lse and the sub-gradients dq_sub/dk_sub/dv_sub are always fp32.
+ *  - `stream` is a cudaStream_t passed as void*. NULL means the legacy default stream. Every
+ *    launch is asynchronous and stream-ordered.
+ *  - Return values report host-side validation and launch errors. Nothing is launched when
+ *    validation fails. Device-side faults that the kernels detect (an out-of-range row id, a
+ *    bounded wait that ran out) set a status word in the workspace; lh_check reports it.
+ *  - Every device pointer must be 16-byte aligned; otherwise LH_ERR_INVALID_ARG.
+ *  - Row ids (idx) are int32 ids into the concatenated pyramid of each (b, h): tokens have ids
+ *    0..N-1; cell j of level l >= 1 has id N + off_l + j with off_l = sum_{l'=1}^{l-1} N/p^l'.
+ *    Levels 1..L-1 are stored in one [B, H, R, d] tensor per X in Q, K, V, level 1 first.
+ *  - Numerics follow SPEC.md: fp32 accumulation everywhere, scores in a fixed fp32 order so
+ *    the selection is reproducible bit for bit, one rounding to the storage dtype.
+ */
+#ifndef LIGHTHOUSE_LH_H
+#define LIGHTHOUSE_LH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LH_OK = 0,
+  LH_ERR_INVALID_ARG = 1,  /* bad shape, null or misaligned pointer */
+  LH_ERR_UNSUPPORTED = 2,  /* valid for the method but not for this GPU path (e.g. d not 64/128) */
+  LH_ERR_WORKSPACE = 3,    /* workspace too small */
+  LH_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  LH_ERR_DEVICE = 5        /* a kernel reported a fault through the workspace status word */
+} lh_status;
+
+typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
+
+/* One layer call. Names follow the pages: N tokens, H heads, d = d_head, pooling factor p,
+ * L levels, S = subsequence length (the top-K budget plus the kept coarsest cells).
+ * The softmax scale is fixed to 1/sqrt(d). */
+typedef struct {
+  int B, H, N, d, p, L, S;
+  int dtype; /* lh_dtype */
+} lh_shape;
+
+/* Sizes derived from a shape (SPEC.md section 0). */
+typedef struct {
+  int64_t R;  /* pooled rows per (b,h): sum_{l=1}^{L-1} N/p^l */
+  int64_t C;  /* chunks = coarsest cells = N/p^(L-1) */
+  int64_t T;  /* tokens per chunk = p^(L-1) */
+  int64_t m;  /* subsequence rows per chunk = S/C */
+  int64_t k;  /* selected entries per chunk besides the coarsest cell = m-1 */
+  int64_t M;  /* candidates per chunk = sum_{l=0}^{L-2} p^(L-1-l) */
+} lh_sizes;
+
+const char* lh_status_string(int status);
+const char* lh_version(void);
+
+/* Validates a shape for the GPU path and fills `out` (may be NULL).
+ * Method constraints: N % p^(L-1) == 0, S % C == 0, 1 <= S/C <= M+1.
+ * GPU constraints: d in {64, 128}, 2 <= p <= 16, L <= 12, p^(L-1) <= 2^20, B*H <= 65535*... */
+int lh_validate(const lh_shape* shape, lh_sizes* out);
+
+/* Bytes of the workspace `ws` that the entry points below take. The first 256 bytes hold the
+ * device status word; clear them once (lh_workspace_init) before first use. */
+size_t lh_workspace_bytes(const lh_shape* shape);
+/* Bytes of the forward-to-backward context `saved` of lh_layer_fwd / lh_layer_bwd. */
+size_t lh_saved_bytes(const lh_shape* shape);
+
+/* Clears the status word of `ws` (stream-ordered). */
+int lh_workspace_init(void* ws, void* stream);
+/* Synchronises `stream`, reads and clears the status word of `ws`.
+ * Returns LH_OK or LH_ERR_DEVICE (then *flags, if non-NULL, holds the fault bits:
+ * 1 = row id out of range, 2 = bounded wait ran out). */
+int lh_check(void* ws, void* stream, uint32_t* flags);
+
+/* Step 1+2 (pyramid, section 2.A; scores, section 2.B). Reads q, k, v [B,H,N,d]; writes the
+ * pooled levels pq, pk, pv [B,H,R,d]. If `score` is non-NULL it also writes the rank score
+ * r = max-pooled |q| + max-pooled |k| for every row id, float [B,H,N+R], in the same pass.
+ * pq/pk/pv may all be NULL to compute only the score (then v is not read). */
+int lh_build_pyramid(const lh_shape* shape, const void* q, const void* k, const void* v,
+                     void* pq, void* pk, void* pv, float* score, void* ws, void* stream);
+
+/* Step 2 alone: the rank score float [B,H,N+R] from q, k [B,H,N,d]. */
+int lh_score(const lh_shape* shape, const void* q, const void* k, float* score, void* ws,
+             void* stream);
+
+/* Step 3 (stratified top-K, section 2.B and the article's four-stage paragraph). Per (b,h) and
+ * chunk: keep the coarsest cell and the k best candidates by (r desc, level desc, position asc);
+ * write their row ids in causal order (end asc, then level asc) to idx int32 [B,H,S]. */
+int lh_select_topk(const lh_shape* shape, const float* score, int32_t* idx, void* stream);
+
+/* Step 4 (gather, section 2.C). x_sub[b,h,i] = row idx[b,h,i] of [x | px]. Any idx whose ids
+ * are in range is accepted; out-of-range ids give zero rows and set status bit 1. */
+int lh_gather(const lh_shape* shape, const void* q, const void* k, const void* v,
+              const void* pq, const void* pk, const void* pv, const int32_t* idx,
+              void* q_sub, void* k_sub, void* v_sub, void* ws, void* stream);
+
+/* Step 5 (dense causal attention on the subsequence, section 2.C). Row j is visible to row i
+ * iff j <= i. Writes o_sub [B,H,S,d] and lse float [B,H,S] (natural log). */
+int lh_attn_fwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
+                void* o_sub, float* lse, void* ws, void* stream);
+
+/* Backward of step 5. do_sub is [B,H,S,d] in shape.dtype; dq_sub, dk_sub, dv_sub are float
+ * [B,H,S,d]. Uses the workspace for D_i = do_sub[i] . o_sub[i]. */
+int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
+                const void* o_sub, const float* lse, const void* do_sub, float* dq_sub,
+                float* dk_sub, float* dv_sub, void* ws, void* stream);
+
+/* Step 6 (deterministic scatter-back, section 2.C). o[t] = sum of o_sub[i] over the rows i of
+ * t's chunk whose span covers t, added in ascending i, no atomics. idx must be a valid
+ * selection (causal order, coarsest cell last in each chunk). */
+int lh_scatter(const lh_shape* shape, const int32_t* idx, const void* o_sub, void* o,
+               void* stream);
+
+/* Backward of step 6: do_sub[i] = sum of d_o over the tokens of span(i). */
+int lh_scatter_bwd(const lh_shape* shape, const int32_t* idx, const void* d_o, void* do_sub,
+                   void* ws, void* stream);
+
+/* Backward of steps 1+4: dx[t] = sum over rows i covering t of dx_sub[i] / p^level(i), for
+ * x in q, k, v. dx_sub are float [B,H,S,d]; dq, dk, dv are [B,H,N,d] in shape.dtype. */
+int lh_gather_bwd(const lh_shape* shape, const int32_t* idx, const float* dq_sub,
+                  const float* dk_sub, const float* dv_sub, void* dq, void* dk, void* dv,
+                  void* stream);
+
+/* The whole layer forward: steps 1-6. Writes o [B,H,N,d] and the context `saved`
+ * (lh_saved_bytes) that lh_layer_bwd reads: idx, q_sub, k_sub, v_sub, o_sub, lse. */
+int lh_layer_fwd(const lh_shape* shape, const void* q, const void* k, const void* v, void* o,
+                 void* saved, void* ws, void* stream);
+
+/* The whole layer backward. Reads `saved` from lh_layer_fwd and d_o [B,H,N,d]; writes
+ * dq, dk, dv [B,H,N,d]. */
+int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void* dq, void* dk,
+                 void* dv, void* ws, void* stream);
+
+/* Number of kernel launches one lh_layer_fwd (*fwd) and one lh_layer_bwd (*bwd) make for this
+ * shape (either pointer may be NULL). Host-side plan only; launches nothing. */
+int lh_launches(const lh_shape* shape, int* fwd, int* bwd);
+
+/* Offsets (bytes) of the tensors inside `saved`, so that callers can read them:
+ * idx, q_sub, k_sub, v_sub, o_sub, lse, in that order. */
+int lh_saved_offsets(const lh_shape* shape, size_t offsets[6]);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIGHTHOUSE_LH_H */

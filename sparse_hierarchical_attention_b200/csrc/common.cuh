@@ -1,0 +1,97 @@
+// Shared device helpers and the internal launch interface of the Lighthouse library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lh.h"
+
+namespace lh {
+
+constexpr uint32_t kFaultIndex = 1u;    // a row id outside [0, N+R)
+constexpr uint32_t kFaultTimeout = 2u;  // a bounded wait ran out
+
+// Sizes derived from one layer shape (SPEC section 0), computed on the host.
+struct Geo {
+  int B, H, N, d, p, L, S, dtype;
+  int64_t BH, R, C, T, m, k, M;
+  int64_t nlev[16];  // N_l = N / p^l
+  int64_t off[16];   // row id of the first cell of level l (off[0] = 0, off[1] = N, ...)
+  int64_t cand_off[16];  // offset of level l inside a chunk's candidate list (levels 0..L-2)
+  int esize;          // bytes per element of the storage dtype
+};
+
+// Raw element <-> fp32 helpers. Loads and stores move 16 bytes per thread.
+template <typename E> struct Vec;
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static inline void unpack(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+  __device__ static inline uint4 pack(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static inline void unpack(const uint4& u, float* f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static inline uint4 pack(const float* f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+__device__ inline float to_f32(float x) { return x; }
+__device__ inline float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename E> __device__ inline E from_f32(float x);
+template <> __device__ inline float from_f32<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ inline uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+__device__ inline void stg16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+__device__ inline void raise_fault(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ---- internal launchers (one per kernel family); all return cudaError_t of the launch ----
+cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,
+                           void* pk, void* pv, float* score, void* tmp, cudaStream_t st);
+size_t pyramid_tmp_bytes(const Geo& g);
+int pool_launches(const Geo& g);  // 1 or 2: the tile kernel, plus the coarse kernel if needed
+cudaError_t launch_select(const Geo& g, const float* score, int32_t* idx, cudaStream_t st);
+cudaError_t launch_gather(const Geo& g, const void* q, const void* k, const void* v,
+                          const void* pq, const void* pk, const void* pv, const int32_t* idx,
+                          void* qs, void* ks, void* vs, uint32_t* status, cudaStream_t st);
+cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool from_f32,
+                          bool scale_by_level, const void* const* src, void* const* dst,
+                          uint32_t* status, cudaStream_t st);
+cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, void* do_sub,
+                            void* tmp, uint32_t* status, cudaStream_t st);
+size_t span_sum_tmp_bytes(const Geo& g);
+int attn_fwd_launches(const Geo& g);
+int attn_bwd_launches(const Geo& g);
+cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
+                                 void* os, float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
+                                 const void* os, const float* lse, const void* dos, float* dq,
+                                 float* dk, float* dv, float* delta, cudaStream_t st);
+
+}  // namespace lh

@@ -1,0 +1,173 @@
+// Gather of the selected triples and the deterministic scatter-back ("Long Context Pre-Training
+// with Lighthouse Attention", technical summary 2.C), and the backward of the gather through
+// the pooling (technical summary 2.B: gradients reach Q, K, V through the gather).
+//
+// gather: one 16-byte lane per column slice, rows independent, a pure copy.
+// spread: one CTA per (b,h, chunk). The chunk's m row ids become a shared-memory map
+//   (level, cell in chunk) -> subsequence row. Each token then adds the rows that cover it,
+//   one per level at most, in ascending level order, which is ascending subsequence order for
+//   nested spans (SPEC sections 4, 6, 7). fp32 accumulation, one rounding, no atomics.
+#include "common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kThreads)
+gather_kernel(const E* __restrict__ q, const E* __restrict__ k, const E* __restrict__ v,
+              const E* __restrict__ pq, const E* __restrict__ pk, const E* __restrict__ pv,
+              const int32_t* __restrict__ idx, E* qs, E* ks, E* vs, int64_t BH, int64_t N,
+              int64_t R, int64_t S, uint32_t* status) {
+  constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, RPC = kThreads / LPR;
+  const int col = threadIdx.x % LPR;
+  const int64_t row = (int64_t)blockIdx.x * RPC + threadIdx.x / LPR;  // over BH*S
+  if (row >= BH * S) return;
+  const int64_t bh = row / S;
+  const int64_t rid = idx[row];
+  const E* src[3];
+  E* dst[3] = {qs, ks, vs};
+  bool ok = rid >= 0 && rid < N + R;
+  if (!ok) {
+    if (col == 0) raise_fault(status, kFaultIndex);
+  } else if (rid < N) {
+    src[0] = q + (bh * N + rid) * D; src[1] = k + (bh * N + rid) * D; src[2] = v + (bh * N + rid) * D;
+  } else {
+    const int64_t pr = bh * R + (rid - N);
+    src[0] = pq + pr * D; src[1] = pk + pr * D; src[2] = pv + pr * D;
+  }
+#pragma unroll
+  for (int xi = 0; xi < 3; ++xi) {
+    const uint4 u = ok ? ldg16(src[xi] + col * VEC) : make_uint4(0, 0, 0, 0);
+    stg16(dst[xi] + row * D + col * VEC, u);
+  }
+}
+
+struct SpreadArgs {
+  const void* src[3];
+  void* dst[3];
+  const int32_t* idx;
+  uint32_t* status;
+  int64_t N, R, S, T, m;
+  int64_t off[16];
+  float inv[16];  // per-level weight: 1 (scatter) or fl32(1/p^l) (gather backward)
+  int p, L, ntensor;
+};
+
+template <typename E, typename SRC, int D>
+__global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
+  constexpr int VEC = 16 / sizeof(E), LPR = D / VEC;
+  extern __shared__ int cmap[];  // (level, cell in chunk) -> subsequence row of this (b,h)
+  const int tid = threadIdx.x;
+  const int64_t bh = blockIdx.y, c = blockIdx.x;
+  const int L = a.L, p = a.p;
+
+  int base[16], per[16];
+  int tot = 0;
+  {
+    int cells = 1;
+    for (int l = L - 1; l >= 0; --l) { per[l] = cells; cells *= p; }
+    for (int l = 0; l < L; ++l) { base[l] = tot; tot += per[l]; }
+  }
+  for (int i = tid; i < tot; i += kThreads) cmap[i] = -1;
+  __syncthreads();
+  for (int64_t i = c * a.m + tid; i < (c + 1) * a.m; i += kThreads) {
+    const int64_t rid = a.idx[bh * a.S + i];
+    int lvl = 0;
+    if (rid < 0 || rid >= a.N + a.R) { raise_fault(a.status, kFaultIndex); continue; }
+    for (int l = 1; l < L; ++l)
+      if (rid >= a.off[l]) lvl = l;
+    const int64_t local = rid - a.off[lvl] - c * per[lvl];
+    if (local < 0 || local >= per[lvl]) { raise_fault(a.status, kFaultIndex); continue; }
+    cmap[base[lvl] + (int)local] = (int)i;
+  }
+  __syncthreads();
+
+  const int64_t items = a.T * LPR;
+  for (int64_t it = tid; it < items; it += kThreads) {
+    const int tl = (int)(it / LPR), col = (int)(it % LPR);
+    for (int xi = 0; xi < a.ntensor; ++xi) {
+      const SRC* src = static_cast<const SRC*>(a.src[xi]) + bh * a.S * D + col * VEC;
+      float acc[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+      int cell = tl;
+      for (int l = 0; l < L; ++l) {
+        const int r = cmap[base[l] + cell];
+        if (r >= 0) {
+          float x[VEC];
+          if constexpr (sizeof(SRC) == sizeof(E)) {
+            Vec<E>::unpack(ldg16(src + (int64_t)r * D), x);
+          } else {  // fp32 source, VEC elements = VEC/4 16-byte loads
+#pragma unroll
+            for (int h = 0; h < VEC / 4; ++h) Vec<float>::unpack(ldg16(src + (int64_t)r * D + 4 * h), x + 4 * h);
+          }
+          const float w = a.inv[l];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] = __fadd_rn(acc[e], __fmul_rn(x[e], w));
+        }
+        cell /= p;
+      }
+      E* dst = static_cast<E*>(a.dst[xi]) + (bh * a.N + c * a.T + tl) * D + col * VEC;
+      stg16(dst, Vec<E>::pack(acc));
+    }
+  }
+}
+
+template <typename E, typename SRC>
+cudaError_t run_spread(const Geo& g, const SpreadArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)(g.M + 1) * sizeof(int);
+  dim3 grid((unsigned)g.C, (unsigned)g.BH);
+  cudaError_t e;
+  if (g.d == 64) {
+    e = cudaFuncSetAttribute(spread_kernel<E, SRC, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) spread_kernel<E, SRC, 64><<<grid, kThreads, smem, st>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(spread_kernel<E, SRC, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) spread_kernel<E, SRC, 128><<<grid, kThreads, smem, st>>>(a);
+  }
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const Geo& g, const void* q, const void* k, const void* v,
+                          const void* pq, const void* pk, const void* pv, const int32_t* idx,
+                          void* qs, void* ks, void* vs, uint32_t* status, cudaStream_t st) {
+  const int vec = 16 / g.esize, lpr = g.d / vec, rpc = kThreads / lpr;
+  const int64_t rows = g.BH * g.S;
+  const unsigned grid = (unsigned)((rows + rpc - 1) / rpc);
+#define LH_GATHER(E, D)                                                                      \
+  gather_kernel<E, D><<<grid, kThreads, 0, st>>>(                                            \
+      (const E*)q, (const E*)k, (const E*)v, (const E*)pq, (const E*)pk, (const E*)pv, idx, \
+      (E*)qs, (E*)ks, (E*)vs, g.BH, g.N, g.R, g.S, status)
+  if (g.dtype == LH_BF16) {
+    if (g.d == 64) LH_GATHER(__nv_bfloat16, 64); else LH_GATHER(__nv_bfloat16, 128);
+  } else {
+    if (g.d == 64) LH_GATHER(float, 64); else LH_GATHER(float, 128);
+  }
+#undef LH_GATHER
+  return cudaGetLastError();
+}
+
+cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool src_f32,
+                          bool scale_by_level, const void* const* src, void* const* dst,
+                          uint32_t* status, cudaStream_t st) {
+  SpreadArgs a{};
+  for (int i = 0; i < ntensor; ++i) { a.src[i] = src[i]; a.dst[i] = dst[i]; }
+  a.idx = idx; a.status = status;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m;
+  a.p = g.p; a.L = g.L; a.ntensor = ntensor;
+  for (int l = 0; l < 16; ++l) {
+    a.off[l] = l < g.L ? g.off[l] : 0;
+    double pw = 1.0;
+    for (int q = 0; q < l; ++q) pw *= g.p;
+    a.inv[l] = scale_by_level ? (float)(1.0 / pw) : 1.0f;
+  }
+  if (g.dtype == LH_BF16)
+    return src_f32 ? run_spread<__nv_bfloat16, float>(g, a, st) : run_spread<__nv_bfloat16, __nv_bfloat16>(g, a, st);
+  return run_spread<float, float>(g, a, st);
+}
+
+}  // namespace lh

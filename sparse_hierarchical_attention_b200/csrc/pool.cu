@@ -1,0 +1,493 @@
+// Streaming pooling kernels.
+//
+// MODE_PYRAMID: the symmetric average-pooling pyramid over Q, K, V and the l2 rank score of
+//   every cell, in one pass over the inputs ("Long Context Pre-Training with Lighthouse
+//   Attention", technical summary 2.A and 2.B; the Nous Research article's four-stage
+//   paragraph: Theta(N) pyramid, two scalar scores per cell, max-pooled upward).
+// MODE_SPANSUM: dO_sub[i] = sum of dO over span(i) for the selected cells only, the backward
+//   of the scatter-back (technical summary 2.B: gradients flow through scatter-back).
+//
+// Structure (per (b,h)):
+//   tile kernel  - 256 threads; each row of d elements is covered by LPR lanes holding 16 bytes
+//                  each. A "stream" (LPR lanes) walks W = p^A consecutive tokens and keeps fp32
+//                  partial sums of levels 1..A in registers. The STREAMS level-A cells of the
+//                  CTA then go through a shared-memory tree up to level A2. If A2 < L-1 the
+//                  level-A2 fp32 sums (and score maxima) go to a small scratch buffer.
+//   coarse kernel - one CTA per chunk finishes levels A2+1..L-1 from that scratch.
+// Sums are fp32 in ascending child order, never re-read from rounded storage (SPEC section 1);
+// norms follow the fixed fp32 order of SPEC section 2 (16-byte groups, halving tree).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kThreads = 256;
+enum { MODE_PYRAMID = 0, MODE_SPANSUM = 1 };
+
+struct PoolArgs {
+  const void* x[3];  // q, k, v (pyramid) or d_o (span sums)
+  void* px[3];       // pooled outputs [BH, R, D] (pyramid) or do_sub [BH, S, D] (span sums)
+  float* score;      // [BH, N+R] or null
+  float* tmp;        // level-A2 fp32 sums [BH, N/p^A2, ntensor, D] then maxima [BH, N/p^A2, 2]
+  const int32_t* idx;  // span sums: the selection [BH, S]
+  uint32_t* status;
+  int64_t N, R, S, T, m, C;
+  int64_t off[16];    // row id offsets of levels
+  float inv[16];      // fl32(1 / p^l)
+  int p, L, W, A2, U;
+  int do_pyr, do_score;
+};
+
+// fp32 l2 norm in the SPEC section 2 order: each lane sums the squares of its 16-byte group in
+// ascending order (products rounded on their own), then a butterfly over the LPR lanes of the
+// row realises the halving tree (lane i pairs with i+s for s = LPR/2 .. 1).
+template <int VEC, int LPR>
+__device__ inline float row_norm(const float* x) {
+  float a = 0.f;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) a = __fadd_rn(a, __fmul_rn(x[e], x[e]));
+#pragma unroll
+  for (int s = LPR / 2; s >= 1; s >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, s));
+  return __fsqrt_rn(a);
+}
+
+// Row id -> level and cell index, from the level offsets.
+__device__ inline void decode_rid(int64_t rid, const int64_t* off, int L, int& lvl, int64_t& cell) {
+  lvl = 0;
+#pragma unroll 1
+  for (int l = 1; l < L; ++l)
+    if (rid >= off[l]) lvl = l;
+  cell = rid - off[lvl];
+}
+
+template <typename E, int D, int A, int MODE>
+__global__ void __launch_bounds__(kThreads) pool_tile_kernel(const PoolArgs a) {
+  using V = Vec<E>;
+  constexpr int VEC = V::N, LPR = D / VEC, STREAMS = kThreads / LPR;
+  constexpr int NX = MODE == MODE_PYRAMID ? 3 : 1;
+  constexpr int AR = A > 0 ? A : 1;
+  __shared__ float stage[NX][STREAMS][D];
+  __shared__ float smax[2][STREAMS];
+  __shared__ int smap[MODE == MODE_SPANSUM ? 2 * STREAMS * 16 + 64 : 1];  // (level, cell) -> row
+
+  const int tid = threadIdx.x, col = tid % LPR, s = tid / LPR;
+  const int64_t bh = blockIdx.y;
+  const int W = a.W, p = a.p;
+  const int64_t tile = (int64_t)W * STREAMS;
+  const int64_t t_tile = (int64_t)blockIdx.x * tile;
+  const int64_t tok0 = t_tile + (int64_t)s * W;
+  const bool active = tok0 < a.N;
+  const int nx = MODE == MODE_PYRAMID ? (a.do_pyr ? 3 : 2) : 1;
+  const int64_t NR = a.N + a.R;
+
+  // Span sums: map every selected cell of level <= A2 inside this tile to its subsequence row.
+  // Map layout: level l occupies tile/p^l slots starting at moff(l).
+  int map_base[16];
+  if constexpr (MODE == MODE_SPANSUM) {
+    int acc = 0;
+    int64_t cells = tile;
+    for (int l = 0; l <= a.A2; ++l) {
+      map_base[l] = acc;
+      acc += (int)cells;
+      cells /= p;
+    }
+    for (int i = tid; i < acc; i += kThreads) smap[i] = -1;
+    __syncthreads();
+    const int64_t c0 = t_tile / a.T;
+    const int64_t c1 = std::min<int64_t>((t_tile + tile - 1) / a.T, a.C - 1);
+    const int64_t r0 = c0 * a.m, r1 = (c1 + 1) * a.m;
+    for (int64_t i = r0 + tid; i < r1; i += kThreads) {
+      const int64_t rid = a.idx[bh * a.S + i];
+      if (rid < 0 || rid >= NR) { raise_fault(a.status, kFaultIndex); continue; }
+      int lvl; int64_t cell;
+      decode_rid(rid, a.off, a.L, lvl, cell);
+      if (lvl > a.A2) continue;
+      int64_t pw = 1;
+      for (int l = 0; l < lvl; ++l) pw *= p;
+      const int64_t first = t_tile / pw;  // first cell of this level inside the tile
+      if (cell >= first && cell < first + tile / pw)
+        smap[map_base[lvl] + (int)(cell - first)] = (int)i;
+    }
+    __syncthreads();
+  }
+
+  float acc[NX][AR][VEC];
+  float mq[AR], mk[AR];
+#pragma unroll
+  for (int l = 0; l < AR; ++l) {
+    mq[l] = 0.f; mk[l] = 0.f;
+#pragma unroll
+    for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[xi][l][e] = 0.f;
+  }
+
+  // Stores one finished cell (level l, global cell j) from registers.
+  auto store_cell = [&](int l, int64_t j, float (*src)[VEC], float sq, float sk) {
+    if constexpr (MODE == MODE_PYRAMID) {
+      if (a.do_pyr) {
+        const int64_t row = bh * a.R + (a.off[l] - a.N) + j;
+#pragma unroll
+        for (int xi = 0; xi < NX; ++xi) {
+          float o[VEC];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) o[e] = __fmul_rn(src[xi][e], a.inv[l]);
+          stg16(static_cast<E*>(a.px[xi]) + row * D + col * VEC, V::pack(o));
+        }
+      }
+      if (a.do_score && col == 0) a.score[bh * NR + a.off[l] + j] = __fadd_rn(sq, sk);
+    } else {
+      const int64_t first = t_tile;
+      int64_t pw = 1;
+      for (int q = 0; q < l; ++q) pw *= p;
+      const int r = smap[map_base[l] + (int)(j - first / pw)];
+      if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(src[0]));
+    }
+  };
+
+  const E* X[NX];
+#pragma unroll
+  for (int xi = 0; xi < NX; ++xi) X[xi] = static_cast<const E*>(a.x[xi]);
+
+#pragma unroll 1
+  for (int row = 0; row < W; ++row) {
+    const int64_t t = tok0 + row;
+    float x[NX][VEC];
+#pragma unroll
+    for (int xi = 0; xi < NX; ++xi) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (active && xi < nx) u = ldg16(X[xi] + (bh * a.N + t) * D + col * VEC);
+      V::unpack(u, x[xi]);
+    }
+    float nq = 0.f, nk = 0.f;
+    if (MODE == MODE_PYRAMID && a.do_score) {
+      nq = row_norm<VEC, LPR>(x[0]);
+      nk = row_norm<VEC, LPR>(x[1]);
+      if (active && col == 0) a.score[bh * NR + t] = __fadd_rn(nq, nk);
+    }
+    if constexpr (MODE == MODE_SPANSUM) {
+      if (active) {
+        const int r = smap[(int)(t - t_tile)];
+        if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(x[0]));
+      }
+    }
+    if constexpr (A > 0) {
+#pragma unroll
+      for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[xi][0][e] += x[xi][e];
+      mq[0] = fmaxf(mq[0], nq);
+      mk[0] = fmaxf(mk[0], nk);
+      int pw = 1;
+#pragma unroll
+      for (int l = 1; l <= A; ++l) {
+        pw *= p;
+        if ((row + 1) % pw != 0) break;
+        float cur[NX][VEC];
+#pragma unroll
+        for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) cur[xi][e] = acc[xi][l - 1][e];
+        if (active) store_cell(l, (t + 1) / pw - 1, cur, mq[l - 1], mk[l - 1]);
+        if (l < A) {
+#pragma unroll
+          for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[xi][l < A ? l : 0][e] += cur[xi][e];
+          mq[l < A ? l : 0] = fmaxf(mq[l < A ? l : 0], mq[l - 1]);
+          mk[l < A ? l : 0] = fmaxf(mk[l < A ? l : 0], mk[l - 1]);
+        } else {
+#pragma unroll
+          for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = cur[xi][e];
+          if (col == 0) { smax[0][s] = mq[l - 1]; smax[1][s] = mk[l - 1]; }
+        }
+#pragma unroll
+        for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[xi][l - 1][e] = 0.f;
+        mq[l - 1] = 0.f;
+        mk[l - 1] = 0.f;
+      }
+    }
+  }
+  if (A == 0 || (a.U == 0 && a.A2 >= a.L - 1)) return;
+  __syncthreads();
+
+  // Shared-memory tree: levels A+1..A2 from the STREAMS level-A cells of this tile.
+  int cells = STREAMS;
+  int64_t pw = W;  // p^level of the current stage
+  for (int u = 1; u <= a.U; ++u) {
+    const int lvl = A + u;
+    const int nc = cells / p;
+    pw *= p;
+    const int nitems = NX * nc * D;
+    float v[(NX * STREAMS * D + kThreads - 1) / kThreads];
+    float vmax[2] = {0.f, 0.f};
+    int n = 0;
+    for (int it = tid; it < nitems; it += kThreads, ++n) {
+      const int xi = it / (nc * D), rem = it % (nc * D), c = rem / D, dd = rem % D;
+      float sum = 0.f;
+      for (int ch = 0; ch < p; ++ch) sum += stage[xi][c * p + ch][dd];
+      v[n] = sum;
+    }
+    if (tid < nc) {
+      for (int ch = 0; ch < p; ++ch) {
+        vmax[0] = fmaxf(vmax[0], smax[0][tid * p + ch]);
+        vmax[1] = fmaxf(vmax[1], smax[1][tid * p + ch]);
+      }
+    }
+    __syncthreads();
+    n = 0;
+    for (int it = tid; it < nitems; it += kThreads, ++n) {
+      const int xi = it / (nc * D), rem = it % (nc * D), c = rem / D, dd = rem % D;
+      stage[xi][c][dd] = v[n];
+      const int64_t j = t_tile / pw + c;
+      if (j * pw < a.N) {
+        if constexpr (MODE == MODE_PYRAMID) {
+          if (a.do_pyr)
+            static_cast<E*>(a.px[xi])[(bh * a.R + (a.off[lvl] - a.N) + j) * D + dd] =
+                from_f32<E>(__fmul_rn(v[n], a.inv[lvl]));
+        } else {
+          const int r = smap[map_base[lvl] + c];
+          if (r >= 0) static_cast<E*>(a.px[0])[(bh * a.S + r) * D + dd] = from_f32<E>(v[n]);
+        }
+      }
+    }
+    if (tid < nc) {
+      smax[0][tid] = vmax[0];
+      smax[1][tid] = vmax[1];
+      const int64_t j = t_tile / pw + tid;
+      if (MODE == MODE_PYRAMID && a.do_score && j * pw < a.N)
+        a.score[bh * NR + a.off[lvl] + j] = __fadd_rn(vmax[0], vmax[1]);
+    }
+    __syncthreads();
+    cells = nc;
+  }
+
+  // Hand the level-A2 sums to the coarse kernel.
+  if (a.A2 < a.L - 1) {
+    const int64_t n_a2 = a.N / pw;  // cells of level A2 per (b,h)
+    for (int it = tid; it < NX * cells * D; it += kThreads) {
+      const int xi = it / (cells * D), rem = it % (cells * D), c = rem / D, dd = rem % D;
+      const int64_t j = t_tile / pw + c;
+      if (j < n_a2) a.tmp[((bh * n_a2 + j) * NX + xi) * D + dd] = stage[xi][c][dd];
+    }
+    if (tid < cells) {
+      const int64_t j = t_tile / pw + tid;
+      float* mx = a.tmp + (int64_t)gridDim.y * n_a2 * NX * D;
+      if (j < n_a2) {
+        mx[(bh * n_a2 + j) * 2 + 0] = smax[0][tid];
+        mx[(bh * n_a2 + j) * 2 + 1] = smax[1][tid];
+      }
+    }
+  }
+}
+
+// Levels A2+1..L-1 of one chunk from the level-A2 fp32 sums. Thread (xi, dd) walks the
+// chunk's level-A2 cells in order with one partial sum per coarser level.
+template <typename E, int MODE>
+__global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
+  const int64_t bh = blockIdx.y, chunk = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int p = a.p;
+  const int nlev = a.L - 1 - a.A2;  // levels to build here
+  int64_t pw_a2 = 1;
+  for (int l = 0; l < a.A2; ++l) pw_a2 *= p;
+  const int64_t n_a2 = a.N / pw_a2;
+  int64_t ncell = 1;
+  for (int l = 0; l < nlev; ++l) ncell *= p;  // level-A2 cells per chunk
+  const int64_t first = chunk * ncell;
+
+  // Span sums: (level above A2, cell inside the chunk) -> subsequence row, or -1.
+  extern __shared__ int cmap[];
+  int cbase[16];
+  if constexpr (MODE == MODE_SPANSUM) {
+    int tot = 0;
+    int64_t per = ncell;
+    for (int u = 0; u < nlev; ++u) {
+      per /= p;
+      cbase[u] = tot;
+      tot += (int)per;
+    }
+    for (int i = tid; i < tot; i += blockDim.x) cmap[i] = -1;
+    __syncthreads();
+    for (int64_t i = chunk * a.m + tid; i < (chunk + 1) * a.m; i += blockDim.x) {
+      const int64_t rid = a.idx[bh * a.S + i];
+      if (rid < 0 || rid >= a.N + a.R) { raise_fault(a.status, kFaultIndex); continue; }
+      int lvl; int64_t cell;
+      decode_rid(rid, a.off, a.L, lvl, cell);
+      if (lvl <= a.A2) continue;
+      const int u = lvl - a.A2 - 1;
+      int64_t cells_per_chunk = 1;
+      for (int q = lvl; q < a.L - 1; ++q) cells_per_chunk *= p;
+      const int64_t local = cell - chunk * cells_per_chunk;
+      if (local >= 0 && local < cells_per_chunk) cmap[cbase[u] + (int)local] = (int)i;
+    }
+    __syncthreads();
+  }
+
+  if (tid < NX * D) {
+    const int xi = tid / D, dd = tid % D;
+    float acc[16];
+    for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+    for (int64_t c = 0; c < ncell; ++c) {
+      acc[0] += a.tmp[((bh * n_a2 + first + c) * NX + xi) * D + dd];
+      int64_t pw = 1;
+      for (int u = 0; u < nlev; ++u) {
+        pw *= p;
+        if ((c + 1) % pw != 0) break;
+        const int lvl = a.A2 + 1 + u;
+        const int64_t j = (first + c + 1) / pw - 1;
+        if constexpr (MODE == MODE_PYRAMID) {
+          if (a.do_pyr)
+            static_cast<E*>(a.px[xi])[(bh * a.R + (a.off[lvl] - a.N) + j) * D + dd] =
+                from_f32<E>(__fmul_rn(acc[u], a.inv[lvl]));
+        } else {
+          int64_t cells_per_chunk = ncell / pw;
+          const int r = cmap[cbase[u] + (int)(j - chunk * cells_per_chunk)];
+          if (r >= 0) static_cast<E*>(a.px[0])[(bh * a.S + r) * D + dd] = from_f32<E>(acc[u]);
+        }
+        if (u + 1 < nlev) acc[u + 1] += acc[u];
+        acc[u] = 0.f;
+      }
+    }
+  }
+  if (MODE == MODE_PYRAMID && a.do_score && tid == 0) {
+    const float* mx = a.tmp + (int64_t)gridDim.y * n_a2 * NX * D;
+    float q[16], k[16];
+    for (int u = 0; u < 16; ++u) { q[u] = 0.f; k[u] = 0.f; }
+    for (int64_t c = 0; c < ncell; ++c) {
+      q[0] = fmaxf(q[0], mx[(bh * n_a2 + first + c) * 2 + 0]);
+      k[0] = fmaxf(k[0], mx[(bh * n_a2 + first + c) * 2 + 1]);
+      int64_t pw = 1;
+      for (int u = 0; u < nlev; ++u) {
+        pw *= p;
+        if ((c + 1) % pw != 0) break;
+        const int lvl = a.A2 + 1 + u;
+        const int64_t j = (first + c + 1) / pw - 1;
+        a.score[bh * (a.N + a.R) + a.off[lvl] + j] = __fadd_rn(q[u], k[u]);
+        if (u + 1 < nlev) { q[u + 1] = fmaxf(q[u + 1], q[u]); k[u + 1] = fmaxf(k[u + 1], k[u]); }
+        q[u] = 0.f; k[u] = 0.f;
+      }
+    }
+  }
+}
+
+// Register levels A for a pooling factor: the largest A <= min(L-1, 4) with p^A <= 16.
+int pick_A(int p, int L) {
+  int A = 0, pw = 1;
+  while (A < L - 1 && A < 4 && pw * p <= 16) { pw *= p; ++A; }
+  return A;
+}
+
+struct Plan {
+  int A, W, streams, U, A2;
+};
+
+Plan make_plan(const Geo& g) {
+  Plan pl;
+  pl.A = pick_A(g.p, g.L);
+  pl.W = 1;
+  for (int i = 0; i < pl.A; ++i) pl.W *= g.p;
+  const int vec = 16 / g.esize, lpr = g.d / vec;
+  pl.streams = kThreads / lpr;
+  pl.U = 0;
+  if (pl.A > 0) {
+    int sc = pl.streams;
+    while (pl.A + pl.U < g.L - 1 && sc % g.p == 0) { sc /= g.p; ++pl.U; }
+  }
+  pl.A2 = pl.A + pl.U;
+  return pl;
+}
+
+template <typename E, int D, int MODE>
+cudaError_t launch_tile(const Plan& pl, const PoolArgs& a, int64_t BH, cudaStream_t st) {
+  const int64_t tile = (int64_t)pl.W * pl.streams;
+  dim3 grid((unsigned)((a.N + tile - 1) / tile), (unsigned)BH);
+  switch (pl.A) {
+    case 0: pool_tile_kernel<E, D, 0, MODE><<<grid, kThreads, 0, st>>>(a); break;
+    case 1: pool_tile_kernel<E, D, 1, MODE><<<grid, kThreads, 0, st>>>(a); break;
+    case 2: pool_tile_kernel<E, D, 2, MODE><<<grid, kThreads, 0, st>>>(a); break;
+    case 3: pool_tile_kernel<E, D, 3, MODE><<<grid, kThreads, 0, st>>>(a); break;
+    default: pool_tile_kernel<E, D, 4, MODE><<<grid, kThreads, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
+  const Plan pl = make_plan(g);
+  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C;
+  a.p = g.p; a.L = g.L; a.W = pl.W; a.A2 = pl.A2; a.U = pl.U;
+  for (int l = 0; l < 16; ++l) {
+    a.off[l] = l < g.L ? g.off[l] : 0;
+    double pw = 1.0;
+    for (int q = 0; q < l; ++q) pw *= g.p;
+    a.inv[l] = l < g.L ? 1.0f / (float)pw : 0.f;
+  }
+  cudaError_t e;
+  const bool bf = g.dtype == LH_BF16;
+  if (g.d == 64)
+    e = bf ? launch_tile<__nv_bfloat16, 64, MODE>(pl, a, g.BH, st) : launch_tile<float, 64, MODE>(pl, a, g.BH, st);
+  else
+    e = bf ? launch_tile<__nv_bfloat16, 128, MODE>(pl, a, g.BH, st) : launch_tile<float, 128, MODE>(pl, a, g.BH, st);
+  if (e != cudaSuccess || pl.A2 >= g.L - 1) return e;
+  const int nx = MODE == MODE_PYRAMID ? 3 : 1;
+  dim3 grid((unsigned)g.C, (unsigned)g.BH);
+  const int threads = ((nx * g.d + 31) / 32) * 32;
+  // span sums: one map slot per cell of the levels above A2 inside a chunk
+  size_t smem = 0;
+  if (MODE == MODE_SPANSUM) {
+    int64_t per = 1, tot = 0;
+    for (int l = g.L - 1; l > pl.A2; --l) { tot += per; per *= g.p; }
+    smem = (size_t)tot * sizeof(int);
+  }
+  if (bf) pool_coarse_kernel<__nv_bfloat16, MODE><<<grid, threads, smem, st>>>(a, g.d, nx);
+  else pool_coarse_kernel<float, MODE><<<grid, threads, smem, st>>>(a, g.d, nx);
+  return cudaGetLastError();
+}
+
+size_t tmp_bytes(const Geo& g, int nx) {
+  const Plan pl = make_plan(g);
+  if (pl.A2 >= g.L - 1) return 0;
+  int64_t pw = 1;
+  for (int l = 0; l < pl.A2; ++l) pw *= g.p;
+  const int64_t n = g.BH * (g.N / pw);
+  return (size_t)(n * nx * g.d + n * 2) * sizeof(float);
+}
+
+}  // namespace
+
+size_t pyramid_tmp_bytes(const Geo& g) { return tmp_bytes(g, 3); }
+int pool_launches(const Geo& g) { return make_plan(g).A2 >= g.L - 1 ? 1 : 2; }
+size_t span_sum_tmp_bytes(const Geo& g) { return tmp_bytes(g, 1); }
+
+cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,
+                           void* pk, void* pv, float* score, void* tmp, cudaStream_t st) {
+  PoolArgs a{};
+  a.x[0] = q; a.x[1] = k; a.x[2] = v;
+  a.px[0] = pq; a.px[1] = pk; a.px[2] = pv;
+  a.score = score;
+  a.tmp = static_cast<float*>(tmp);
+  a.do_pyr = pq != nullptr;
+  a.do_score = score != nullptr;
+  return run_pool<MODE_PYRAMID>(g, a, st);
+}
+
+cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, void* do_sub,
+                            void* tmp, uint32_t* status, cudaStream_t st) {
+  PoolArgs a{};
+  a.x[0] = d_o;
+  a.px[0] = do_sub;
+  a.idx = idx;
+  a.status = status;
+  a.tmp = static_cast<float*>(tmp);
+  a.do_pyr = 1;
+  return run_pool<MODE_SPANSUM>(g, a, st);
+}
+
+}  // namespace lh

@@ -1,0 +1,161 @@
+// Stratified top-K ("Long Context Pre-Training with Lighthouse Attention", technical summary
+// 2.B: joint top-K over all levels; the Nous Research article's four-stage paragraph: the
+// selection is stratified and always keeps the coarsest level).
+//
+// One CTA per (b,h, chunk). The chunk's M candidate scores become 64-bit keys that encode the
+// total ranking order of SPEC section 3: high word = the fp32 score bits (scores are >= +0, so
+// the bit pattern orders like the value), then the level (higher wins), then the position
+// (lower wins). A most-significant-digit radix select (8-bit digits, shared-memory histograms,
+// one warp scanning the 256 bins) finds the k-th largest key; it stops as soon as the bucket
+// that holds the k-th key is taken whole. The k winners are then placed in causal order
+// (end, level) by counting, and the chunk's coarsest cell goes last.
+#include "common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kSelThreads = 256;
+
+struct SelArgs {
+  const float* score;
+  int32_t* idx;
+  int64_t N, R, S, m, k, M;
+  int64_t off[16];
+  int64_t cand_off[16];
+  int p, L;
+};
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
+  extern __shared__ unsigned long long keys[];  // [M] candidate keys, then [k] winners
+  __shared__ unsigned hist[256];
+  __shared__ int s_digit, s_need, s_cnt, s_nsel;
+
+  const int tid = threadIdx.x;
+  const int64_t bh = blockIdx.y, c = blockIdx.x;
+  const float* sc = a.score + bh * (a.N + a.R);
+  int32_t* out = a.idx + bh * a.S + c * a.m;
+  const int L = a.L, p = a.p;
+  const int M = (int)a.M, k = (int)a.k;
+
+  // 1. candidate keys: level l holds p^(L-1-l) cells per chunk
+  for (int l = 0; l < L - 1; ++l) {
+    int per = 1;
+    for (int q = l; q < L - 1; ++q) per *= p;
+    const int base = (int)a.cand_off[l];
+    for (int jl = tid; jl < per; jl += kSelThreads) {
+      const float r = sc[a.off[l] + c * per + jl];
+      const unsigned long long key = ((unsigned long long)__float_as_uint(r) << 32) |
+                                     ((unsigned long long)l << 24) | (unsigned)(0xFFFFFF - jl);
+      keys[base + jl] = key;
+    }
+  }
+  if (tid == 0) s_nsel = 0;
+  __syncthreads();
+
+  if (k > 0) {
+    // 2. radix select of the k-th largest key
+    unsigned long long prefix = 0, mask = 0;
+    int need = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (int q = tid; q < M; q += kSelThreads) {
+        const unsigned long long key = keys[q];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // lane l covers bins 255-8l .. 248-8l, taken from the top
+        unsigned cnt[8], tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { cnt[i] = hist[255 - 8 * tid - i]; tot += cnt[i]; }
+        unsigned incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
+        const int first = __ffs(ball) - 1;
+        if (ball == 0 && tid == 0) {  // cannot happen for a consistent histogram; stop safely
+          s_digit = 0; s_need = need; s_cnt = -1;
+        }
+        if (tid == first) {
+          unsigned cum = incl - tot;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (cum + cnt[i] >= (unsigned)need) {
+              s_digit = 255 - 8 * tid - i;
+              s_need = need - (int)cum;
+              s_cnt = (int)cnt[i];
+              break;
+            }
+            cum += cnt[i];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (unsigned long long)s_digit << shift;
+      mask |= 0xFFull << shift;
+      need = s_need;
+      const bool done = s_cnt == need || s_cnt < 0;
+      __syncthreads();
+      if (done) break;
+    }
+    // 3. winners: keys whose masked value is >= the prefix (exactly k of them)
+    unsigned long long* win = keys + M;
+    for (int q = tid; q < M; q += kSelThreads) {
+      const unsigned long long key = keys[q];
+      if ((key & mask) >= prefix) {
+        const int pos = atomicAdd(&s_nsel, 1);
+        if (pos < k) win[pos] = key;  // exactly k winners; the guard keeps shared memory safe
+      }
+    }
+    __syncthreads();
+    // 4. causal order: rank by (end, level) among the winners
+    const int nsel = s_nsel < k ? s_nsel : k;
+    for (int w = tid; w < nsel; w += kSelThreads) {
+      const unsigned long long key = win[w];
+      const int l = (int)((key >> 24) & 0xFF);
+      const int jl = 0xFFFFFF - (int)(key & 0xFFFFFF);
+      int64_t pw = 1;
+      for (int q = 0; q < l; ++q) pw *= p;
+      const int64_t ord = (((int64_t)jl + 1) * pw) * 16 + l;
+      int rank = 0;
+      for (int u = 0; u < nsel; ++u) {
+        const unsigned long long k2 = win[u];
+        const int l2 = (int)((k2 >> 24) & 0xFF);
+        const int j2 = 0xFFFFFF - (int)(k2 & 0xFFFFFF);
+        int64_t pw2 = 1;
+        for (int q = 0; q < l2; ++q) pw2 *= p;
+        rank += ((((int64_t)j2 + 1) * pw2) * 16 + l2) < ord;
+      }
+      int per = 1;
+      for (int q = l; q < L - 1; ++q) per *= p;
+      if (rank < a.m - 1) out[rank] = (int32_t)(a.off[l] + c * per + jl);
+    }
+  }
+  if (tid == 0) out[a.m - 1] = (int32_t)(a.off[L - 1] + c);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const Geo& g, const float* score, int32_t* idx, cudaStream_t st) {
+  SelArgs a{};
+  a.score = score; a.idx = idx;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.m = g.m; a.k = g.k; a.M = g.M;
+  a.p = g.p; a.L = g.L;
+  for (int l = 0; l < 16; ++l) {
+    a.off[l] = l < g.L ? g.off[l] : 0;
+    a.cand_off[l] = l < g.L ? g.cand_off[l] : 0;
+  }
+  const size_t smem = (size_t)(g.M + g.k) * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)g.C, (unsigned)g.BH);
+  select_kernel<<<grid, kSelThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace lh

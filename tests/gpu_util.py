@@ -1,0 +1,65 @@
+"""Helpers shared by the GPU parity tests: conversions and the acceptance rule of SPEC 9."""
+import numpy as np
+import torch
+
+import oracle as O
+
+
+def np64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def store_of(dtype):
+    return "bf16" if dtype == torch.bfloat16 else "f32"
+
+
+def assert_close(got, want, dtype, what="", mode="scaled"):
+    """The acceptance rule (SPEC section 9).
+
+    mode "literal": absolute error; max <= 2e-2, mean <= 2e-3 (bf16) or max <= 1e-4 (fp32).
+    mode "scaled": error / max(|oracle element|, RMS of the oracle tensor), same limits.
+    mode "tail": scaled error of a row-scaled workload: mean <= 2e-3, 99.9th percentile
+      <= 2e-2, max <= 0.25 (bf16; fp32 limits are 1/200 of these).
+    """
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    if got.size == 0:
+        return 0.0, 0.0
+    err = np.abs(got - want)
+    if mode in ("scaled", "tail"):
+        rms = float(np.sqrt(np.mean(want ** 2))) or 1.0
+        err = err / np.maximum(np.abs(want), rms)
+    mx, mean = float(err.max()), float(err.mean())
+    lim = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    msg = f"{what} ({mode}): max {mx:.3g} mean {mean:.3g}"
+    if mode == "tail":
+        q = float(np.quantile(err, 0.999))
+        assert mean <= lim / 10 and q <= lim and mx <= 12.5 * lim, msg + f" p99.9 {q:.3g}"
+    elif dtype == torch.bfloat16:
+        assert mx <= lim and mean <= lim / 10, msg
+    else:
+        assert mx <= lim, msg
+    return mx, mean
+
+
+def assert_pyramid(got, x, geo, dtype, what="pyramid"):
+    """Pooled cells against the exact span means, within a derived forward-error bound.
+
+    The GPU adds p children per level in fp32 (at most (p-1)(L-1) additions deep, each with
+    relative error 2^-24 of the running sum of |x|), scales by 1/p^l once, and rounds once to
+    the storage type (half an ulp: at most 2^-8 relative for bf16, 2^-24 for fp32).
+    """
+    want = O.build_pyramid(x, geo)
+    mean_abs = O.build_pyramid(np.abs(x), geo)
+    depth = max(1, (geo.p - 1) * (geo.L - 1) + 1)
+    half_ulp = 2.0 ** -8 if dtype == torch.bfloat16 else 2.0 ** -24  # unit roundoff
+    bound = 1.01 * (depth * 2.0 ** -24 * mean_abs + half_ulp * (np.abs(want) + depth * 2.0 ** -24 * mean_abs)) + 1e-30
+    bad = np.abs(np.asarray(got, np.float64) - want) > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} cells outside the bound"
+
+
+def g_of(dtype):
+    """Score group size of SPEC section 2: 16 bytes of the storage dtype."""
+    return 8 if dtype == torch.bfloat16 else 4

@@ -1,0 +1,82 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, validates shapes
+and sizes its buffers; invalid calls return errors before any launch."""
+import ctypes
+
+import pytest
+import torch
+
+import sparse_hierarchical_attention_b200 as lh
+from sparse_hierarchical_attention_b200 import Shape, _lib
+
+
+def test_every_declared_symbol_is_exported():
+    names = _lib.header_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(_lib._lib, n), n
+
+
+def test_version():
+    assert "sm_100a" in lh.lh_version()
+
+
+@pytest.mark.parametrize("N,p,L,S,want", [
+    (131072, 4, 6, 8192, dict(R=43648, C=128, T=1024, m=64, k=63, M=1364)),
+    (1048576, 4, 7, 16384, dict(R=349440, C=256, T=4096, m=64, k=63, M=5460)),
+    (98304, 4, 6, 6144, dict(R=32736, C=96, T=1024, m=64, k=63, M=1364)),
+    (2048, 4, 3, 512, dict(R=640, C=128, T=16, m=4, k=3, M=20)),
+    (640, 4, 1, 640, dict(R=0, C=640, T=1, m=1, k=0, M=0)),
+])
+def test_sizes(N, p, L, S, want):
+    assert lh.lh_validate(Shape(1, 2, N, 128, p, L, S)) == want
+
+
+@pytest.mark.parametrize("bad", [
+    Shape(1, 2, 1000, 128, 4, 6, 64),      # N not a multiple of p^(L-1)
+    Shape(1, 2, 4096, 128, 4, 6, 102),     # S not a multiple of C = 4
+    Shape(1, 2, 4096, 128, 4, 3, 256 * 22),  # m = 22 > M + 1 = 21
+    Shape(0, 2, 4096, 128, 4, 3, 256),     # empty batch
+    Shape(1, 2, 4096, 128, 1, 3, 256),     # p < 2
+])
+def test_invalid_shapes(bad):
+    assert _lib.lh_validate_status(bad) == 1
+    assert lh.lh_workspace_bytes(bad) == 0
+
+
+def test_unsupported_head_dim():
+    assert _lib.lh_validate_status(Shape(1, 2, 4096, 96, 4, 3, 256 * 4)) == 2
+
+
+def test_null_pointers_rejected_before_launch():
+    s = Shape(1, 2, 4096, 128, 4, 3, 1024).c()
+    rc = _lib._lib.lh_layer_fwd(ctypes.byref(s), None, None, None, None, None, None, None)
+    assert rc == 1
+    rc = _lib._lib.lh_select_topk(ctypes.byref(s), None, None, None)
+    assert rc == 1
+
+
+def test_misaligned_pointer_rejected_before_launch():
+    s = Shape(1, 2, 4096, 128, 4, 3, 1024).c()
+    p = ctypes.c_void_p(0x1000 + 4)
+    rc = _lib._lib.lh_select_topk(ctypes.byref(s), p, ctypes.c_void_p(0x2000), None)
+    assert rc == 1
+
+
+def test_workspace_and_saved_sizes_grow_with_shape():
+    a, b = Shape(1, 2, 4096, 128, 4, 3, 1024), Shape(1, 4, 4096, 128, 4, 3, 1024)
+    assert 0 < lh.lh_workspace_bytes(a) < lh.lh_workspace_bytes(b)
+    assert 0 < lh.lh_saved_bytes(a) < lh.lh_saved_bytes(b)
+    offs = lh.lh_saved_offsets(a)
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+
+
+def test_launch_plan():
+    f, b = lh.lh_launches(Shape(1, 32, 131072, 128, 4, 6, 8192))
+    assert f >= 5 and b >= 3
+
+
+def test_binding_refuses_host_tensors():
+    s = Shape(1, 1, 256, 64, 4, 3, 64)
+    x = torch.zeros(1, 1, 256 + 80, dtype=torch.float32)
+    with pytest.raises(lh.LighthouseError):
+        lh.lh_select_topk(s, x, torch.zeros(1, 1, 64, dtype=torch.int32))
