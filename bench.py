@@ -142,7 +142,7 @@ def stage_work(w, geo):
         "select": ("hbm", BH * (N + R) * 4 + BH * S * 4),
         "gather": ("hbm", 2 * 3 * BH * S * d * e + BH * S * 4),
         "attn_fwd": ("tensor", 2 * BH * S * S * d),
-        "scatter": ("hbm", BH * S * d * e + BH * N * d * e + BH * S * 4),
+        "scatter": ("hbm", BH * S * d * 4 + BH * N * d * e + BH * S * 4),
         "scatter_bwd": ("hbm", BH * N * d * e + BH * S * d * e + BH * S * 4),
         "attn_bwd": ("tensor", 5 * BH * S * S * d),
         "gather_bwd": ("hbm", 3 * BH * S * d * 4 + 3 * BH * N * d * e + BH * S * 4),
@@ -165,7 +165,8 @@ def run_ours(args, world, rank, local):
     pq, pk, pv = E(B, H, max(R, 1), d), E(B, H, max(R, 1), d), E(B, H, max(R, 1), d)
     score = E(B, H, N + R, t=torch.float32)
     idx = E(B, H, S, t=torch.int32)
-    qs, ks, vs, os_ = (E(B, H, S, d) for _ in range(4))
+    qs, ks, vs = (E(B, H, S, d) for _ in range(3))
+    os_ = E(B, H, S, d, t=torch.float32)
     lse = E(B, H, S, t=torch.float32)
     o = E(B, H, N, d)
     dos = E(B, H, S, d)
@@ -331,14 +332,22 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w):
-    frac = 4
+def cpu_baseline(w, budget_s=25.0):
+    """The oracle on one head: the whole head if it fits the budget, else a prefix."""
+    frac = 16
     value, dt, N, S = time_oracle(w, frac)
+    for f in (4, 1):  # grow the sample while the projected time (about linear in N) fits
+        if dt * (frac / f) * 1.3 <= budget_s:
+            frac = f
+            value, dt, N, S = time_oracle(w, frac)
+        else:
+            break
     return {"value": round(value, 2), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"head 0 of {w.B * w.H}, first {N} of {w.N} tokens (S={S}, same p, L, "
                       f"rows per chunk), fwd+bwd in {dt:.2f}s; tokens/s = {N}/({dt:.2f}s x "
-                      f"{w.B * w.H} heads). A prefix has cheaper attention per token than the "
-                      "whole sequence, so this overstates the oracle's full-workload rate."}
+                      f"{w.B * w.H} heads)." + ("" if N == w.N else " A prefix has cheaper "
+                      "attention per token than the whole sequence, so this overstates the "
+                      "oracle's full-workload rate.")}
 
 
 def run_reference(args, world, rank):

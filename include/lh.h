@@ -19,8 +19,8 @@
  *  - Tensors are contiguous [B, H, rows, d] with d fastest. They live in device memory that the
  *    caller allocates and frees. The library never allocates, frees or synchronises, except for
  *    lh_check, which synchronises the stream it is given.
- *  - The element type of Q, K, V, pyramid, subsequence and output tensors is shape.dtype (fp32
- *    or bf16). Score, lse and the sub-gradients dq_sub/dk_sub/dv_sub are always fp32.
+ *  - The element type of Q, K, V, pyramid, q/k/v/do_sub and output tensors is shape.dtype (fp32
+ *    or bf16). Score, lse, o_sub and the sub-gradients dq_sub/dk_sub/dv_sub are always fp32.
  *  - `stream` is a cudaStream_t passed as void*. NULL means the legacy default stream. Every
  *    launch is asynchronous and stream-ordered.
  *  - Return values report host-side validation and launch errors. Nothing is launched when
@@ -116,20 +116,21 @@ int lh_gather(const lh_shape* shape, const void* q, const void* k, const void* v
               void* q_sub, void* k_sub, void* v_sub, void* ws, void* stream);
 
 /* Step 5 (dense causal attention on the subsequence, section 2.C). Row j is visible to row i
- * iff j <= i. Writes o_sub [B,H,S,d] and lse float [B,H,S] (natural log). */
+ * iff j <= i. Writes o_sub float [B,H,S,d] (kept in fp32: the scatter-back and the backward's
+ * D_i = do_sub[i] . o_sub[i] use the unrounded output) and lse float [B,H,S] (natural log). */
 int lh_attn_fwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
-                void* o_sub, float* lse, void* ws, void* stream);
+                float* o_sub, float* lse, void* ws, void* stream);
 
-/* Backward of step 5. do_sub is [B,H,S,d] in shape.dtype; dq_sub, dk_sub, dv_sub are float
- * [B,H,S,d]. Uses the workspace for D_i = do_sub[i] . o_sub[i]. */
+/* Backward of step 5. o_sub is float (from lh_attn_fwd); do_sub is [B,H,S,d] in shape.dtype;
+ * dq_sub, dk_sub, dv_sub are float [B,H,S,d]. Uses the workspace for D_i = do_sub[i].o_sub[i]. */
 int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
-                const void* o_sub, const float* lse, const void* do_sub, float* dq_sub,
+                const float* o_sub, const float* lse, const void* do_sub, float* dq_sub,
                 float* dk_sub, float* dv_sub, void* ws, void* stream);
 
 /* Step 6 (deterministic scatter-back, section 2.C). o[t] = sum of o_sub[i] over the rows i of
  * t's chunk whose span covers t, added in ascending i, no atomics. idx must be a valid
- * selection (causal order, coarsest cell last in each chunk). */
-int lh_scatter(const lh_shape* shape, const int32_t* idx, const void* o_sub, void* o,
+ * selection (causal order, coarsest cell last in each chunk). o_sub is float [B,H,S,d]. */
+int lh_scatter(const lh_shape* shape, const int32_t* idx, const float* o_sub, void* o,
                void* stream);
 
 /* Backward of step 6: do_sub[i] = sum of d_o over the tokens of span(i). */

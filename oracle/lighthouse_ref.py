@@ -324,6 +324,30 @@ def round_to(x, store):
     raise ValueError(store)
 
 
+def pool_stored(x, geo: Geometry, store, mean=True):
+    """The stored pooled levels 1..L-1 of x, [B,H,R,d] (SPEC sections 1 and 9).
+
+    Rounding a pooled value to the storage type is a quantisation, so it is decided on the same
+    fp32 value that the layer rounds: each level adds its p children's unrounded fp32 sums from
+    left to right, in fp32; the cell is fl32(sum * fl32(1/p^l)) (mean=True) or the sum itself
+    (mean=False, the span sums of the backward), then rounded once to `store`.
+    """
+    B, H, N, d = x.shape
+    sums = np.asarray(x, dtype=np.float32)
+    out = []
+    for l in range(1, geo.L):
+        ch = sums.reshape(B, H, -1, geo.p, d)
+        acc = ch[:, :, :, 0, :]
+        for c in range(1, geo.p):
+            acc = acc + ch[:, :, :, c, :]  # float32, left to right
+        sums = acc
+        val = acc * (np.float32(1.0) / np.float32(geo.p ** l)) if mean else acc
+        out.append(round_to(val.astype(np.float64), store))
+    if not out:
+        return np.zeros((B, H, 0, d))
+    return np.concatenate(out, axis=2)
+
+
 # ---------------------------------------------------------------------------------------
 # Whole layer
 # ---------------------------------------------------------------------------------------
@@ -331,18 +355,21 @@ def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
     """Forward of the layer. g is the score group size (8 for bf16 inputs, 4 for fp32).
 
     idx may be given to force a selection (used for the dense recovery identity). store names
-    the storage type of the stored intermediates (pyramid cells and O_sub), SPEC section 9.
+    the storage type of the stored intermediates, SPEC section 9: the pooled cells (and, in
+    layer_bwd, the span sums dO_sub) are then the fp32 sums of SPEC section 1 rounded to it.
     Returns (O [B,H,N,d] float64, saved dict for layer_bwd).
     """
     geo.check()
-    pq, pk, pv = (round_to(build_pyramid(x, geo), store) for x in (q, k, v))
+    if store is None:
+        pq, pk, pv = (build_pyramid(x, geo) for x in (q, k, v))
+    else:
+        pq, pk, pv = (pool_stored(x, geo, store) for x in (q, k, v))
     r = None
     if idx is None:
         r = score(q, k, geo, g)
         idx = select_topk(r, geo)
     qs, ks, vs = gather(q, pq, idx), gather(k, pk, idx), gather(v, pv, idx)
-    os_, lse = attn_fwd(qs, ks, vs)
-    os_ = round_to(os_, store)
+    os_, lse = attn_fwd(qs, ks, vs)  # O_sub is kept in fp32 by the layer: no storage rounding
     o = scatter(idx, os_, geo)
     saved = dict(idx=idx, score=r, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, geo=geo, store=store)
     return o, saved
@@ -350,7 +377,12 @@ def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
 
 def layer_bwd(saved, d_o):
     """Backward of the layer: returns (dQ, dK, dV) [B,H,N,d] float64."""
-    geo, idx = saved["geo"], saved["idx"]
-    dos = round_to(scatter_bwd(idx, d_o, geo), saved.get("store"))
+    geo, idx, store = saved["geo"], saved["idx"], saved.get("store")
+    if store is None:
+        dos = scatter_bwd(idx, d_o, geo)
+    else:  # the stored span sums: fp32 children sums in the pyramid's order, then rounded
+        full = np.concatenate([np.asarray(d_o, np.float64),
+                               pool_stored(d_o, geo, store, mean=False)], axis=2)
+        dos = np.take_along_axis(full, idx[..., None].astype(np.int64), axis=2)
     dqs, dks, dvs = attn_bwd(saved["qs"], saved["ks"], saved["vs"], saved["os"], saved["lse"], dos)
     return gather_bwd(idx, dqs, geo), gather_bwd(idx, dks, geo), gather_bwd(idx, dvs, geo)

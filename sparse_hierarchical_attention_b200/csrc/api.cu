@@ -115,7 +115,7 @@ SavedLayout saved_layout(const Geo& g) {
   s.qs = o; o += sub;
   s.ks = o; o += sub;
   s.vs = o; o += sub;
-  s.os = o; o += sub;
+  s.os = o; o += align256((size_t)(g.BH * g.S * g.d) * 4);  // fp32 o_sub
   s.lse = o; o += align256((size_t)(g.BH * g.S) * 4);
   s.total = o;
   return s;
@@ -142,14 +142,14 @@ template <typename T> const T* at(const void* base, size_t off) {
     if (e_ != cudaSuccess) return fail_cuda(e_); \
   }
 
-cudaError_t attn_fwd(const Geo& g, const void* qs, const void* ks, const void* vs, void* os,
+cudaError_t attn_fwd(const Geo& g, const void* qs, const void* ks, const void* vs, float* os,
                      float* lse, uint32_t* status, cudaStream_t st) {
   (void)status;
   return launch_attn_fwd_simt(g, qs, ks, vs, os, lse, st);
 }
 
 cudaError_t attn_bwd(const Geo& g, const void* qs, const void* ks, const void* vs,
-                     const void* os, const float* lse, const void* dos, float* dq, float* dk,
+                     const float* os, const float* lse, const void* dos, float* dq, float* dk,
                      float* dv, float* delta, uint32_t* status, cudaStream_t st) {
   (void)status;
   return launch_attn_bwd_simt(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, st);
@@ -270,7 +270,7 @@ int lh_gather(const lh_shape* shape, const void* q, const void* k, const void* v
 }
 
 int lh_attn_fwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
-                void* o_sub, float* lse, void* ws, void* stream) {
+                float* o_sub, float* lse, void* ws, void* stream) {
   LH_CHECK_GEO(shape, g);
   LH_REQUIRE_PTR(q_sub); LH_REQUIRE_PTR(k_sub); LH_REQUIRE_PTR(v_sub);
   LH_REQUIRE_PTR(o_sub); LH_REQUIRE_PTR(lse); LH_REQUIRE_PTR(ws);
@@ -280,7 +280,7 @@ int lh_attn_fwd(const lh_shape* shape, const void* q_sub, const void* k_sub, con
 }
 
 int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, const void* v_sub,
-                const void* o_sub, const float* lse, const void* do_sub, float* dq_sub,
+                const float* o_sub, const float* lse, const void* do_sub, float* dq_sub,
                 float* dk_sub, float* dv_sub, void* ws, void* stream) {
   LH_CHECK_GEO(shape, g);
   LH_REQUIRE_PTR(q_sub); LH_REQUIRE_PTR(k_sub); LH_REQUIRE_PTR(v_sub); LH_REQUIRE_PTR(o_sub);
@@ -292,13 +292,13 @@ int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, con
   return LH_OK;
 }
 
-int lh_scatter(const lh_shape* shape, const int32_t* idx, const void* o_sub, void* o,
+int lh_scatter(const lh_shape* shape, const int32_t* idx, const float* o_sub, void* o,
                void* stream) {
   LH_CHECK_GEO(shape, g);
   LH_REQUIRE_PTR(idx); LH_REQUIRE_PTR(o_sub); LH_REQUIRE_PTR(o);
   const void* src[1] = {o_sub};
   void* dst[1] = {o};
-  LH_CUDA(launch_spread(g, idx, 1, false, false, src, dst, nullptr, static_cast<cudaStream_t>(stream)));
+  LH_CUDA(launch_spread(g, idx, 1, true, false, src, dst, nullptr, static_cast<cudaStream_t>(stream)));
   return LH_OK;
 }
 
@@ -343,10 +343,10 @@ int lh_layer_fwd(const lh_shape* shape, const void* q, const void* k, const void
   LH_CUDA(launch_gather(g, q, k, v, pq, pk, pv, idx, at<char>(saved, s.qs), at<char>(saved, s.ks),
                         at<char>(saved, s.vs), status, st));
   LH_CUDA(attn_fwd(g, at<char>(saved, s.qs), at<char>(saved, s.ks), at<char>(saved, s.vs),
-                   at<char>(saved, s.os), at<float>(saved, s.lse), status, st));
-  const void* src[1] = {at<char>(saved, s.os)};
+                   at<float>(saved, s.os), at<float>(saved, s.lse), status, st));
+  const void* src[1] = {at<float>(saved, s.os)};
   void* dst[1] = {o};
-  LH_CUDA(launch_spread(g, idx, 1, false, false, src, dst, status, st));
+  LH_CUDA(launch_spread(g, idx, 1, true, false, src, dst, status, st));
   return LH_OK;
 }
 
@@ -366,7 +366,7 @@ int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void
   float* dvs = at<float>(ws, w.dv);
   LH_CUDA(launch_span_sum(g, idx, d_o, dos, at<char>(ws, w.stmp), status, st));
   LH_CUDA(attn_bwd(g, at<char>(saved, s.qs), at<char>(saved, s.ks), at<char>(saved, s.vs),
-                   at<char>(saved, s.os), at<float>(saved, s.lse), dos, dqs, dks, dvs,
+                   at<float>(saved, s.os), at<float>(saved, s.lse), dos, dqs, dks, dvs,
                    at<float>(ws, w.delta), status, st));
   const void* src[3] = {dqs, dks, dvs};
   void* dst[3] = {dq, dk, dv};

@@ -34,7 +34,7 @@ __device__ inline void load_tile(float* dst, const E* src, int64_t row0, int64_t
 
 template <typename E, int D>
 __global__ void __launch_bounds__(kThreads)
-attn_fwd_simt(const E* __restrict__ Q, const E* __restrict__ K, const E* __restrict__ V, E* O,
+attn_fwd_simt(const E* __restrict__ Q, const E* __restrict__ K, const E* __restrict__ V, float* O,
               float* lse, int64_t S, float sigma) {
   constexpr int P = D + 1, CC = D / 16;
   extern __shared__ float sm[];
@@ -129,21 +129,21 @@ attn_fwd_simt(const E* __restrict__ Q, const E* __restrict__ K, const E* __restr
     if (i >= S) continue;
     const float inv = 1.f / l_i[ii];
 #pragma unroll
-    for (int cc = 0; cc < CC; ++cc) O[(bh * S + i) * D + tc + 16 * cc] = from_f32<E>(o[ii][cc] * inv);
+    for (int cc = 0; cc < CC; ++cc) O[(bh * S + i) * D + tc + 16 * cc] = o[ii][cc] * inv;
     if (tc == 0) lse[bh * S + i] = m_i[ii] + logf(l_i[ii]);
   }
 }
 
-// D_i = dO_sub[i] . O_sub[i] in fp32; one warp per row.
+// D_i = dO_sub[i] . O_sub[i] in fp32 (O_sub kept in fp32); one warp per row.
 template <typename E, int D>
-__global__ void attn_delta(const E* __restrict__ O, const E* __restrict__ dO, float* delta,
+__global__ void attn_delta(const float* __restrict__ O, const E* __restrict__ dO, float* delta,
                            int64_t rows) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= rows) return;
   float acc = 0.f;
   for (int c = lane; c < D; c += 32)
-    acc = fmaf(to_f32(O[row * D + c]), to_f32(dO[row * D + c]), acc);
+    acc = fmaf(O[row * D + c], to_f32(dO[row * D + c]), acc);
 #pragma unroll
   for (int o2 = 16; o2 >= 1; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
   if (lane == 0) delta[row] = acc;
@@ -347,23 +347,23 @@ attn_bwd_dq_simt(const E* __restrict__ Q, const E* __restrict__ K, const E* __re
 }
 
 template <typename E, int D>
-cudaError_t fwd(const Geo& g, const void* qs, const void* ks, const void* vs, void* os, float* lse,
+cudaError_t fwd(const Geo& g, const void* qs, const void* ks, const void* vs, float* os, float* lse,
                 cudaStream_t st) {
   const size_t smem = (size_t)(3 * BM * (D + 1) + BM * 65) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_simt<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((g.S + BM - 1) / BM), (unsigned)g.BH);
-  attn_fwd_simt<E, D><<<grid, kThreads, smem, st>>>((const E*)qs, (const E*)ks, (const E*)vs, (E*)os, lse,
+  attn_fwd_simt<E, D><<<grid, kThreads, smem, st>>>((const E*)qs, (const E*)ks, (const E*)vs, os, lse,
                                                     g.S, 1.0f / sqrtf((float)D));
   return cudaGetLastError();
 }
 
 template <typename E, int D>
-cudaError_t bwd(const Geo& g, const void* qs, const void* ks, const void* vs, const void* os,
+cudaError_t bwd(const Geo& g, const void* qs, const void* ks, const void* vs, const float* os,
                 const float* lse, const void* dos, float* dq, float* dk, float* dv, float* delta,
                 cudaStream_t st) {
   const int64_t rows = g.BH * g.S;
-  attn_delta<E, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const E*)os, (const E*)dos, delta, rows);
+  attn_delta<E, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(os, (const E*)dos, delta, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float sigma = 1.0f / sqrtf((float)D);
@@ -388,7 +388,7 @@ int attn_fwd_launches(const Geo&) { return 1; }
 int attn_bwd_launches(const Geo&) { return 3; }
 
 cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
-                                 void* os, float* lse, cudaStream_t st) {
+                                 float* os, float* lse, cudaStream_t st) {
   if (g.dtype == LH_BF16)
     return g.d == 64 ? fwd<__nv_bfloat16, 64>(g, qs, ks, vs, os, lse, st)
                      : fwd<__nv_bfloat16, 128>(g, qs, ks, vs, os, lse, st);
@@ -396,7 +396,7 @@ cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, c
 }
 
 cudaError_t launch_attn_bwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
-                                 const void* os, const float* lse, const void* dos, float* dq,
+                                 const float* os, const float* lse, const void* dos, float* dq,
                                  float* dk, float* dv, float* delta, cudaStream_t st) {
   if (g.dtype == LH_BF16)
     return g.d == 64 ? bwd<__nv_bfloat16, 64>(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, st)

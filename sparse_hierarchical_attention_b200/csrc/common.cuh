@@ -89,9 +89,9 @@ size_t span_sum_tmp_bytes(const Geo& g);
 int attn_fwd_launches(const Geo& g);
 int attn_bwd_launches(const Geo& g);
 cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
-                                 void* os, float* lse, cudaStream_t st);
+                                 float* os, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
-                                 const void* os, const float* lse, const void* dos, float* dq,
+                                 const float* os, const float* lse, const void* dos, float* dq,
                                  float* dk, float* dv, float* delta, cudaStream_t st);
 
 }  // namespace lh

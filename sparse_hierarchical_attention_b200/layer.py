@@ -11,7 +11,6 @@ def saved_views(shape: Shape, saved: torch.Tensor):
     """Views of the forward context: idx, q_sub, k_sub, v_sub, o_sub, lse."""
     offs = _lib.lh_saved_offsets(shape)
     rows = shape.B * shape.H * shape.S
-    esz = torch.tensor([], dtype=shape.dtype).element_size()
 
     def view(off, n, dtype, shp):
         nbytes = n * torch.tensor([], dtype=dtype).element_size()
@@ -23,9 +22,9 @@ def saved_views(shape: Shape, saved: torch.Tensor):
         q_sub=view(offs[1], rows * shape.d, shape.dtype, sub),
         k_sub=view(offs[2], rows * shape.d, shape.dtype, sub),
         v_sub=view(offs[3], rows * shape.d, shape.dtype, sub),
-        o_sub=view(offs[4], rows * shape.d, shape.dtype, sub),
+        o_sub=view(offs[4], rows * shape.d, torch.float32, sub),
         lse=view(offs[5], rows, torch.float32, (shape.B, shape.H, shape.S)),
-    ) if esz else None
+    )
 
 
 class LighthouseLayer:

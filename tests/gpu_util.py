@@ -16,10 +16,10 @@ def store_of(dtype):
 def assert_close(got, want, dtype, what="", mode="scaled"):
     """The acceptance rule (SPEC section 9).
 
-    mode "literal": absolute error; max <= 2e-2, mean <= 2e-3 (bf16) or max <= 1e-4 (fp32).
-    mode "scaled": error / max(|oracle element|, RMS of the oracle tensor), same limits.
-    mode "tail": scaled error of a row-scaled workload: mean <= 2e-3, 99.9th percentile
-      <= 2e-2, max <= 0.25 (bf16; fp32 limits are 1/200 of these).
+    mode "literal": absolute error, for O on unit-variance workloads.
+    mode "scaled": each error divided by max(|oracle element|, RMS of the oracle tensor), for
+    gradients and for row-scaled workloads (heavy-tailed tensors).
+    bf16: max <= 2e-2 and mean <= 2e-3; fp32: max <= 1e-4.
     """
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
@@ -28,19 +28,15 @@ def assert_close(got, want, dtype, what="", mode="scaled"):
     if got.size == 0:
         return 0.0, 0.0
     err = np.abs(got - want)
-    if mode in ("scaled", "tail"):
+    if mode == "scaled":
         rms = float(np.sqrt(np.mean(want ** 2))) or 1.0
         err = err / np.maximum(np.abs(want), rms)
     mx, mean = float(err.max()), float(err.mean())
-    lim = 2e-2 if dtype == torch.bfloat16 else 1e-4
     msg = f"{what} ({mode}): max {mx:.3g} mean {mean:.3g}"
-    if mode == "tail":
-        q = float(np.quantile(err, 0.999))
-        assert mean <= lim / 10 and q <= lim and mx <= 12.5 * lim, msg + f" p99.9 {q:.3g}"
-    elif dtype == torch.bfloat16:
-        assert mx <= lim and mean <= lim / 10, msg
+    if dtype == torch.bfloat16:
+        assert mx <= 2e-2 and mean <= 2e-3, msg
     else:
-        assert mx <= lim, msg
+        assert mx <= 1e-4, msg
     return mx, mean
 
 

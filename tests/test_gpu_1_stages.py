@@ -61,7 +61,12 @@ def test_pyramid_and_score(B, H, N, d, p, L, S, dt):
     bad = np.argwhere(got_r != want_r)
     assert bad.size == 0, f"{len(bad)} score mismatches, first {bad[:3]}"
     for x, px in ((q, pq), (k, pk), (v, pv)):
-        assert_pyramid(np64(px)[:, :, :R], np64(x), geo, dtype)
+        got = np64(px)[:, :, :R]
+        # the stored cells follow SPEC's fp32 order and one rounding: bit-exact
+        want = O.pool_stored(np64(x), geo, store_of(dtype))
+        bad = np.argwhere(got != want)
+        assert bad.size == 0, f"{len(bad)} pooled values differ, first {bad[:3]}"
+        assert_pyramid(got, np64(x), geo, dtype)  # and within the bound of the exact mean
 
 
 SEL_SHAPES = [(1, 2, 4096, 128, 4, 5, 1024), (2, 3, 2048, 64, 4, 3, 512),
@@ -100,7 +105,7 @@ def test_attention_fwd_bwd(B, H, S, d, dt):
     N = S  # an L = 1 shape carries (S, d) to the attention entry points
     shape = Shape(B, H, N, d, 4, 1, S, dtype)
     qs, ks, vs, dos = rand_sub(B, H, S, d, dtype, seed=S)
-    os_ = torch.empty_like(qs)
+    os_ = torch.empty(B, H, S, d, dtype=torch.float32, device="cuda")
     lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
     ws = ws_for(shape)
     lh.lh_attn_fwd(shape, qs, ks, vs, os_, lse, ws)
@@ -141,7 +146,7 @@ def test_gather_scatter_and_backward(B, H, N, d, p, L, S, dt):
     pq, pk, pv = (torch.randn(B, H, R, d, generator=gen, device="cuda").to(dtype) for _ in range(3))
     subs = [torch.empty(B, H, S, d, dtype=dtype, device="cuda") for _ in range(3)]
     lh.lh_gather(shape, q, k, v, pq, pk, pv, idx, *subs, ws)
-    o_sub = torch.randn(B, H, S, d, generator=gen, device="cuda").to(dtype)
+    o_sub = torch.randn(B, H, S, d, generator=gen, device="cuda")
     o = torch.empty(B, H, N, d, dtype=dtype, device="cuda")
     lh.lh_scatter(shape, idx, o_sub, o)
     d_o = torch.randn(B, H, N, d, generator=gen, device="cuda").to(dtype)
@@ -156,8 +161,10 @@ def test_gather_scatter_and_backward(B, H, N, d, p, L, S, dt):
         want = O.gather(np64(x), np64(px)[:, :, :geo.R], idx_np)
         assert np.array_equal(np64(sub), want)
     assert_close(np64(o), O.scatter(idx_np, np64(o_sub), geo), dtype, "scatter")
-    want = O.round_to(O.scatter_bwd(idx_np, np64(d_o), geo), store_of(dtype))  # stored dO_sub
-    assert_close(np64(do_sub), want, dtype, "scatter_bwd")
+    assert_close(np64(do_sub), O.scatter_bwd(idx_np, np64(d_o), geo), dtype, "scatter_bwd")
+    # the stored span sums follow the pyramid's fp32 order and one rounding: bit-exact
+    full = np.concatenate([np64(d_o), O.pool_stored(np64(d_o), geo, store_of(dtype), mean=False)], 2)
+    assert np.array_equal(np64(do_sub), np.take_along_axis(full, idx_np[..., None].astype(np.int64), 2))
     for got, ds in zip(dx, dsub):
         assert_close(np64(got), O.gather_bwd(idx_np, np64(ds), geo), dtype, "gather_bwd")
 

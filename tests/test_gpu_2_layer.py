@@ -54,10 +54,9 @@ def test_layer_matches_oracle(name, B, H, N, S):
     wo, sv, wgrads = oracle_layer(q, k, v, d_o, geo, w.dtype)
     idx = saved_views(shape, saved)["idx"].cpu().numpy()
     assert np.array_equal(idx, sv["idx"]), "selection differs from the oracle"
-    mode = "scaled" if w.scale == "none" else "tail"
-    assert_close(np64(o), wo, w.dtype, "O", mode=mode)
+    assert_close(np64(o), wo, w.dtype, "O")
     for got, want, n in zip(grads, wgrads, ("dQ", "dK", "dV")):
-        assert_close(np64(got), want, w.dtype, n, mode=mode)
+        assert_close(np64(got), want, w.dtype, n)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -112,7 +111,7 @@ def test_dense_recovery_matches_torch_sdpa(dtype):
     ref.backward(d_o.float())
     assert_close(np64(o), np64(ref), dtype, "O", mode="literal")
     for got, t, n in ((dq, tq, "dQ"), (dk, tk, "dK"), (dv, tv, "dV")):
-        assert_close(np64(got), np64(t.grad), dtype, n, mode="scaled")
+        assert_close(np64(got), np64(t.grad), dtype, n)
 
 
 def test_deterministic_bits():
@@ -162,6 +161,6 @@ def test_full_size_sampled_heads(name, unit):
     h = w.H - 1
     sl = (slice(0, 1), slice(h, h + 1))
     wo, sv, wgrads = oracle_layer(q[sl], k[sl], v[sl], d_o[sl], geo, w.dtype)
-    assert_close(np64(o[sl]), wo, w.dtype, "O", mode="literal" if unit else "tail")
+    assert_close(np64(o[sl]), wo, w.dtype, "O", mode="literal" if unit else "scaled")
     for got, want, n in zip(grads, wgrads, ("dQ", "dK", "dV")):
-        assert_close(np64(got[sl]), want, w.dtype, n, mode="scaled" if unit else "tail")
+        assert_close(np64(got[sl]), want, w.dtype, n)

@@ -339,3 +339,32 @@ def test_bf16_rounding_matches_library_conversion():
     assert O.round_to(np.float64(1 + 3 * 2 ** -8), "bf16") == 1 + 2 ** -6
     y = rand(1000).astype(np.float64) / 3
     np.testing.assert_array_equal(O.round_to(y, "f32"), y.astype(np.float32).astype(np.float64))
+
+
+@pytest.mark.parametrize("N,p,L,S", SMALL)
+@pytest.mark.parametrize("store", ["f32", "bf16"])
+def test_stored_pyramid_is_the_rounded_mean(N, p, L, S, store):
+    """The fp32-ordered stored cells are the exact span means up to a derived bound: fp32 sums
+    at most (p-1)(L-1) additions deep, one scaling, one rounding to the storage type."""
+    geo = O.Geometry(N, p, L, S)
+    x = rand(2, 2, N, 8, scale=3.0)
+    got = O.pool_stored(x, geo, store)
+    exact = O.build_pyramid(x, geo)
+    mean_abs = O.build_pyramid(np.abs(x), geo)
+    u = 2.0 ** -8 if store == "bf16" else 2.0 ** -24
+    depth = (p - 1) * (L - 1) + 1
+    bound = depth * 2.0 ** -24 * mean_abs * (1 + u) + u * np.abs(exact) * (1 + 1e-6) + 1e-300
+    assert (np.abs(got - exact) <= bound).all()
+    sums = O.pool_stored(x, geo, store, mean=False)  # span sums: p^l times the mean
+    scale = np.concatenate([np.full(N // p ** l, float(p ** l)) for l in range(1, L)]) if L > 1 \
+        else np.zeros(0)
+    np.testing.assert_allclose(sums, exact * scale[None, None, :, None],
+                               rtol=8 * u + depth * 2.0 ** -23, atol=1e-5 * np.abs(x).max() * N)
+
+
+def test_stored_pyramid_follows_the_fixed_order():
+    """Children are added left to right in fp32: 2^24 + 1 + 1 + 1 stays 2^24 (ties to even)."""
+    geo = O.Geometry(4, 4, 2, 1)
+    x = np.array([2.0 ** 24, 1.0, 1.0, 1.0], np.float32).reshape(1, 1, 4, 1)
+    assert O.pool_stored(x, geo, "f32", mean=False)[0, 0, 0, 0] == 2.0 ** 24
+    assert O.build_pyramid(x, geo)[0, 0, 0, 0] * 4 == 2.0 ** 24 + 3
