@@ -153,6 +153,25 @@ int lh_layer_fwd(const lh_shape* shape, const void* q, const void* k, const void
 int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void* dq, void* dk,
                  void* dv, void* ws, void* stream);
 
+/* lh_attn_bwd without a workspace argument, for callers that cannot allocate device memory:
+ * a plugin whose host framework owns every device allocation, or code that must not call the
+ * allocator at all. The paper has no counterpart; this is a deployment variant of the same
+ * kernels, with the same results as lh_attn_bwd.
+ *  - The per-row scratch (D_i = do_sub[i] . o_sub[i]) lives in a file-scope device array of
+ *    256 + 4 * LH_STATIC_SCRATCH_ROWS bytes (about 4 MiB). Every GPU that loads the library
+ *    holds it until the process exits. The call itself allocates and frees nothing.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current. Make that first call before any stream capture.
+ *  - Returns LH_ERR_WORKSPACE, launching nothing, when B*H*S > LH_STATIC_SCRATCH_ROWS.
+ *  - All calls share the one array, which keeps the previous call's contents. Calls that
+ *    overlap on the GPU (different streams, no ordering between them) race on it.
+ *  - Other arguments, layouts and errors as lh_attn_bwd. */
+#define LH_STATIC_SCRATCH_ROWS (1 << 20)
+int lh_attn_bwd_static(const lh_shape* shape, const void* q_sub, const void* k_sub,
+                       const void* v_sub, const float* o_sub, const float* lse,
+                       const void* do_sub, float* dq_sub, float* dk_sub, float* dv_sub,
+                       void* stream);
+
 /* Number of kernel launches one lh_layer_fwd (*fwd) and one lh_layer_bwd (*bwd) make for this
  * shape (either pointer may be NULL). Host-side plan only; launches nothing. */
 int lh_launches(const lh_shape* shape, int* fwd, int* bwd);

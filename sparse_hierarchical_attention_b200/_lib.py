@@ -62,6 +62,7 @@ def _load():
         "lh_gather_bwd": ([SP, P, P, P, P, P, P, P, P], I),
         "lh_layer_fwd": ([SP, P, P, P, P, P, P, P], I),
         "lh_layer_bwd": ([SP, P, P, P, P, P, P, P], I),
+        "lh_attn_bwd_static": ([SP, P, P, P, P, P, P, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -214,3 +215,14 @@ def lh_layer_fwd(shape, q, k, v, o, saved, ws, stream=None):
 def lh_layer_bwd(shape, saved, d_o, dq, dk, dv, ws, stream=None):
     _check(_lib.lh_layer_bwd(ctypes.byref(shape.c()), _ptr(saved), _ptr(d_o), _ptr(dq), _ptr(dk),
                              _ptr(dv), _ptr(ws), _stream(stream)))
+
+
+LH_STATIC_SCRATCH_ROWS = 1 << 20
+
+
+def lh_attn_bwd_static(shape, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, dv_sub,
+                       stream=None):
+    """lh_attn_bwd for callers that cannot allocate: scratch in the library's static array."""
+    _check(_lib.lh_attn_bwd_static(ctypes.byref(shape.c()), _ptr(q_sub), _ptr(k_sub),
+                                   _ptr(v_sub), _ptr(o_sub), _ptr(lse), _ptr(do_sub),
+                                   _ptr(dq_sub), _ptr(dk_sub), _ptr(dv_sub), _stream(stream)))

@@ -1,0 +1,79 @@
+// lh_attn_bwd_static: the attention backward without a caller-supplied workspace.
+//
+// Some callers cannot allocate device memory at all. Examples are a plugin whose host
+// framework owns every device allocation, and code running where the allocator is off limits.
+// Those callers cannot provide the workspace that lh_attn_bwd takes for its per-row
+// D_i = dO_sub[i] . O_sub[i]. This entry point keeps that scratch in a file-scope device
+// array instead:
+//   - its size is fixed at compile time;
+//   - every GPU that loads this library holds it until the process exits.
+// The caller still passes every input and output buffer.
+//
+// The paper has no counterpart: this is a deployment variant of the same kernels.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace lh {
+namespace {
+
+// 256 bytes of status word, then D for up to LH_STATIC_SCRATCH_ROWS rows (4 MiB).
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kStaticBytes = kStatusBytes + (size_t)LH_STATIC_SCRATCH_ROWS * sizeof(float);
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_dev_ptr[kMaxDevices] = {};  // device address of g_static_scratch, per device ordinal
+
+// Device address of the static scratch on the current device. The first call on a device
+// resolves it with cudaGetSymbolAddress; later calls reuse the cached address.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_dev_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_dev_ptr[dev] = p;
+  }
+  *out = g_dev_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace lh
+
+using namespace lh;
+
+extern "C" int lh_attn_bwd_static(const lh_shape* shape, const void* q_sub, const void* k_sub,
+                                  const void* v_sub, const float* o_sub, const float* lse,
+                                  const void* do_sub, float* dq_sub, float* dk_sub, float* dv_sub,
+                                  void* stream) {
+  if (!shape) return LH_ERR_INVALID_ARG;
+  if (lh_validate(shape, nullptr) != LH_OK) return lh_validate(shape, nullptr);
+  const int64_t rows = (int64_t)shape->B * shape->H * shape->S;
+  if (rows > (int64_t)LH_STATIC_SCRATCH_ROWS) return LH_ERR_WORKSPACE;
+  const void* ptrs[] = {q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, dv_sub};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return LH_ERR_INVALID_ARG;
+  Geo g{};
+  g.B = shape->B; g.H = shape->H; g.N = shape->N; g.d = shape->d; g.p = shape->p;
+  g.L = shape->L; g.S = shape->S; g.dtype = shape->dtype;
+  g.BH = (int64_t)g.B * g.H;
+  g.esize = g.dtype == LH_BF16 ? 2 : 4;
+  void* base = nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (scratch_address(&base) != cudaSuccess) return LH_ERR_CUDA;
+  // the status word must start at zero; D is written in full before it is read
+  if (cudaMemsetAsync(base, 0, kStatusBytes, st) != cudaSuccess) return LH_ERR_CUDA;
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(base) + kStatusBytes);
+  if (launch_attn_bwd_simt(g, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, dv_sub,
+                           delta, st) != cudaSuccess)
+    return LH_ERR_CUDA;
+  return LH_OK;
+}
