@@ -144,7 +144,7 @@ template <typename T> const T* at(const void* base, size_t off) {
 
 cudaError_t attn_fwd(const Geo& g, const void* qs, const void* ks, const void* vs, float* os,
                      float* lse, uint32_t* status, cudaStream_t st) {
-  (void)status;
+  if (attn_tc_eligible(g)) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, status, st);
   return launch_attn_fwd_simt(g, qs, ks, vs, os, lse, st);
 }
 

@@ -99,7 +99,8 @@ def rand_sub(B, H, S, d, dtype, seed):
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("B,H,S,d", [(1, 2, 64, 64), (2, 2, 333, 128), (1, 3, 1000, 64),
-                                     (1, 1, 1, 128), (1, 2, 4096, 128)])
+                                     (1, 1, 1, 128), (1, 2, 4096, 128), (1, 1, 128, 128),
+                                     (2, 3, 256, 64), (1, 2, 1024, 128), (1, 1, 2048, 64)])
 def test_attention_fwd_bwd(B, H, S, d, dt):
     dtype = DT[dt]
     N = S  # an L = 1 shape carries (S, d) to the attention entry points
