@@ -151,11 +151,19 @@ cudaError_t attn_fwd(const Geo& g, const void* qs, const void* ks, const void* v
 cudaError_t attn_bwd(const Geo& g, const void* qs, const void* ks, const void* vs,
                      const float* os, const float* lse, const void* dos, float* dq, float* dk,
                      float* dv, float* delta, uint32_t* status, cudaStream_t st) {
-  (void)status;
-  return launch_attn_bwd_simt(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, st);
+  return attn_bwd_dispatch(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, status, st);
 }
 
 }  // namespace
+
+cudaError_t attn_bwd_dispatch(const Geo& g, const void* qs, const void* ks, const void* vs,
+                              const float* os, const float* lse, const void* dos, float* dq,
+                              float* dk, float* dv, float* delta, uint32_t* status, cudaStream_t st) {
+  if (attn_tc_eligible(g))
+    return launch_attn_bwd_tc(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, status, st);
+  return launch_attn_bwd_simt(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, st);
+}
+
 }  // namespace lh
 
 using namespace lh;

@@ -1,0 +1,532 @@
+// Causal attention backward on the gathered subsequence with tcgen05 tensor cores ("Long Context
+// Pre-Training with Lighthouse Attention", technical summary 2.B: gradients flow through the
+// attention to Q, K and V; SPEC section 7 gives the formulas).
+//
+// Two deterministic kernels; neither uses atomics:
+//   dkdv: one CTA per 128-key block. Thread t owns key row t (TMEM lane t). It steps through
+//         the 64-row query blocks that can see the keys:
+//           S^T = K Q^T and dP^T = V dO^T (two MMAs);
+//           P^T = exp2(S^T c - lse2) and dS^T = P^T (dP^T - D) in fp32 registers;
+//           dV += P^T dO and dK += dS^T Q (A from shared memory, K-major; B = dO or Q read
+//           as MN-major operands).
+//   dq:   one CTA per 128-query block. Thread t owns query row t. It steps through the 64-row
+//         key blocks it sees:
+//           S = Q K^T and dP = dO V^T;
+//           dS as above;
+//           dQ += dS K.
+// dQ, dK and dV all sum P or dS against rows with mixed signs. Coarse rows carry dO_sub that
+// sums thousands of tokens, and there those sums cancel by orders of magnitude. So P^T, dS^T
+// and dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That
+// is one extra MMA per product and keeps the operand to ~16 bits. With one bf16 term, single
+// dV elements were off by 34% of their size.
+// Q/dO (dkdv) and K/V (dq) come through two-stage TMA rings. S and dP live in TMEM and are
+// reused every step; accumulators stay in TMEM until the epilogue writes fp32 results.
+// All waits are bounded and report through the status word.
+#include "tc.cuh"
+
+namespace lh {
+
+bool make_tmap_rows_box(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows);
+
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 128;
+constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
+constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
+
+// ------------------------------------------------------------------------------------ dK, dV
+template <int D>
+struct LayDKV {
+  static constexpr int KB = D / 64;
+  static constexpr int K = 0;                     // [128][D]
+  static constexpr int V = K + KB * T128;         // [128][D]
+  static constexpr int Q = V + KB * T128;         // 2 stages of [64][D]
+  static constexpr int DO = Q + 2 * KB * T64;     // 2 stages of [64][D]
+  static constexpr int PT = DO + 2 * KB * T64;    // hi, lo: [128 keys][64 queries] each
+  static constexpr int DST = PT + 2 * T128;       // hi, lo: [128 keys][64 queries] each
+  static constexpr int VEC = DST + 2 * T128;      // lse2[2][64], delta[2][64]
+  static constexpr int BAR = VEC + 4 * 64 * 4;
+  static constexpr int BYTES = BAR + 128;
+  static constexpr uint32_t TMEM_COLS = D == 128 ? 512 : 256;
+};
+
+// bars: 0 K+V, 1-2 Q/dO stages, 3 S^T+dP^T, 4 dV+dK
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                 const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                 const float* __restrict__ lse, const float* __restrict__ delta,
+                 float* __restrict__ dK, float* __restrict__ dV, int S, float sigma,
+                 float scale_log2, uint32_t* status) {
+  using Ly = LayDKV<D>;
+  constexpr int KB = Ly::KB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 8) + 1;
+  float* lse2_s = reinterpret_cast<float*>(sm + Ly::VEC);  // [2][64]
+  float* del_s = lse2_s + 128;                             // [2][64]
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int kb = blockIdx.x;  // low key blocks see the most queries: they start first
+  const int bh = blockIdx.y;
+  const int g0 = bh * S;
+  const int k0 = kb * 128;
+  const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
+  const float LOG2E = 1.4426950408889634f;
+
+  if (tid == 0) {
+    for (int i = 0; i < 8; ++i) mbar_init(bar + i, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, Ly::TMEM_COLS);
+  auto load_vec = [&](int it) {  // lse2 and delta of query block it into stage it & 1
+    if (tid < 64) {
+      const int qi = g0 + k0 + it * 64 + tid;
+      lse2_s[(it & 1) * 64 + tid] = lse[qi] * LOG2E;
+      del_s[(it & 1) * 64 + tid] = delta[qi];
+    }
+  };
+  load_vec(0);
+  if (nit > 1) load_vec(1);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t t_st = tbase, t_dpt = tbase + 64, t_dv = tbase + 128, t_dk = tbase + 128 + D;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
+  const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
+  const uint32_t s_pt = smem_u32(sm + Ly::PT), s_dst = smem_u32(sm + Ly::DST);
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
+
+  auto load_qdo = [&](int it) {
+    uint64_t* b = bar + 1 + (it & 1);
+    mbar_expect_tx(b, 2 * KB * T64);
+    for (int c = 0; c < KB; ++c) {
+      tma_load_2d(sm + Ly::Q + (it & 1) * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
+      tma_load_2d(sm + Ly::DO + (it & 1) * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
+    }
+  };
+  auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T
+    const uint32_t qb = s_q + (it & 1) * KB * T64, ob = s_do + (it & 1) * KB * T64;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
+      mma_ss(t_st, sw128_desc(s_k + offA, 16, 1024), sw128_desc(qb + offB, 16, 1024), IDESC_S, ks > 0);
+      mma_ss(t_dpt, sw128_desc(s_v + offA, 16, 1024), sw128_desc(ob + offB, 16, 1024), IDESC_S, ks > 0);
+    }
+    mma_commit(bar + 3);
+  };
+  auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
+    const uint32_t qb = s_q + (it & 1) * KB * T64, ob = s_do + (it & 1) * KB * T64;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      mma_ss(t_dv, sw128_desc(s_pt + ks * 32, 16, 1024), sw128_desc(ob + ks * 2048, T64, 1024),
+             IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+      mma_ss(t_dv, sw128_desc(s_pt + T128 + ks * 32, 16, 1024), sw128_desc(ob + ks * 2048, T64, 1024),
+             IDESC_ACC, 1u);
+      mma_ss(t_dk, sw128_desc(s_dst + ks * 32, 16, 1024), sw128_desc(qb + ks * 2048, T64, 1024),
+             IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+      mma_ss(t_dk, sw128_desc(s_dst + T128 + ks * 32, 16, 1024), sw128_desc(qb + ks * 2048, T64, 1024),
+             IDESC_ACC, 1u);
+    }
+    mma_commit(bar + 4);
+  };
+  auto wait_all = [&](uint64_t* b, uint32_t parity) {
+    bool ok = mbar_wait(b, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  if (tid == 0) {
+    mbar_expect_tx(bar, 2 * KB * T128);
+    for (int c = 0; c < KB; ++c) {
+      tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
+      tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
+    }
+    load_qdo(0);
+    if (nit > 1) load_qdo(1);
+    if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
+  }
+  __syncwarp();
+
+  const int row = tid;  // key row within the block = TMEM lane
+  const int kj = k0 + row;
+  for (int it = 0; it < nit; ++it) {
+    const bool ok_s = wait_all(bar + 3, it & 1);
+    tc_fence_after();
+    float st[64], dpt[64];
+    if (ok_s) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(t_st + lane_off + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) st[c * 32 + e] = __uint_as_float(r[e]);
+        tmem_ld32(t_dpt + lane_off + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dpt[c * 32 + e] = __uint_as_float(r[e]);
+      }
+    }
+    const float* l2 = lse2_s + (it & 1) * 64;
+    const float* dl = del_s + (it & 1) * 64;
+    const int q0 = k0 + it * 64;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const bool vis = kj <= q0 + c;
+      const float p = vis ? exp2f(st[c] * scale_log2 - l2[c]) : 0.f;
+      st[c] = p;
+      dpt[c] = p * (dpt[c] - dl[c]);
+    }
+    // the accumulate MMAs of the previous step read P^T, dS^T and the other Q/dO stage
+    bool ok_m = true;
+    if (it > 0) {
+      ok_m = wait_all(bar + 4, (it - 1) & 1);
+      tc_fence_after();
+      if (tid == 0 && ok_m && it + 1 < nit && it >= 1) load_qdo(it + 1);
+      __syncwarp();
+      if (it + 1 < nit && it >= 1) load_vec(it + 1);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // 8 chunks of 8 queries, K-major, 128-byte swizzle
+      uint32_t wp[4], wq[4], wh[4], wl[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float u = st[c * 8 + 2 * h], v = st[c * 8 + 2 * h + 1];
+        __nv_bfloat162 ph = __floats2bfloat162_rn(u, v);
+        __nv_bfloat162 pl = __floats2bfloat162_rn(u - __low2float(ph), v - __high2float(ph));
+        const float x = dpt[c * 8 + 2 * h], y = dpt[c * 8 + 2 * h + 1];
+        __nv_bfloat162 hi = __floats2bfloat162_rn(x, y);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(x - __low2float(hi), y - __high2float(hi));
+        wp[h] = *reinterpret_cast<uint32_t*>(&ph);
+        wq[h] = *reinterpret_cast<uint32_t*>(&pl);
+        wh[h] = *reinterpret_cast<uint32_t*>(&hi);
+        wl[h] = *reinterpret_cast<uint32_t*>(&lo);
+      }
+      const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_pt + off), "r"(wp[0]), "r"(wp[1]),
+                   "r"(wp[2]), "r"(wp[3])
+                   : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_pt + T128 + off), "r"(wq[0]),
+                   "r"(wq[1]), "r"(wq[2]), "r"(wq[3])
+                   : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_dst + off), "r"(wh[0]), "r"(wh[1]),
+                   "r"(wh[2]), "r"(wh[3])
+                   : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_dst + T128 + off), "r"(wl[0]),
+                   "r"(wl[1]), "r"(wl[2]), "r"(wl[3])
+                   : "memory");
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) break;
+    if (tid == 0) {
+      issue_acc(it);
+      if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
+        issue_s(it + 1);
+    }
+    __syncwarp();
+  }
+
+  const bool ok_end = !*abort_flag && wait_all(bar + 4, (nit - 1) & 1);
+  tc_fence_after();
+  if (ok_end) {
+    float* dvrow = dV + (size_t)(g0 + kj) * D;
+    float* dkrow = dK + (size_t)(g0 + kj) * D;
+    uint32_t r[32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      tmem_ld32(t_dv + lane_off + c * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dvrow + c * 32 + e) =
+            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                        __uint_as_float(r[e + 3]));
+      tmem_ld32(t_dk + lane_off + c * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dkrow + c * 32 + e) =
+            make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
+                        __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 1000000ull) {
+    }
+  }
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, Ly::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------ dQ
+template <int D>
+struct LayDQ {
+  static constexpr int KB = D / 64;
+  static constexpr int Q = 0;                    // [128][D]
+  static constexpr int DO = Q + KB * T128;       // [128][D]
+  static constexpr int K = DO + KB * T128;       // 2 stages of [64][D]
+  static constexpr int V = K + 2 * KB * T64;     // 2 stages of [64][D]
+  static constexpr int DS = V + 2 * KB * T64;    // hi, lo: [128 queries][64 keys] each
+  static constexpr int BAR = DS + 2 * T128;
+  static constexpr int BYTES = BAR + 128;
+};
+
+// bars: 0 Q+dO, 1-2 K/V stages, 3 S+dP, 4 dQ
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+               const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+               const float* __restrict__ lse, const float* __restrict__ delta,
+               float* __restrict__ dQ, int S, float sigma, float scale_log2, uint32_t* status) {
+  using Ly = LayDQ<D>;
+  constexpr int KB = Ly::KB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 8) + 1;
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int nqb = S / 128;
+  const int qb = nqb - 1 - (int)blockIdx.x;  // heaviest first
+  const int bh = blockIdx.y;
+  const int g0 = bh * S;
+  const int q0 = qb * 128;
+  const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
+  const float LOG2E = 1.4426950408889634f;
+
+  if (tid == 0) {
+    for (int i = 0; i < 8; ++i) mbar_init(bar + i, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t t_s = tbase, t_dp = tbase + 64, t_dq = tbase + 128;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
+  const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
+  const uint32_t s_ds = smem_u32(sm + Ly::DS);
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
+
+  auto load_kv = [&](int it) {
+    uint64_t* b = bar + 1 + (it & 1);
+    mbar_expect_tx(b, 2 * KB * T64);
+    for (int c = 0; c < KB; ++c) {
+      tma_load_2d(sm + Ly::K + (it & 1) * KB * T64 + c * T64, &tk, c * 64, g0 + it * 64, b);
+      tma_load_2d(sm + Ly::V + (it & 1) * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
+    }
+  };
+  auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T
+    const uint32_t kbs = s_k + (it & 1) * KB * T64, vbs = s_v + (it & 1) * KB * T64;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
+      mma_ss(t_s, sw128_desc(s_q + offA, 16, 1024), sw128_desc(kbs + offB, 16, 1024), IDESC_S, ks > 0);
+      mma_ss(t_dp, sw128_desc(s_do + offA, 16, 1024), sw128_desc(vbs + offB, 16, 1024), IDESC_S, ks > 0);
+    }
+    mma_commit(bar + 3);
+  };
+  auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
+    const uint32_t kbs = s_k + (it & 1) * KB * T64;
+#pragma unroll
+    for (int part = 0; part < 2; ++part)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_ss(t_dq, sw128_desc(s_ds + part * T128 + ks * 32, 16, 1024),
+               sw128_desc(kbs + ks * 2048, T64, 1024), IDESC_ACC, (it > 0 || part > 0 || ks > 0) ? 1u : 0u);
+    mma_commit(bar + 4);
+  };
+  auto wait_all = [&](uint64_t* b, uint32_t parity) {
+    bool ok = mbar_wait(b, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  if (tid == 0) {
+    mbar_expect_tx(bar, 2 * KB * T128);
+    for (int c = 0; c < KB; ++c) {
+      tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
+      tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
+    }
+    load_kv(0);
+    if (nit > 1) load_kv(1);
+    if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
+  }
+  __syncwarp();
+
+  const int row = tid;  // query row within the block = TMEM lane
+  const int qi = q0 + row;
+  const float l2 = lse[g0 + qi] * LOG2E;
+  const float dl = delta[g0 + qi];
+  for (int it = 0; it < nit; ++it) {
+    const bool ok_s = wait_all(bar + 3, it & 1);
+    tc_fence_after();
+    float s[64], dp[64];
+    if (ok_s) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(t_s + lane_off + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+        tmem_ld32(t_dp + lane_off + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dp[c * 32 + e] = __uint_as_float(r[e]);
+      }
+    }
+    const int kj0 = it * 64;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const bool vis = kj0 + c <= qi;
+      const float p = vis ? exp2f(s[c] * scale_log2 - l2) : 0.f;
+      dp[c] = p * (dp[c] - dl);
+    }
+    bool ok_m = true;
+    if (it > 0) {
+      ok_m = wait_all(bar + 4, (it - 1) & 1);
+      tc_fence_after();
+      if (tid == 0 && ok_m && it + 1 < nit && it >= 1) load_kv(it + 1);
+      __syncwarp();
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // dS = hi + lo, K-major, 128-byte swizzle
+      uint32_t wh[4], wl[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float a = dp[c * 8 + 2 * h], b = dp[c * 8 + 2 * h + 1];
+        __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
+        wh[h] = *reinterpret_cast<uint32_t*>(&hi);
+        wl[h] = *reinterpret_cast<uint32_t*>(&lo);
+      }
+      const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_ds + off), "r"(wh[0]), "r"(wh[1]),
+                   "r"(wh[2]), "r"(wh[3])
+                   : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_ds + T128 + off), "r"(wl[0]),
+                   "r"(wl[1]), "r"(wl[2]), "r"(wl[3])
+                   : "memory");
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) break;
+    if (tid == 0) {
+      issue_acc(it);
+      if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
+        issue_s(it + 1);
+    }
+    __syncwarp();
+  }
+
+  const bool ok_end = !*abort_flag && wait_all(bar + 4, (nit - 1) & 1);
+  tc_fence_after();
+  if (ok_end) {
+    float* dqrow = dQ + (size_t)(g0 + qi) * D;
+    uint32_t r[32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      tmem_ld32(t_dq + lane_off + c * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dqrow + c * 32 + e) =
+            make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
+                        __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 1000000ull) {
+    }
+  }
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
+// D_i = dO_sub[i] . O_sub[i] (fp32 O_sub); one warp per row.
+__global__ void delta_kernel(const float* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
+                             float* __restrict__ delta, int64_t rows, int D) {
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int c = lane * 4; c < D; c += 128) {
+    const float4 o = *reinterpret_cast<const float4*>(O + row * D + c);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(dO + row * D + c);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dO + row * D + c + 2);
+    acc = fmaf(o.x, __low2float(a), acc);
+    acc = fmaf(o.y, __high2float(a), acc);
+    acc = fmaf(o.z, __low2float(b), acc);
+    acc = fmaf(o.w, __high2float(b), acc);
+  }
+#pragma unroll
+  for (int o2 = 16; o2 >= 1; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+  if (lane == 0) delta[row] = acc;
+}
+
+template <int D>
+cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs, const float* os,
+                    const float* lse, const void* dos, float* dq, float* dk, float* dv, float* delta,
+                    uint32_t* status, cudaStream_t st) {
+  const int64_t rows = g.BH * g.S;
+  CUtensorMap q64, do64, k128, v128, q128, do128, k64, v64;
+  if (!make_tmap_rows_box(&q64, qs, rows, D, 64) || !make_tmap_rows_box(&do64, dos, rows, D, 64) ||
+      !make_tmap_rows_box(&k128, ks, rows, D, 128) || !make_tmap_rows_box(&v128, vs, rows, D, 128) ||
+      !make_tmap_rows_box(&q128, qs, rows, D, 128) || !make_tmap_rows_box(&do128, dos, rows, D, 128) ||
+      !make_tmap_rows_box(&k64, ks, rows, D, 64) || !make_tmap_rows_box(&v64, vs, rows, D, 64))
+    return cudaErrorInvalidValue;
+  delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(os, (const __nv_bfloat16*)dos, delta, rows, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const float sigma = 1.0f / sqrtf((float)D);
+  const float scale_log2 = sigma * 1.4426950408889634f;
+  const int smem1 = LayDKV<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(attn_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
+  if (e != cudaSuccess) return e;
+  attn_bwd_dkdv_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem1, st>>>(
+      k128, v128, q64, do64, lse, delta, dk, dv, g.S, sigma, scale_log2, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int smem2 = LayDQ<D>::BYTES + 1024;
+  e = cudaFuncSetAttribute(attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+  if (e != cudaSuccess) return e;
+  attn_bwd_dq_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem2, st>>>(
+      q128, do128, k64, v64, lse, delta, dq, g.S, sigma, scale_log2, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
+                               const float* os, const float* lse, const void* dos, float* dq,
+                               float* dk, float* dv, float* delta, uint32_t* status, cudaStream_t st) {
+  return g.d == 128 ? run_bwd<128>(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, status, st)
+                    : run_bwd<64>(g, qs, ks, vs, os, lse, dos, dq, dk, dv, delta, status, st);
+}
+
+}  // namespace lh

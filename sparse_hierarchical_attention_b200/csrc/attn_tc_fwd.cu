@@ -279,17 +279,21 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// [rows, D] bf16 matrix, boxes of [128 rows][64 columns] with 128-byte swizzle.
-bool make_tmap_rows(CUtensorMap* map, const void* base, int64_t rows, int D) {
+// [rows, D] bf16 matrix, boxes of [box_rows][64 columns] with 128-byte swizzle.
+bool make_tmap_rows_box(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_rows(CUtensorMap* map, const void* base, int64_t rows, int D) {
+  return make_tmap_rows_box(map, base, rows, D, 128);
 }
 
 bool attn_tc_eligible(const Geo& g) {

@@ -89,6 +89,13 @@ size_t span_sum_tmp_bytes(const Geo& g);
 bool attn_tc_eligible(const Geo& g);  // bf16, d in {64,128}, S % 128 == 0
 cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
                                float* os, float* lse, uint32_t* status, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
+                               const float* os, const float* lse, const void* dos, float* dq,
+                               float* dk, float* dv, float* delta, uint32_t* status, cudaStream_t st);
+// The attention backward as the library runs it: tensor cores where eligible, else fp32 FMA.
+cudaError_t attn_bwd_dispatch(const Geo& g, const void* qs, const void* ks, const void* vs,
+                              const float* os, const float* lse, const void* dos, float* dq,
+                              float* dk, float* dv, float* delta, uint32_t* status, cudaStream_t st);
 int attn_fwd_launches(const Geo& g);
 int attn_bwd_launches(const Geo& g);
 cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,

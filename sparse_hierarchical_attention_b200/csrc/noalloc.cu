@@ -72,8 +72,9 @@ extern "C" int lh_attn_bwd_static(const lh_shape* shape, const void* q_sub, cons
   // the status word must start at zero; D is written in full before it is read
   if (cudaMemsetAsync(base, 0, kStatusBytes, st) != cudaSuccess) return LH_ERR_CUDA;
   float* delta = reinterpret_cast<float*>(static_cast<char*>(base) + kStatusBytes);
-  if (launch_attn_bwd_simt(g, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, dv_sub,
-                           delta, st) != cudaSuccess)
+  uint32_t* dev_status = reinterpret_cast<uint32_t*>(base);
+  if (attn_bwd_dispatch(g, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, dv_sub, delta,
+                        dev_status, st) != cudaSuccess)
     return LH_ERR_CUDA;
   return LH_OK;
 }
