@@ -3,14 +3,16 @@
 // attention to Q, K and V; SPEC section 7 gives the formulas).
 //
 // Two deterministic kernels; neither uses atomics:
-//   dkdv: one CTA per 128-key block. Thread t owns key row t (TMEM lane t). It steps through
+//   dkdv: one CTA per 128-key block, 256 threads: warp w owns TMEM lanes 32(w%4)..+31 (key rows)
+//         and the column half w/4 of every step, so that the element-wise work of a step is
+//         spread over 8 warps. It steps through
 //         the 64-row query blocks that can see the keys:
 //           S^T = K Q^T and dP^T = V dO^T (two MMAs);
 //           P^T = exp2(S^T c - lse2) and dS^T = P^T (dP^T - D) in fp32 registers;
 //           dV += P^T dO and dK += dS^T Q (A from shared memory, K-major; B = dO or Q read
 //           as MN-major operands).
-//   dq:   one CTA per 128-query block. Thread t owns query row t. It steps through the 64-row
-//         key blocks it sees:
+//   dq:   one CTA per 128-query block, 256 threads split the same way (query rows). It steps
+//         through the 64-row key blocks it sees:
 //           S = Q K^T and dP = dO V^T;
 //           dS as above;
 //           dQ += dS K.
@@ -32,7 +34,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // two warpgroups share each step's columns
 constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
 
@@ -99,7 +101,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t t_st = tbase, t_dpt = tbase + 64, t_dv = tbase + 128, t_dk = tbase + 128 + D;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_pt = smem_u32(sm + Ly::PT), s_dst = smem_u32(sm + Ly::DST);
@@ -156,31 +158,29 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   }
   __syncwarp();
 
-  const int row = tid;  // key row within the block = TMEM lane
+  const int row = (warp % 4) * 32 + (tid % 32);  // key row within the block = TMEM lane
+  const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
   const int kj = k0 + row;
   for (int it = 0; it < nit; ++it) {
     const bool ok_s = wait_all(bar + 3, it & 1);
     tc_fence_after();
-    float st[64], dpt[64];
+    float st[32], dpt[32];
     if (ok_s) {
-      uint32_t r[32];
+      uint32_t r0[32], r2[32];
+      tmem_ld32(t_st + lane_off + half * 32, r0);
+      tmem_ld32(t_dpt + lane_off + half * 32, r2);
+      tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(t_st + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) st[c * 32 + e] = __uint_as_float(r[e]);
-        tmem_ld32(t_dpt + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dpt[c * 32 + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 32; ++e) {
+        st[e] = __uint_as_float(r0[e]);
+        dpt[e] = __uint_as_float(r2[e]);
       }
     }
-    const float* l2 = lse2_s + (it & 1) * 64;
-    const float* dl = del_s + (it & 1) * 64;
-    const int q0 = k0 + it * 64;
+    const float* l2 = lse2_s + (it & 1) * 64 + half * 32;
+    const float* dl = del_s + (it & 1) * 64 + half * 32;
+    const int q0 = k0 + it * 64 + half * 32;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
+    for (int c = 0; c < 32; ++c) {
       const bool vis = kj <= q0 + c;
       const float p = vis ? exp2f(st[c] * scale_log2 - l2[c]) : 0.f;
       st[c] = p;
@@ -196,14 +196,15 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       if (it + 1 < nit && it >= 1) load_vec(it + 1);
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {  // 8 chunks of 8 queries, K-major, 128-byte swizzle
+    for (int cc = 0; cc < 4; ++cc) {  // this half's 4 chunks of 8 queries, K-major, 128B swizzle
+      const int c = half * 4 + cc;
       uint32_t wp[4], wq[4], wh[4], wl[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const float u = st[c * 8 + 2 * h], v = st[c * 8 + 2 * h + 1];
+        const float u = st[cc * 8 + 2 * h], v = st[cc * 8 + 2 * h + 1];
         __nv_bfloat162 ph = __floats2bfloat162_rn(u, v);
         __nv_bfloat162 pl = __floats2bfloat162_rn(u - __low2float(ph), v - __high2float(ph));
-        const float x = dpt[c * 8 + 2 * h], y = dpt[c * 8 + 2 * h + 1];
+        const float x = dpt[cc * 8 + 2 * h], y = dpt[cc * 8 + 2 * h + 1];
         __nv_bfloat162 hi = __floats2bfloat162_rn(x, y);
         __nv_bfloat162 lo = __floats2bfloat162_rn(x - __low2float(hi), y - __high2float(hi));
         wp[h] = *reinterpret_cast<uint32_t*>(&ph);
@@ -231,9 +232,10 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     tc_fence_after();
     if (*abort_flag) break;
     if (tid == 0) {
-      issue_acc(it);
+      // the next step's S and dP first: its softmax then overlaps this step's accumulation
       if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
         issue_s(it + 1);
+      issue_acc(it);
     }
     __syncwarp();
   }
@@ -245,7 +247,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     float* dkrow = dK + (size_t)(g0 + kj) * D;
     uint32_t r[32];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int cc = 0; cc < D / 64; ++cc) {
+      const int c = half * (D / 64) + cc;
       tmem_ld32(t_dv + lane_off + c * 32, r);
       tmem_wait_ld();
 #pragma unroll
@@ -322,7 +325,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t t_s = tbase, t_dp = tbase + 64, t_dq = tbase + 128;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_ds = smem_u32(sm + Ly::DS);
@@ -374,31 +377,29 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   }
   __syncwarp();
 
-  const int row = tid;  // query row within the block = TMEM lane
+  const int row = (warp % 4) * 32 + (tid % 32);  // query row within the block = TMEM lane
+  const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
   const int qi = q0 + row;
   const float l2 = lse[g0 + qi] * LOG2E;
   const float dl = delta[g0 + qi];
   for (int it = 0; it < nit; ++it) {
     const bool ok_s = wait_all(bar + 3, it & 1);
     tc_fence_after();
-    float s[64], dp[64];
+    float s[32], dp[32];
     if (ok_s) {
-      uint32_t r[32];
+      uint32_t r0[32], r2[32];
+      tmem_ld32(t_s + lane_off + half * 32, r0);
+      tmem_ld32(t_dp + lane_off + half * 32, r2);
+      tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(t_s + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
-        tmem_ld32(t_dp + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) dp[c * 32 + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 32; ++e) {
+        s[e] = __uint_as_float(r0[e]);
+        dp[e] = __uint_as_float(r2[e]);
       }
     }
-    const int kj0 = it * 64;
+    const int kj0 = it * 64 + half * 32;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
+    for (int c = 0; c < 32; ++c) {
       const bool vis = kj0 + c <= qi;
       const float p = vis ? exp2f(s[c] * scale_log2 - l2) : 0.f;
       dp[c] = p * (dp[c] - dl);
@@ -411,11 +412,12 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       __syncwarp();
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {  // dS = hi + lo, K-major, 128-byte swizzle
+    for (int cc = 0; cc < 4; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
+      const int c = half * 4 + cc;
       uint32_t wh[4], wl[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const float a = dp[c * 8 + 2 * h], b = dp[c * 8 + 2 * h + 1];
+        const float a = dp[cc * 8 + 2 * h], b = dp[cc * 8 + 2 * h + 1];
         __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
         __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
         wh[h] = *reinterpret_cast<uint32_t*>(&hi);
@@ -435,9 +437,10 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     tc_fence_after();
     if (*abort_flag) break;
     if (tid == 0) {
-      issue_acc(it);
+      // the next step's S and dP first: its softmax then overlaps this step's accumulation
       if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
         issue_s(it + 1);
+      issue_acc(it);
     }
     __syncwarp();
   }
@@ -448,7 +451,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     float* dqrow = dQ + (size_t)(g0 + qi) * D;
     uint32_t r[32];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int cc = 0; cc < D / 64; ++cc) {
+      const int c = half * (D / 64) + cc;
       tmem_ld32(t_dq + lane_off + c * 32, r);
       tmem_wait_ld();
 #pragma unroll

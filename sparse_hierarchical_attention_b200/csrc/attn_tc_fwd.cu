@@ -148,13 +148,19 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     __syncwarp();
     // ---- softmax of S_j (row per thread)
     if (ok_s) {
-      uint32_t r[32];
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      const uint32_t ts = tbase + (j & 1) * 128 + lane_off;
+      tmem_ld32(ts, r0);
+      tmem_ld32(ts + 32, r1);
+      tmem_ld32(ts + 64, r2);
+      tmem_ld32(ts + 96, r3);
+      tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        tmem_ld32(tbase + (j & 1) * 128 + lane_off + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * scale_log2;
+      for (int e = 0; e < 32; ++e) {
+        s[e] = __uint_as_float(r0[e]) * scale_log2;
+        s[32 + e] = __uint_as_float(r1[e]) * scale_log2;
+        s[64 + e] = __uint_as_float(r2[e]) * scale_log2;
+        s[96 + e] = __uint_as_float(r3[e]) * scale_log2;
       }
     }
     if (j == qb) {  // diagonal block: key column > query row is invisible

@@ -5,8 +5,9 @@
 // gather: one 16-byte lane per column slice, rows independent, a pure copy.
 // spread: one CTA per (b,h, chunk). The chunk's m row ids become a shared-memory map
 //   (level, cell in chunk) -> subsequence row. Each token then adds the rows that cover it,
-//   one per level at most, in ascending level order, which is ascending subsequence order for
-//   nested spans (SPEC sections 4, 6, 7). fp32 accumulation, one rounding, no atomics.
+//   one per level at most, from the coarsest level down, sharing the partial sums of the
+//   coarse levels among the tokens below them (SPEC sections 6, 7). fp32 accumulation, one
+//   rounding, no atomics.
 #include "common.cuh"
 
 namespace lh {
@@ -56,10 +57,25 @@ struct SpreadArgs {
 };
 
 template <typename E, typename SRC, int D>
+__device__ inline void load_row(const SRC* src, int r, int col, float* x) {
+  constexpr int VEC = 16 / sizeof(E);
+  if constexpr (sizeof(SRC) == sizeof(E)) {
+    Vec<E>::unpack(ldg16(src + (int64_t)r * D + col * VEC), x);
+  } else {  // fp32 source: VEC elements = VEC/4 16-byte loads
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h) Vec<float>::unpack(ldg16(src + (int64_t)r * D + col * VEC + 4 * h), x + 4 * h);
+  }
+}
+
+// One CTA per (b,h, chunk). Covering cells are nested, so each token's sum is formed top-down:
+// a stream of LPR lanes takes a group of p^A tokens (A = 2 when L >= 3), adds the rows of levels
+// L-1..A that cover the whole group once, then the level-1 row once per p tokens, then the
+// token's own level-0 row (SPEC sections 6 and 7: coarsest covering row first).
+template <typename E, typename SRC, int D>
 __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
-  constexpr int VEC = 16 / sizeof(E), LPR = D / VEC;
+  constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, STREAMS = kThreads / LPR;
   extern __shared__ int cmap[];  // (level, cell in chunk) -> subsequence row of this (b,h)
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, col = tid % LPR, stream = tid / LPR;
   const int64_t bh = blockIdx.y, c = blockIdx.x;
   const int L = a.L, p = a.p;
 
@@ -84,33 +100,65 @@ __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
   }
   __syncthreads();
 
-  const int64_t items = a.T * LPR;
-  for (int64_t it = tid; it < items; it += kThreads) {
-    const int tl = (int)(it / LPR), col = (int)(it % LPR);
-    for (int xi = 0; xi < a.ntensor; ++xi) {
-      const SRC* src = static_cast<const SRC*>(a.src[xi]) + bh * a.S * D + col * VEC;
-      float acc[VEC];
+  const int A = L >= 3 ? 2 : L - 1;  // levels handled inside a group
+  const int G = A == 2 ? p * p : (A == 1 ? p : 1);
+  const int ngroups = (int)(a.T / G);
+  for (int xi = 0; xi < a.ntensor; ++xi) {
+    const SRC* src = static_cast<const SRC*>(a.src[xi]) + bh * a.S * D;
+    E* dst = static_cast<E*>(a.dst[xi]) + (bh * a.N + c * a.T) * D + col * VEC;
+    for (int g = stream; g < ngroups; g += STREAMS) {
+      float coarse[VEC];
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-      int cell = tl;
-      for (int l = 0; l < L; ++l) {
-        const int r = cmap[base[l] + cell];
+      for (int e = 0; e < VEC; ++e) coarse[e] = 0.f;
+      // levels L-1 .. A cover the whole group: cell of level l = g / p^(l-A)
+      int cells[16];
+      cells[A] = g;
+      for (int l = A + 1; l < L; ++l) cells[l] = cells[l - 1] / p;
+      for (int l = L - 1; l >= A; --l) {
+        const int r = cmap[base[l] + cells[l]];
         if (r >= 0) {
           float x[VEC];
-          if constexpr (sizeof(SRC) == sizeof(E)) {
-            Vec<E>::unpack(ldg16(src + (int64_t)r * D), x);
-          } else {  // fp32 source, VEC elements = VEC/4 16-byte loads
-#pragma unroll
-            for (int h = 0; h < VEC / 4; ++h) Vec<float>::unpack(ldg16(src + (int64_t)r * D + 4 * h), x + 4 * h);
-          }
+          load_row<E, SRC, D>(src, r, col, x);
           const float w = a.inv[l];
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[e] = __fadd_rn(acc[e], __fmul_rn(x[e], w));
+          for (int e = 0; e < VEC; ++e) coarse[e] = __fadd_rn(coarse[e], __fmul_rn(x[e], w));
         }
-        cell /= p;
       }
-      E* dst = static_cast<E*>(a.dst[xi]) + (bh * a.N + c * a.T + tl) * D + col * VEC;
-      stg16(dst, Vec<E>::pack(acc));
+      const int n1 = A >= 1 ? p : 1;          // level-1 cells in the group (or 1)
+      const int n0 = A == 2 ? p : (A == 1 ? p : 1);  // tokens per level-1 cell
+      for (int c1 = 0; c1 < (A == 2 ? n1 : 1); ++c1) {
+        float part[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) part[e] = coarse[e];
+        if (A == 2) {
+          const int r = cmap[base[1] + g * p + c1];
+          if (r >= 0) {
+            float x[VEC];
+            load_row<E, SRC, D>(src, r, col, x);
+            const float w = a.inv[1];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) part[e] = __fadd_rn(part[e], __fmul_rn(x[e], w));
+          }
+        }
+        const int t0 = A == 2 ? (g * p + c1) * p : g * G;
+        for (int c0 = 0; c0 < (A == 0 ? 1 : n0); ++c0) {
+          const int t = t0 + c0;
+          float out[VEC];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) out[e] = part[e];
+          if (A >= 1) {  // with L = 1 the token is the coarsest level, already in `coarse`
+            const int r = cmap[t];
+            if (r >= 0) {
+              float x[VEC];
+              load_row<E, SRC, D>(src, r, col, x);
+              const float w = a.inv[0];
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(x[e], w));
+            }
+          }
+          stg16(dst + (int64_t)t * D, Vec<E>::pack(out));
+        }
+      }
     }
   }
 }

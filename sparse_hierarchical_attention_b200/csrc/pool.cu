@@ -25,6 +25,13 @@ namespace {
 
 constexpr int kThreads = 256;
 enum { MODE_PYRAMID = 0, MODE_SPANSUM = 1 };
+// Rows fetched ahead per thread, and the CTAs per SM the register budget is sized for.
+#ifndef LH_POOL_UNROLL
+#define LH_POOL_UNROLL 4
+#endif
+#ifndef LH_POOL_MINB
+#define LH_POOL_MINB 2
+#endif
 
 struct PoolArgs {
   const void* x[3];  // q, k, v (pyramid) or d_o (span sums)
@@ -63,7 +70,7 @@ __device__ inline void decode_rid(int64_t rid, const int64_t* off, int L, int& l
 }
 
 template <typename E, int D, int A, int MODE>
-__global__ void __launch_bounds__(kThreads) pool_tile_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const PoolArgs a) {
   using V = Vec<E>;
   constexpr int VEC = V::N, LPR = D / VEC, STREAMS = kThreads / LPR;
   constexpr int NX = MODE == MODE_PYRAMID ? 3 : 1;
@@ -151,16 +158,27 @@ __global__ void __launch_bounds__(kThreads) pool_tile_kernel(const PoolArgs a) {
 #pragma unroll
   for (int xi = 0; xi < NX; ++xi) X[xi] = static_cast<const E*>(a.x[xi]);
 
+  // Rows are fetched U at a time (3U x 16 bytes in flight per thread), then processed.
+  constexpr int U = LH_POOL_UNROLL;
 #pragma unroll 1
-  for (int row = 0; row < W; ++row) {
+  for (int row0 = 0; row0 < W; row0 += U) {
+    uint4 raw[U][NX];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int xi = 0; xi < NX; ++xi) {
+        raw[u][xi] = make_uint4(0, 0, 0, 0);
+        if (active && xi < nx && row0 + u < W)
+          raw[u][xi] = ldg16(X[xi] + (bh * a.N + tok0 + row0 + u) * D + col * VEC);
+      }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int row = row0 + u;
+    if (row >= W) break;  // the same for every thread of the CTA
     const int64_t t = tok0 + row;
     float x[NX][VEC];
 #pragma unroll
-    for (int xi = 0; xi < NX; ++xi) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (active && xi < nx) u = ldg16(X[xi] + (bh * a.N + t) * D + col * VEC);
-      V::unpack(u, x[xi]);
-    }
+    for (int xi = 0; xi < NX; ++xi) V::unpack(raw[u][xi], x[xi]);
     float nq = 0.f, nk = 0.f;
     if (MODE == MODE_PYRAMID && a.do_score) {
       nq = row_norm<VEC, LPR>(x[0]);
@@ -213,6 +231,7 @@ __global__ void __launch_bounds__(kThreads) pool_tile_kernel(const PoolArgs a) {
         mk[l - 1] = 0.f;
       }
     }
+  }
   }
   if (A == 0 || (a.U == 0 && a.A2 >= a.L - 1)) return;
   __syncthreads();
