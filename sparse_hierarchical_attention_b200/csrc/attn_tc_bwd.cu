@@ -21,8 +21,10 @@
 // and dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That
 // is one extra MMA per product and keeps the operand to ~16 bits. With one bf16 term, single
 // dV elements were off by 34% of their size.
-// Q/dO (dkdv) and K/V (dq) come through two-stage TMA rings. S and dP live in TMEM and are
-// reused every step; accumulators stay in TMEM until the epilogue writes fp32 results.
+// Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, and S/dP are double-buffered in
+// TMEM, so the S/dP MMAs of step it+1 are issued at the start of step it: the tensor cores work
+// on them (and on step it-1's accumulation) while the warps do step it's element-wise part.
+// Accumulators stay in TMEM until the epilogue writes fp32 results.
 // All waits are bounded and report through the status word.
 #include "tc.cuh"
 
@@ -44,17 +46,16 @@ struct LayDKV {
   static constexpr int KB = D / 64;
   static constexpr int K = 0;                     // [128][D]
   static constexpr int V = K + KB * T128;         // [128][D]
-  static constexpr int Q = V + KB * T128;         // 2 stages of [64][D]
-  static constexpr int DO = Q + 2 * KB * T64;     // 2 stages of [64][D]
-  static constexpr int PT = DO + 2 * KB * T64;    // hi, lo: [128 keys][64 queries] each
+  static constexpr int Q = V + KB * T128;         // 3 stages of [64][D]
+  static constexpr int DO = Q + 3 * KB * T64;     // 3 stages of [64][D]
+  static constexpr int PT = DO + 3 * KB * T64;    // hi, lo: [128 keys][64 queries] each
   static constexpr int DST = PT + 2 * T128;       // hi, lo: [128 keys][64 queries] each
   static constexpr int VEC = DST + 2 * T128;      // lse2[2][64], delta[2][64]
   static constexpr int BAR = VEC + 4 * 64 * 4;
   static constexpr int BYTES = BAR + 128;
-  static constexpr uint32_t TMEM_COLS = D == 128 ? 512 : 256;
 };
 
-// bars: 0 K+V, 1-2 Q/dO stages, 3 S^T+dP^T, 4 dV+dK
+// bars: 0 K+V, 1-3 Q/dO stages, 4-5 S^T+dP^T buffers, 6 dV+dK
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -86,7 +87,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     fence_barrier_init();
     prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
   }
-  if (warp == 0) tmem_alloc(tmem_slot, Ly::TMEM_COLS);
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
   auto load_vec = [&](int it) {  // lse2 and delta of query block it into stage it & 1
     if (tid < 64) {
       const int qi = g0 + k0 + it * 64 + tid;
@@ -100,7 +101,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t t_st = tbase, t_dpt = tbase + 64, t_dv = tbase + 128, t_dk = tbase + 128 + D;
+  // S^T / dP^T buffer b at columns 128b / 128b + 64; dV at 256, dK at 256 + D
+  const uint32_t t_dv = tbase + 256, t_dk = tbase + 256 + D;
   const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
@@ -108,26 +110,28 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  auto load_qdo = [&](int it) {
-    uint64_t* b = bar + 1 + (it & 1);
+  auto load_qdo = [&](int it) {  // into stage it % 3
+    const int sg = it % 3;
+    uint64_t* b = bar + 1 + sg;
     mbar_expect_tx(b, 2 * KB * T64);
     for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::Q + (it & 1) * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
-      tma_load_2d(sm + Ly::DO + (it & 1) * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
+      tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
+      tma_load_2d(sm + Ly::DO + sg * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
     }
   };
-  auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T
-    const uint32_t qb = s_q + (it & 1) * KB * T64, ob = s_do + (it & 1) * KB * T64;
+  auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T into TMEM buffer it & 1
+    const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
+    const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
       mma_ss(t_st, sw128_desc(s_k + offA, 16, 1024), sw128_desc(qb + offB, 16, 1024), IDESC_S, ks > 0);
       mma_ss(t_dpt, sw128_desc(s_v + offA, 16, 1024), sw128_desc(ob + offB, 16, 1024), IDESC_S, ks > 0);
     }
-    mma_commit(bar + 3);
+    mma_commit(bar + 4 + (it & 1));
   };
   auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
-    const uint32_t qb = s_q + (it & 1) * KB * T64, ob = s_do + (it & 1) * KB * T64;
+    const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       mma_ss(t_dv, sw128_desc(s_pt + ks * 32, 16, 1024), sw128_desc(ob + ks * 2048, T64, 1024),
@@ -139,7 +143,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       mma_ss(t_dk, sw128_desc(s_dst + T128 + ks * 32, 16, 1024), sw128_desc(qb + ks * 2048, T64, 1024),
              IDESC_ACC, 1u);
     }
-    mma_commit(bar + 4);
+    mma_commit(bar + 6);
   };
   auto wait_all = [&](uint64_t* b, uint32_t parity) {
     bool ok = mbar_wait(b, parity, abort_flag, status);
@@ -152,8 +156,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
       tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
     }
-    load_qdo(0);
-    if (nit > 1) load_qdo(1);
+    for (int i = 0; i < 3 && i < nit; ++i) load_qdo(i);
     if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
   }
   __syncwarp();
@@ -162,11 +165,16 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
   const int kj = k0 + row;
   for (int it = 0; it < nit; ++it) {
-    const bool ok_s = wait_all(bar + 3, it & 1);
+    const bool ok_s = wait_all(bar + 4 + (it & 1), (it >> 1) & 1);
     tc_fence_after();
+    if (tid == 0 && ok_s && it + 1 < nit &&
+        mbar_wait(bar + 1 + (it + 1) % 3, ((it + 1) / 3) & 1, abort_flag, status))
+      issue_s(it + 1);  // the other buffer: its previous step was read before the last barrier
+    __syncwarp();
     float st[32], dpt[32];
     if (ok_s) {
       uint32_t r0[32], r2[32];
+      const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
       tmem_ld32(t_st + lane_off + half * 32, r0);
       tmem_ld32(t_dpt + lane_off + half * 32, r2);
       tmem_wait_ld();
@@ -176,24 +184,34 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         dpt[e] = __uint_as_float(r2[e]);
       }
     }
-    const float* l2 = lse2_s + (it & 1) * 64 + half * 32;
-    const float* dl = del_s + (it & 1) * 64 + half * 32;
+    const float4* l2 = reinterpret_cast<const float4*>(lse2_s + (it & 1) * 64 + half * 32);
+    const float4* dl = reinterpret_cast<const float4*>(del_s + (it & 1) * 64 + half * 32);
     const int q0 = k0 + it * 64 + half * 32;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const bool vis = kj <= q0 + c;
-      const float p = vis ? exp2f(st[c] * scale_log2 - l2[c]) : 0.f;
-      st[c] = p;
-      dpt[c] = p * (dpt[c] - dl[c]);
+    for (int c4 = 0; c4 < 8; ++c4) {
+      const float4 lv = l2[c4], dv = dl[c4];
+      const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = c4 * 4 + e;
+        const float p = ex2(fmaf(st[c], scale_log2, -la[e]));
+        st[c] = p;
+        dpt[c] = p * (dpt[c] - da[e]);
+      }
     }
-    // the accumulate MMAs of the previous step read P^T, dS^T and the other Q/dO stage
+    if (q0 < k0 + 128) {  // steps that reach the diagonal: keys after the query are invisible
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
+    }
+    // the accumulate MMAs of the previous step read P^T, dS^T and Q/dO stage (it-1) % 3
     bool ok_m = true;
     if (it > 0) {
-      ok_m = wait_all(bar + 4, (it - 1) & 1);
+      ok_m = wait_all(bar + 6, (it - 1) & 1);
       tc_fence_after();
-      if (tid == 0 && ok_m && it + 1 < nit && it >= 1) load_qdo(it + 1);
+      if (tid == 0 && ok_m && it + 2 < nit) load_qdo(it + 2);  // into stage (it-1) % 3
       __syncwarp();
-      if (it + 1 < nit && it >= 1) load_vec(it + 1);
+      if (it + 1 < nit) load_vec(it + 1);
     }
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {  // this half's 4 chunks of 8 queries, K-major, 128B swizzle
@@ -201,16 +219,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       uint32_t wp[4], wq[4], wh[4], wl[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const float u = st[cc * 8 + 2 * h], v = st[cc * 8 + 2 * h + 1];
-        __nv_bfloat162 ph = __floats2bfloat162_rn(u, v);
-        __nv_bfloat162 pl = __floats2bfloat162_rn(u - __low2float(ph), v - __high2float(ph));
-        const float x = dpt[cc * 8 + 2 * h], y = dpt[cc * 8 + 2 * h + 1];
-        __nv_bfloat162 hi = __floats2bfloat162_rn(x, y);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(x - __low2float(hi), y - __high2float(hi));
-        wp[h] = *reinterpret_cast<uint32_t*>(&ph);
-        wq[h] = *reinterpret_cast<uint32_t*>(&pl);
-        wh[h] = *reinterpret_cast<uint32_t*>(&hi);
-        wl[h] = *reinterpret_cast<uint32_t*>(&lo);
+        split_bf16x2(st[cc * 8 + 2 * h], st[cc * 8 + 2 * h + 1], wp[h], wq[h]);
+        split_bf16x2(dpt[cc * 8 + 2 * h], dpt[cc * 8 + 2 * h + 1], wh[h], wl[h]);
       }
       const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
       asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_pt + off), "r"(wp[0]), "r"(wp[1]),
@@ -231,16 +241,11 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     if (*abort_flag) break;
-    if (tid == 0) {
-      // the next step's S and dP first: its softmax then overlaps this step's accumulation
-      if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
-        issue_s(it + 1);
-      issue_acc(it);
-    }
+    if (tid == 0) issue_acc(it);
     __syncwarp();
   }
 
-  const bool ok_end = !*abort_flag && wait_all(bar + 4, (nit - 1) & 1);
+  const bool ok_end = !*abort_flag && wait_all(bar + 6, (nit - 1) & 1);
   tc_fence_after();
   if (ok_end) {
     float* dvrow = dV + (size_t)(g0 + kj) * D;
@@ -273,7 +278,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     }
   }
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tbase, Ly::TMEM_COLS);
+  if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
 // ------------------------------------------------------------------------------------ dQ
@@ -282,14 +287,14 @@ struct LayDQ {
   static constexpr int KB = D / 64;
   static constexpr int Q = 0;                    // [128][D]
   static constexpr int DO = Q + KB * T128;       // [128][D]
-  static constexpr int K = DO + KB * T128;       // 2 stages of [64][D]
-  static constexpr int V = K + 2 * KB * T64;     // 2 stages of [64][D]
-  static constexpr int DS = V + 2 * KB * T64;    // hi, lo: [128 queries][64 keys] each
+  static constexpr int K = DO + KB * T128;       // 3 stages of [64][D]
+  static constexpr int V = K + 3 * KB * T64;     // 3 stages of [64][D]
+  static constexpr int DS = V + 3 * KB * T64;    // hi, lo: [128 queries][64 keys] each
   static constexpr int BAR = DS + 2 * T128;
   static constexpr int BYTES = BAR + 128;
 };
 
-// bars: 0 Q+dO, 1-2 K/V stages, 3 S+dP, 4 dQ
+// bars: 0 Q+dO, 1-3 K/V stages, 4-5 S+dP buffers, 6 dQ
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -319,12 +324,13 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     fence_barrier_init();
     prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
   }
-  if (warp == 0) tmem_alloc(tmem_slot, 256);
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t t_s = tbase, t_dp = tbase + 64, t_dq = tbase + 128;
+  // S / dP buffer b at columns 128b / 128b + 64; dQ at 256
+  const uint32_t t_dq = tbase + 256;
   const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
@@ -332,33 +338,35 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  auto load_kv = [&](int it) {
-    uint64_t* b = bar + 1 + (it & 1);
+  auto load_kv = [&](int it) {  // into stage it % 3
+    const int sg = it % 3;
+    uint64_t* b = bar + 1 + sg;
     mbar_expect_tx(b, 2 * KB * T64);
     for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::K + (it & 1) * KB * T64 + c * T64, &tk, c * 64, g0 + it * 64, b);
-      tma_load_2d(sm + Ly::V + (it & 1) * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
+      tma_load_2d(sm + Ly::K + sg * KB * T64 + c * T64, &tk, c * 64, g0 + it * 64, b);
+      tma_load_2d(sm + Ly::V + sg * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
     }
   };
-  auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T
-    const uint32_t kbs = s_k + (it & 1) * KB * T64, vbs = s_v + (it & 1) * KB * T64;
+  auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T into TMEM buffer it & 1
+    const uint32_t kbs = s_k + (it % 3) * KB * T64, vbs = s_v + (it % 3) * KB * T64;
+    const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
       mma_ss(t_s, sw128_desc(s_q + offA, 16, 1024), sw128_desc(kbs + offB, 16, 1024), IDESC_S, ks > 0);
       mma_ss(t_dp, sw128_desc(s_do + offA, 16, 1024), sw128_desc(vbs + offB, 16, 1024), IDESC_S, ks > 0);
     }
-    mma_commit(bar + 3);
+    mma_commit(bar + 4 + (it & 1));
   };
   auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
-    const uint32_t kbs = s_k + (it & 1) * KB * T64;
+    const uint32_t kbs = s_k + (it % 3) * KB * T64;
 #pragma unroll
     for (int part = 0; part < 2; ++part)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         mma_ss(t_dq, sw128_desc(s_ds + part * T128 + ks * 32, 16, 1024),
                sw128_desc(kbs + ks * 2048, T64, 1024), IDESC_ACC, (it > 0 || part > 0 || ks > 0) ? 1u : 0u);
-    mma_commit(bar + 4);
+    mma_commit(bar + 6);
   };
   auto wait_all = [&](uint64_t* b, uint32_t parity) {
     bool ok = mbar_wait(b, parity, abort_flag, status);
@@ -371,8 +379,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
       tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
     }
-    load_kv(0);
-    if (nit > 1) load_kv(1);
+    for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
     if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
   }
   __syncwarp();
@@ -383,11 +390,16 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   const float l2 = lse[g0 + qi] * LOG2E;
   const float dl = delta[g0 + qi];
   for (int it = 0; it < nit; ++it) {
-    const bool ok_s = wait_all(bar + 3, it & 1);
+    const bool ok_s = wait_all(bar + 4 + (it & 1), (it >> 1) & 1);
     tc_fence_after();
+    if (tid == 0 && ok_s && it + 1 < nit &&
+        mbar_wait(bar + 1 + (it + 1) % 3, ((it + 1) / 3) & 1, abort_flag, status))
+      issue_s(it + 1);  // the other buffer: its previous step was read before the last barrier
+    __syncwarp();
     float s[32], dp[32];
     if (ok_s) {
       uint32_t r0[32], r2[32];
+      const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
       tmem_ld32(t_s + lane_off + half * 32, r0);
       tmem_ld32(t_dp + lane_off + half * 32, r2);
       tmem_wait_ld();
@@ -399,16 +411,17 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
     const int kj0 = it * 64 + half * 32;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const bool vis = kj0 + c <= qi;
-      const float p = vis ? exp2f(s[c] * scale_log2 - l2) : 0.f;
-      dp[c] = p * (dp[c] - dl);
+    for (int c = 0; c < 32; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
+    if (kj0 + 32 > q0) {  // steps that reach the diagonal: keys after the query are invisible
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (kj0 + c > qi) dp[c] = 0.f;
     }
     bool ok_m = true;
     if (it > 0) {
-      ok_m = wait_all(bar + 4, (it - 1) & 1);
+      ok_m = wait_all(bar + 6, (it - 1) & 1);
       tc_fence_after();
-      if (tid == 0 && ok_m && it + 1 < nit && it >= 1) load_kv(it + 1);
+      if (tid == 0 && ok_m && it + 2 < nit) load_kv(it + 2);  // into stage (it-1) % 3
       __syncwarp();
     }
 #pragma unroll
@@ -416,13 +429,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       const int c = half * 4 + cc;
       uint32_t wh[4], wl[4];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float a = dp[cc * 8 + 2 * h], b = dp[cc * 8 + 2 * h + 1];
-        __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
-        wh[h] = *reinterpret_cast<uint32_t*>(&hi);
-        wl[h] = *reinterpret_cast<uint32_t*>(&lo);
-      }
+      for (int h = 0; h < 4; ++h) split_bf16x2(dp[cc * 8 + 2 * h], dp[cc * 8 + 2 * h + 1], wh[h], wl[h]);
       const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
       asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_ds + off), "r"(wh[0]), "r"(wh[1]),
                    "r"(wh[2]), "r"(wh[3])
@@ -436,16 +443,11 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     if (*abort_flag) break;
-    if (tid == 0) {
-      // the next step's S and dP first: its softmax then overlaps this step's accumulation
-      if (it + 1 < nit && mbar_wait(bar + 1 + ((it + 1) & 1), ((it + 1) >> 1) & 1, abort_flag, status))
-        issue_s(it + 1);
-      issue_acc(it);
-    }
+    if (tid == 0) issue_acc(it);
     __syncwarp();
   }
 
-  const bool ok_end = !*abort_flag && wait_all(bar + 4, (nit - 1) & 1);
+  const bool ok_end = !*abort_flag && wait_all(bar + 6, (nit - 1) & 1);
   tc_fence_after();
   if (ok_end) {
     float* dqrow = dQ + (size_t)(g0 + qi) * D;
@@ -470,7 +472,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
   }
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tbase, 256);
+  if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
 // D_i = dO_sub[i] . O_sub[i] (fp32 O_sub); one warp per row.
@@ -510,13 +512,14 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
   if (e != cudaSuccess) return e;
   const float sigma = 1.0f / sqrtf((float)D);
   const float scale_log2 = sigma * 1.4426950408889634f;
-  const int smem1 = LayDKV<D>::BYTES + 1024;
+  const int smem1 = LayDKV<D>::BYTES + 1024 > 120 * 1024 ? LayDKV<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
   attn_bwd_dkdv_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem1, st>>>(
       k128, v128, q64, do64, lse, delta, dk, dv, g.S, sigma, scale_log2, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int smem2 = LayDQ<D>::BYTES + 1024;
+  // both kernels hold all 512 TMEM columns: padded so that two CTAs never share an SM
+  const int smem2 = LayDQ<D>::BYTES + 1024 > 120 * 1024 ? LayDQ<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
   if (e != cudaSuccess) return e;
   attn_bwd_dq_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem2, st>>>(

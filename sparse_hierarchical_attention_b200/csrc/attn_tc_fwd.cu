@@ -177,7 +177,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     float sum = 0.f;
 #pragma unroll
     for (int e = 0; e < BN; ++e) {
-      s[e] = exp2f(s[e] - m_new);
+      s[e] = ex2(s[e] - m_new);
       sum += s[e];
     }
     l = l * alpha + sum;
@@ -207,13 +207,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     for (int c = 0; c < BN / 8; ++c) {
       uint32_t wh[4], wl[4];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float a = s[c * 8 + 2 * h], b = s[c * 8 + 2 * h + 1];
-        __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
-        __nv_bfloat162 lo = __floats2bfloat162_rn(a - __low2float(hi), b - __high2float(hi));
-        wh[h] = *reinterpret_cast<uint32_t*>(&hi);
-        wl[h] = *reinterpret_cast<uint32_t*>(&lo);
-      }
+      for (int h = 0; h < 4; ++h) split_bf16x2(s[c * 8 + 2 * h], s[c * 8 + 2 * h + 1], wh[h], wl[h]);
       const uint32_t addr = s_p + (c / 8) * TILE + row * 128 + (((c % 8) ^ (row % 8)) * 16);
       asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(wh[0]), "r"(wh[1]),
                    "r"(wh[2]), "r"(wh[3])

@@ -173,5 +173,23 @@ __device__ inline void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// 2^x with the hardware approximation (flush-to-zero; relative error ~2^-22), for softmax
+// weights that are then rounded to bf16 pairs.
+__device__ inline float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (a, b) -> hi = bf16x2(a, b) and lo = bf16x2(a - hi.a, b - hi.b): a two-term bf16 split that
+// carries ~16 bits of each value.
+__device__ inline void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xffff0000u);
+  __nv_bfloat162 l = __floats2bfloat162_rn(a - ha, b - hb);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 }  // namespace tc
 }  // namespace lh
