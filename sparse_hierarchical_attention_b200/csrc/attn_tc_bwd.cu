@@ -3,29 +3,27 @@
 // attention to Q, K and V; SPEC section 7 gives the formulas).
 //
 // Two deterministic kernels; neither uses atomics:
-//   dkdv: one CTA per 128-key block, 256 threads: warp w owns TMEM lanes 32(w%4)..+31 (key rows)
-//         and the column half w/4 of every step, so that the element-wise work of a step is
-//         spread over 8 warps. It steps through
-//         the 64-row query blocks that can see the keys:
-//           S^T = K Q^T and dP^T = V dO^T (two MMAs);
+//   dkdv: one CTA per 128-key block steps through the 64-row query blocks that can see the keys:
+//           S^T = K Q^T and dP^T = V dO^T;
 //           P^T = exp2(S^T c - lse2) and dS^T = P^T (dP^T - D) in fp32 registers;
-//           dV += P^T dO and dK += dS^T Q (A from shared memory, K-major; B = dO or Q read
-//           as MN-major operands).
-//   dq:   one CTA per 128-query block, 256 threads split the same way (query rows). It steps
-//         through the 64-row key blocks it sees:
-//           S = Q K^T and dP = dO V^T;
-//           dS as above;
-//           dQ += dS K.
+//           dV += P^T dO and dK += dS^T Q (A operands from shared memory, K-major; B = dO or Q
+//           read as MN-major operands).
+//   dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
+//           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K.
+// Warp roles: warps 0-7 compute (warp w owns TMEM lanes 32(w%4)..+31 and column half w/4 of each
+// step); warp 8, lane 0, is the producer: it issues every TMA load and every MMA. The two sides
+// meet only at mbarriers (S ready, S buffer free, P written, accumulation done), so the tensor
+// cores work on step it+1's S/dP and step it-1's accumulation while the warps do step it.
+// Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, with lse and D riding along as
+// 1-D bulk copies; S/dP are double-buffered in TMEM; accumulators stay in TMEM until the
+// epilogue writes fp32 results.
 // dQ, dK and dV all sum P or dS against rows with mixed signs. Coarse rows carry dO_sub that
-// sums thousands of tokens, and there those sums cancel by orders of magnitude. So P^T, dS^T
-// and dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That
-// is one extra MMA per product and keeps the operand to ~16 bits. With one bf16 term, single
-// dV elements were off by 34% of their size.
-// Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, and S/dP are double-buffered in
-// TMEM, so the S/dP MMAs of step it+1 are issued at the start of step it: the tensor cores work
-// on them (and on step it-1's accumulation) while the warps do step it's element-wise part.
-// Accumulators stay in TMEM until the epilogue writes fp32 results.
-// All waits are bounded and report through the status word.
+// sums thousands of tokens, and there those sums cancel by orders of magnitude. So P^T, dS^T and
+// dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That is
+// one extra MMA per product and keeps the operand to ~16 bits. With one bf16 term, single dV
+// elements were off by 34% of their size.
+// Every barrier that could run two phases ahead of a waiter is doubled, so that no parity wait
+// is ambiguous. All waits are bounded and report through the status word.
 #include "tc.cuh"
 
 namespace lh {
@@ -36,9 +34,17 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 256;  // two warpgroups share each step's columns
+constexpr int kCompute = 256;              // warps 0-7
+constexpr int kThreads = kCompute + 32;    // + the producer warp
 constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ inline void store_pair4(uint32_t addr, const uint32_t (&w)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3])
+               : "memory");
+}
 
 // ------------------------------------------------------------------------------------ dK, dV
 template <int D>
@@ -50,12 +56,12 @@ struct LayDKV {
   static constexpr int DO = Q + 3 * KB * T64;     // 3 stages of [64][D]
   static constexpr int PT = DO + 3 * KB * T64;    // hi, lo: [128 keys][64 queries] each
   static constexpr int DST = PT + 2 * T128;       // hi, lo: [128 keys][64 queries] each
-  static constexpr int VEC = DST + 2 * T128;      // lse2[2][64], delta[2][64]
-  static constexpr int BAR = VEC + 4 * 64 * 4;
+  static constexpr int VEC = DST + 2 * T128;      // 3 stages of lse[64], delta[64]
+  static constexpr int BAR = VEC + 3 * 512;
   static constexpr int BYTES = BAR + 128;
 };
 
-// bars: 0 K+V, 1-3 Q/dO stages, 4-5 S^T+dP^T buffers, 6 dV+dK
+// bars: 0 K+V | 1-3 Q/dO stages | 4-5 S buffers | 6-7 S buffers free | 8 P written | 9-10 acc
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -68,10 +74,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 8) + 1;
-  float* lse2_s = reinterpret_cast<float*>(sm + Ly::VEC);  // [2][64]
-  float* del_s = lse2_s + 128;                             // [2][64]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int kb = blockIdx.x;  // low key blocks see the most queries: they start first
@@ -79,200 +83,189 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   const int g0 = bh * S;
   const int k0 = kb * 128;
   const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
-  const float LOG2E = 1.4426950408889634f;
 
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bar + i, 1);
+    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute : 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
   }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
-  auto load_vec = [&](int it) {  // lse2 and delta of query block it into stage it & 1
-    if (tid < 64) {
-      const int qi = g0 + k0 + it * 64 + tid;
-      lse2_s[(it & 1) * 64 + tid] = lse[qi] * LOG2E;
-      del_s[(it & 1) * 64 + tid] = delta[qi];
-    }
-  };
-  load_vec(0);
-  if (nit > 1) load_vec(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   // S^T / dP^T buffer b at columns 128b / 128b + 64; dV at 256, dK at 256 + D
   const uint32_t t_dv = tbase + 256, t_dk = tbase + 256 + D;
-  const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_pt = smem_u32(sm + Ly::PT), s_dst = smem_u32(sm + Ly::DST);
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  auto load_qdo = [&](int it) {  // into stage it % 3
-    const int sg = it % 3;
-    uint64_t* b = bar + 1 + sg;
-    mbar_expect_tx(b, 2 * KB * T64);
-    for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
-      tma_load_2d(sm + Ly::DO + sg * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
-    }
-  };
-  auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T into TMEM buffer it & 1
-    const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
-    const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
+  if (warp == 8) {
+    // ------------------------------------------------------------------ producer
+    if ((tid % 32) == 0) {
+      prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
+      auto load_stage = [&](int it) {  // Q, dO, lse, D of query block it into stage it % 3
+        const int sg = it % 3;
+        uint64_t* b = bar + 1 + sg;
+        mbar_expect_tx(b, 2 * KB * T64 + 512);
+        for (int c = 0; c < KB; ++c) {
+          tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
+          tma_load_2d(sm + Ly::DO + sg * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
+        }
+        bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + k0 + it * 64, 256, b);
+        bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + k0 + it * 64, 256, b);
+      };
+      auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T into TMEM buffer it & 1
+        const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
+        const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
-      mma_ss(t_st, sw128_desc(s_k + offA, 16, 1024), sw128_desc(qb + offB, 16, 1024), IDESC_S, ks > 0);
-      mma_ss(t_dpt, sw128_desc(s_v + offA, 16, 1024), sw128_desc(ob + offB, 16, 1024), IDESC_S, ks > 0);
-    }
-    mma_commit(bar + 4 + (it & 1));
-  };
-  auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
-    const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
+          mma_ss(t_st, sw128_desc(s_k + offA, 16, 1024), sw128_desc(qb + offB, 16, 1024), IDESC_S, ks > 0);
+          mma_ss(t_dpt, sw128_desc(s_v + offA, 16, 1024), sw128_desc(ob + offB, 16, 1024), IDESC_S, ks > 0);
+        }
+        mma_commit(bar + 4 + (it & 1));
+      };
+      auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
+        const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      mma_ss(t_dv, sw128_desc(s_pt + ks * 32, 16, 1024), sw128_desc(ob + ks * 2048, T64, 1024),
-             IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-      mma_ss(t_dv, sw128_desc(s_pt + T128 + ks * 32, 16, 1024), sw128_desc(ob + ks * 2048, T64, 1024),
-             IDESC_ACC, 1u);
-      mma_ss(t_dk, sw128_desc(s_dst + ks * 32, 16, 1024), sw128_desc(qb + ks * 2048, T64, 1024),
-             IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-      mma_ss(t_dk, sw128_desc(s_dst + T128 + ks * 32, 16, 1024), sw128_desc(qb + ks * 2048, T64, 1024),
-             IDESC_ACC, 1u);
-    }
-    mma_commit(bar + 6);
-  };
-  auto wait_all = [&](uint64_t* b, uint32_t parity) {
-    bool ok = mbar_wait(b, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, ok);
-  };
-
-  if (tid == 0) {
-    mbar_expect_tx(bar, 2 * KB * T128);
-    for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
-      tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
-    }
-    for (int i = 0; i < 3 && i < nit; ++i) load_qdo(i);
-    if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
-  }
-  __syncwarp();
-
-  const int row = (warp % 4) * 32 + (tid % 32);  // key row within the block = TMEM lane
-  const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
-  const int kj = k0 + row;
-  for (int it = 0; it < nit; ++it) {
-    const bool ok_s = wait_all(bar + 4 + (it & 1), (it >> 1) & 1);
-    tc_fence_after();
-    if (tid == 0 && ok_s && it + 1 < nit &&
-        mbar_wait(bar + 1 + (it + 1) % 3, ((it + 1) / 3) & 1, abort_flag, status))
-      issue_s(it + 1);  // the other buffer: its previous step was read before the last barrier
-    __syncwarp();
-    float st[32], dpt[32];
-    if (ok_s) {
-      uint32_t r0[32], r2[32];
-      const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
-      tmem_ld32(t_st + lane_off + half * 32, r0);
-      tmem_ld32(t_dpt + lane_off + half * 32, r2);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        st[e] = __uint_as_float(r0[e]);
-        dpt[e] = __uint_as_float(r2[e]);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bq = sw128_desc(qb + ks * 2048, T64, 1024), bo = sw128_desc(ob + ks * 2048, T64, 1024);
+          mma_ss(t_dv, sw128_desc(s_pt + ks * 32, 16, 1024), bo, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dv, sw128_desc(s_pt + T128 + ks * 32, 16, 1024), bo, IDESC_ACC, 1u);
+          mma_ss(t_dk, sw128_desc(s_dst + ks * 32, 16, 1024), bq, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dk, sw128_desc(s_dst + T128 + ks * 32, 16, 1024), bq, IDESC_ACC, 1u);
+        }
+        mma_commit(bar + 9 + (it & 1));
+      };
+      mbar_expect_tx(bar, 2 * KB * T128);
+      for (int c = 0; c < KB; ++c) {
+        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
+        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
+      }
+      for (int i = 0; i < 3 && i < nit; ++i) load_stage(i);
+      bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
+      if (ok) issue_s(0);
+      for (int it = 0; it < nit && ok; ++it) {
+        if (it + 1 < nit) {  // next step's S/dP into the other buffer once it is free
+          const int n = it + 1;
+          ok = mbar_wait(bar + 1 + n % 3, (n / 3) & 1, abort_flag, status);
+          if (ok && n >= 2) ok = mbar_wait(bar + 6 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(n);
+        }
+        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
+        tc_fence_after();
+        issue_acc(it);
+        if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
+          if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
+          load_stage(it + 2);
+        }
       }
     }
-    const float4* l2 = reinterpret_cast<const float4*>(lse2_s + (it & 1) * 64 + half * 32);
-    const float4* dl = reinterpret_cast<const float4*>(del_s + (it & 1) * 64 + half * 32);
-    const int q0 = k0 + it * 64 + half * 32;
-#pragma unroll
-    for (int c4 = 0; c4 < 8; ++c4) {
-      const float4 lv = l2[c4], dv = dl[c4];
-      const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = c4 * 4 + e;
-        const float p = ex2(fmaf(st[c], scale_log2, -la[e]));
-        st[c] = p;
-        dpt[c] = p * (dpt[c] - da[e]);
-      }
-    }
-    if (q0 < k0 + 128) {  // steps that reach the diagonal: keys after the query are invisible
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
-    }
-    // the accumulate MMAs of the previous step read P^T, dS^T and Q/dO stage (it-1) % 3
-    bool ok_m = true;
-    if (it > 0) {
-      ok_m = wait_all(bar + 6, (it - 1) & 1);
+  } else {
+    // ------------------------------------------------------------------ compute warps
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
+    const int row = (warp % 4) * 32 + (tid % 32);  // key row within the block = TMEM lane
+    const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
+    const int kj = k0 + row;
+    auto wait_all = [&](uint64_t* b, uint32_t parity) {
+      bool ok = mbar_wait(b, parity, abort_flag, status);
+      return __all_sync(0xffffffffu, ok);
+    };
+    for (int it = 0; it < nit; ++it) {
+      if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
+      if (!wait_all(bar + 1 + it % 3, (it / 3) & 1)) break;  // lse, D of this step (visibility)
       tc_fence_after();
-      if (tid == 0 && ok_m && it + 2 < nit) load_qdo(it + 2);  // into stage (it-1) % 3
-      __syncwarp();
-      if (it + 1 < nit) load_vec(it + 1);
-    }
+      float st[32], dpt[32];
+      {
+        uint32_t r0[32], r2[32];
+        const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
+        tmem_ld32(t_st + lane_off + half * 32, r0);
+        tmem_ld32(t_dpt + lane_off + half * 32, r2);
+        tmem_wait_ld();
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {  // this half's 4 chunks of 8 queries, K-major, 128B swizzle
-      const int c = half * 4 + cc;
-      uint32_t wp[4], wq[4], wh[4], wl[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        split_bf16x2(st[cc * 8 + 2 * h], st[cc * 8 + 2 * h + 1], wp[h], wq[h]);
-        split_bf16x2(dpt[cc * 8 + 2 * h], dpt[cc * 8 + 2 * h + 1], wh[h], wl[h]);
+        for (int e = 0; e < 32; ++e) {
+          st[e] = __uint_as_float(r0[e]);
+          dpt[e] = __uint_as_float(r2[e]);
+        }
       }
-      const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_pt + off), "r"(wp[0]), "r"(wp[1]),
-                   "r"(wp[2]), "r"(wp[3])
-                   : "memory");
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_pt + T128 + off), "r"(wq[0]),
-                   "r"(wq[1]), "r"(wq[2]), "r"(wq[3])
-                   : "memory");
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_dst + off), "r"(wh[0]), "r"(wh[1]),
-                   "r"(wh[2]), "r"(wh[3])
-                   : "memory");
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_dst + T128 + off), "r"(wl[0]),
-                   "r"(wl[1]), "r"(wl[2]), "r"(wl[3])
-                   : "memory");
+      tc_fence_before();
+      mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
+      const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512) + half * 8;
+      const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512 + 256) + half * 8;
+      const int q0 = k0 + it * 64 + half * 32;
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 lv = lv4[c4], dv = dv4[c4];
+        const float la[4] = {lv.x * kLog2e, lv.y * kLog2e, lv.z * kLog2e, lv.w * kLog2e};
+        const float da[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c4 * 4 + e;
+          const float p = ex2(fmaf(st[c], scale_log2, -la[e]));
+          st[c] = p;
+          dpt[c] = p * (dpt[c] - da[e]);
+        }
+      }
+      if (q0 < k0 + 128) {  // steps that reach the diagonal: keys after the query are invisible
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
+      }
+      // the accumulate MMAs of the previous step read P^T and dS^T
+      if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {  // this half's 4 chunks of 8 queries, K-major, 128B swizzle
+        const int c = half * 4 + cc;
+        uint32_t wp[4], wq[4], wh[4], wl[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          split_bf16x2(st[cc * 8 + 2 * h], st[cc * 8 + 2 * h + 1], wp[h], wq[h]);
+          split_bf16x2(dpt[cc * 8 + 2 * h], dpt[cc * 8 + 2 * h + 1], wh[h], wl[h]);
+        }
+        const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
+        store_pair4(s_pt + off, wp);
+        store_pair4(s_pt + T128 + off, wq);
+        store_pair4(s_dst + off, wh);
+        store_pair4(s_dst + T128 + off, wl);
+      }
+      fence_async_smem();
+      mbar_arrive(bar + 8);  // P^T, dS^T of step it are written
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
+    // ---- epilogue: dV, dK rows
+    const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
     tc_fence_after();
-    if (*abort_flag) break;
-    if (tid == 0) issue_acc(it);
-    __syncwarp();
-  }
-
-  const bool ok_end = !*abort_flag && wait_all(bar + 6, (nit - 1) & 1);
-  tc_fence_after();
-  if (ok_end) {
-    float* dvrow = dV + (size_t)(g0 + kj) * D;
-    float* dkrow = dK + (size_t)(g0 + kj) * D;
-    uint32_t r[32];
+    if (ok_end) {
+      float* dvrow = dV + (size_t)(g0 + kj) * D;
+      float* dkrow = dK + (size_t)(g0 + kj) * D;
+      uint32_t r[32];
 #pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      const int c = half * (D / 64) + cc;
-      tmem_ld32(t_dv + lane_off + c * 32, r);
-      tmem_wait_ld();
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c = half * (D / 64) + cc;
+        tmem_ld32(t_dv + lane_off + c * 32, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dvrow + c * 32 + e) =
-            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                        __uint_as_float(r[e + 3]));
-      tmem_ld32(t_dk + lane_off + c * 32, r);
-      tmem_wait_ld();
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dvrow + c * 32 + e) =
+              make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                          __uint_as_float(r[e + 3]));
+        tmem_ld32(t_dk + lane_off + c * 32, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dkrow + c * 32 + e) =
-            make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
-                        __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dkrow + c * 32 + e) =
+              make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
+                          __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag) {
+  if (*abort_flag) {  // let operations already in flight finish before the memory is released
     const uint64_t t0 = globaltimer();
     while (globaltimer() - t0 < 1000000ull) {
     }
@@ -294,7 +287,7 @@ struct LayDQ {
   static constexpr int BYTES = BAR + 128;
 };
 
-// bars: 0 Q+dO, 1-3 K/V stages, 4-5 S+dP buffers, 6 dQ
+// bars: 0 Q+dO | 1-3 K/V stages | 4-5 S buffers | 6-7 S buffers free | 8 dS written | 9-10 acc
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -306,8 +299,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 8) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / 128;
@@ -316,13 +309,11 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   const int g0 = bh * S;
   const int q0 = qb * 128;
   const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
-  const float LOG2E = 1.4426950408889634f;
 
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bar + i, 1);
+    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute : 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
   }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -331,137 +322,140 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   const uint32_t tbase = *tmem_slot;
   // S / dP buffer b at columns 128b / 128b + 64; dQ at 256
   const uint32_t t_dq = tbase + 256;
-  const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_ds = smem_u32(sm + Ly::DS);
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  auto load_kv = [&](int it) {  // into stage it % 3
-    const int sg = it % 3;
-    uint64_t* b = bar + 1 + sg;
-    mbar_expect_tx(b, 2 * KB * T64);
-    for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::K + sg * KB * T64 + c * T64, &tk, c * 64, g0 + it * 64, b);
-      tma_load_2d(sm + Ly::V + sg * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
-    }
-  };
-  auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T into TMEM buffer it & 1
-    const uint32_t kbs = s_k + (it % 3) * KB * T64, vbs = s_v + (it % 3) * KB * T64;
-    const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
+  if (warp == 8) {
+    // ------------------------------------------------------------------ producer
+    if ((tid % 32) == 0) {
+      prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
+      auto load_kv = [&](int it) {  // K, V of key block it into stage it % 3
+        const int sg = it % 3;
+        uint64_t* b = bar + 1 + sg;
+        mbar_expect_tx(b, 2 * KB * T64);
+        for (int c = 0; c < KB; ++c) {
+          tma_load_2d(sm + Ly::K + sg * KB * T64 + c * T64, &tk, c * 64, g0 + it * 64, b);
+          tma_load_2d(sm + Ly::V + sg * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
+        }
+      };
+      auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T into TMEM buffer it & 1
+        const uint32_t kbs = s_k + (it % 3) * KB * T64, vbs = s_v + (it % 3) * KB * T64;
+        const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
-      mma_ss(t_s, sw128_desc(s_q + offA, 16, 1024), sw128_desc(kbs + offB, 16, 1024), IDESC_S, ks > 0);
-      mma_ss(t_dp, sw128_desc(s_do + offA, 16, 1024), sw128_desc(vbs + offB, 16, 1024), IDESC_S, ks > 0);
-    }
-    mma_commit(bar + 4 + (it & 1));
-  };
-  auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
-    const uint32_t kbs = s_k + (it % 3) * KB * T64;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
+          mma_ss(t_s, sw128_desc(s_q + offA, 16, 1024), sw128_desc(kbs + offB, 16, 1024), IDESC_S, ks > 0);
+          mma_ss(t_dp, sw128_desc(s_do + offA, 16, 1024), sw128_desc(vbs + offB, 16, 1024), IDESC_S, ks > 0);
+        }
+        mma_commit(bar + 4 + (it & 1));
+      };
+      auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
+        const uint32_t kbs = s_k + (it % 3) * KB * T64;
 #pragma unroll
-    for (int part = 0; part < 2; ++part)
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_ss(t_dq, sw128_desc(s_ds + part * T128 + ks * 32, 16, 1024),
-               sw128_desc(kbs + ks * 2048, T64, 1024), IDESC_ACC, (it > 0 || part > 0 || ks > 0) ? 1u : 0u);
-    mma_commit(bar + 6);
-  };
-  auto wait_all = [&](uint64_t* b, uint32_t parity) {
-    bool ok = mbar_wait(b, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, ok);
-  };
-
-  if (tid == 0) {
-    mbar_expect_tx(bar, 2 * KB * T128);
-    for (int c = 0; c < KB; ++c) {
-      tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
-      tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
-    }
-    for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
-    if (mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status)) issue_s(0);
-  }
-  __syncwarp();
-
-  const int row = (warp % 4) * 32 + (tid % 32);  // query row within the block = TMEM lane
-  const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
-  const int qi = q0 + row;
-  const float l2 = lse[g0 + qi] * LOG2E;
-  const float dl = delta[g0 + qi];
-  for (int it = 0; it < nit; ++it) {
-    const bool ok_s = wait_all(bar + 4 + (it & 1), (it >> 1) & 1);
-    tc_fence_after();
-    if (tid == 0 && ok_s && it + 1 < nit &&
-        mbar_wait(bar + 1 + (it + 1) % 3, ((it + 1) / 3) & 1, abort_flag, status))
-      issue_s(it + 1);  // the other buffer: its previous step was read before the last barrier
-    __syncwarp();
-    float s[32], dp[32];
-    if (ok_s) {
-      uint32_t r0[32], r2[32];
-      const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
-      tmem_ld32(t_s + lane_off + half * 32, r0);
-      tmem_ld32(t_dp + lane_off + half * 32, r2);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        s[e] = __uint_as_float(r0[e]);
-        dp[e] = __uint_as_float(r2[e]);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bk = sw128_desc(kbs + ks * 2048, T64, 1024);
+          mma_ss(t_dq, sw128_desc(s_ds + ks * 32, 16, 1024), bk, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dq, sw128_desc(s_ds + T128 + ks * 32, 16, 1024), bk, IDESC_ACC, 1u);
+        }
+        mma_commit(bar + 9 + (it & 1));
+      };
+      mbar_expect_tx(bar, 2 * KB * T128);
+      for (int c = 0; c < KB; ++c) {
+        tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
+        tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
+      }
+      for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
+      bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
+      if (ok) issue_s(0);
+      for (int it = 0; it < nit && ok; ++it) {
+        if (it + 1 < nit) {
+          const int n = it + 1;
+          ok = mbar_wait(bar + 1 + n % 3, (n / 3) & 1, abort_flag, status);
+          if (ok && n >= 2) ok = mbar_wait(bar + 6 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(n);
+        }
+        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // dS of step it
+        tc_fence_after();
+        issue_acc(it);
+        if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
+          if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
+          load_kv(it + 2);
+        }
       }
     }
-    const int kj0 = it * 64 + half * 32;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
-    if (kj0 + 32 > q0) {  // steps that reach the diagonal: keys after the query are invisible
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (kj0 + c > qi) dp[c] = 0.f;
-    }
-    bool ok_m = true;
-    if (it > 0) {
-      ok_m = wait_all(bar + 6, (it - 1) & 1);
+  } else {
+    // ------------------------------------------------------------------ compute warps
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
+    const int row = (warp % 4) * 32 + (tid % 32);  // query row within the block = TMEM lane
+    const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
+    const int qi = q0 + row;
+    const float l2 = lse[g0 + qi] * kLog2e;
+    const float dl = delta[g0 + qi];
+    auto wait_all = [&](uint64_t* b, uint32_t parity) {
+      bool ok = mbar_wait(b, parity, abort_flag, status);
+      return __all_sync(0xffffffffu, ok);
+    };
+    for (int it = 0; it < nit; ++it) {
+      if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
       tc_fence_after();
-      if (tid == 0 && ok_m && it + 2 < nit) load_kv(it + 2);  // into stage (it-1) % 3
-      __syncwarp();
-    }
+      float s[32], dp[32];
+      {
+        uint32_t r0[32], r2[32];
+        const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
+        tmem_ld32(t_s + lane_off + half * 32, r0);
+        tmem_ld32(t_dp + lane_off + half * 32, r2);
+        tmem_wait_ld();
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
-      const int c = half * 4 + cc;
-      uint32_t wh[4], wl[4];
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(r0[e]);
+          dp[e] = __uint_as_float(r2[e]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
+      const int kj0 = it * 64 + half * 32;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) split_bf16x2(dp[cc * 8 + 2 * h], dp[cc * 8 + 2 * h + 1], wh[h], wl[h]);
-      const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_ds + off), "r"(wh[0]), "r"(wh[1]),
-                   "r"(wh[2]), "r"(wh[3])
-                   : "memory");
-      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(s_ds + T128 + off), "r"(wl[0]),
-                   "r"(wl[1]), "r"(wl[2]), "r"(wl[3])
-                   : "memory");
+      for (int c = 0; c < 32; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
+      if (kj0 + 32 > q0) {  // steps that reach the diagonal: keys after the query are invisible
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (kj0 + c > qi) dp[c] = 0.f;
+      }
+      if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
+        const int c = half * 4 + cc;
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) split_bf16x2(dp[cc * 8 + 2 * h], dp[cc * 8 + 2 * h + 1], wh[h], wl[h]);
+        const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
+        store_pair4(s_ds + off, wh);
+        store_pair4(s_ds + T128 + off, wl);
+      }
+      fence_async_smem();
+      mbar_arrive(bar + 8);  // dS of step it is written
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
+    const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
     tc_fence_after();
-    if (*abort_flag) break;
-    if (tid == 0) issue_acc(it);
-    __syncwarp();
-  }
-
-  const bool ok_end = !*abort_flag && wait_all(bar + 6, (nit - 1) & 1);
-  tc_fence_after();
-  if (ok_end) {
-    float* dqrow = dQ + (size_t)(g0 + qi) * D;
-    uint32_t r[32];
+    if (ok_end) {
+      float* dqrow = dQ + (size_t)(g0 + qi) * D;
+      uint32_t r[32];
 #pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      const int c = half * (D / 64) + cc;
-      tmem_ld32(t_dq + lane_off + c * 32, r);
-      tmem_wait_ld();
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c = half * (D / 64) + cc;
+        tmem_ld32(t_dq + lane_off + c * 32, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dqrow + c * 32 + e) =
-            make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
-                        __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dqrow + c * 32 + e) =
+              make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
+                          __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
+      }
     }
   }
   tc_fence_before();
@@ -511,14 +505,14 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const float sigma = 1.0f / sqrtf((float)D);
-  const float scale_log2 = sigma * 1.4426950408889634f;
+  const float scale_log2 = sigma * kLog2e;
+  // both kernels hold all 512 TMEM columns: padded so that two CTAs never share an SM
   const int smem1 = LayDKV<D>::BYTES + 1024 > 120 * 1024 ? LayDKV<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
   attn_bwd_dkdv_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem1, st>>>(
       k128, v128, q64, do64, lse, delta, dk, dv, g.S, sigma, scale_log2, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // both kernels hold all 512 TMEM columns: padded so that two CTAs never share an SM
   const int smem2 = LayDQ<D>::BYTES + 1024 > 120 * 1024 ? LayDQ<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
   if (e != cudaSuccess) return e;
