@@ -10,9 +10,10 @@
 //           read as MN-major operands).
 //   dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
 //           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K.
-// Warp roles: warps 0-7 compute (warp w owns TMEM lanes 32(w%4)..+31 and column half w/4 of each
-// step); warp 8, lane 0, is the producer: it issues every TMA load and every MMA. The two sides
-// meet only at mbarriers (S ready, S buffer free, P written, accumulation done), so the tensor
+// Warp roles: warps 0-15 compute (warp w owns TMEM lanes 32(w%4)..+31 and column quarter w/4 of
+// each step); warp 16, lane 0, is the producer: it issues every TMA load and every MMA. The two sides
+// meet only at mbarriers (S ready, S buffer free, P written, accumulation done; one arrival
+// per warp), so the tensor
 // cores work on step it+1's S/dP and step it-1's accumulation while the warps do step it.
 // Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, with lse and D riding along as
 // 1-D bulk copies; S/dP are double-buffered in TMEM; accumulators stay in TMEM until the
@@ -34,7 +35,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kCompute = 256;              // warps 0-7
+constexpr int kCompute = 512;              // warps 0-15
 constexpr int kThreads = kCompute + 32;    // + the producer warp
 constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
@@ -78,14 +79,15 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
-  const int kb = blockIdx.x;  // low key blocks see the most queries: they start first
-  const int bh = blockIdx.y;
+  // grid (BH, blocks): heads vary fastest, so every head's heaviest blocks launch first
+  const int kb = blockIdx.y;  // low key blocks see the most queries
+  const int bh = blockIdx.x;
   const int g0 = bh * S;
   const int k0 = kb * 128;
   const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
 
   if (tid == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute : 1);
+    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -102,7 +104,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  if (warp == 8) {
+  if (warp == kCompute / 32) {
     // ------------------------------------------------------------------ producer
     if ((tid % 32) == 0) {
       prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
@@ -117,26 +119,31 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + k0 + it * 64, 256, b);
         bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + k0 + it * 64, 256, b);
       };
+      // K-major operands: LBO 16, SBO 1024; MN-major Q/dO stages: LBO = one [64][64] sub-tile
+      const uint64_t dK_ = desc_base(16, 1024) + (s_k >> 4), dV_ = desc_base(16, 1024) + (s_v >> 4);
+      const uint64_t dQk = desc_base(16, 1024) + (s_q >> 4), dOk = desc_base(16, 1024) + (s_do >> 4);
+      const uint64_t dQm = desc_base(T64, 1024) + (s_q >> 4), dOm = desc_base(T64, 1024) + (s_do >> 4);
+      const uint64_t dPT = desc_base(16, 1024) + (s_pt >> 4), dST = desc_base(16, 1024) + (s_dst >> 4);
       auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T into TMEM buffer it & 1
-        const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
+        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
         const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
-          mma_ss(t_st, sw128_desc(s_k + offA, 16, 1024), sw128_desc(qb + offB, 16, 1024), IDESC_S, ks > 0);
-          mma_ss(t_dpt, sw128_desc(s_v + offA, 16, 1024), sw128_desc(ob + offB, 16, 1024), IDESC_S, ks > 0);
+          const uint32_t offA = ((ks / 4) * T128 + (ks % 4) * 32) >> 4, offB = ((ks / 4) * T64 + (ks % 4) * 32) >> 4;
+          mma_ss(t_st, dK_ + offA, dQk + sg + offB, IDESC_S, ks > 0);
+          mma_ss(t_dpt, dV_ + offA, dOk + sg + offB, IDESC_S, ks > 0);
         }
         mma_commit(bar + 4 + (it & 1));
       };
       auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
-        const uint32_t qb = s_q + (it % 3) * KB * T64, ob = s_do + (it % 3) * KB * T64;
+        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bq = sw128_desc(qb + ks * 2048, T64, 1024), bo = sw128_desc(ob + ks * 2048, T64, 1024);
-          mma_ss(t_dv, sw128_desc(s_pt + ks * 32, 16, 1024), bo, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dv, sw128_desc(s_pt + T128 + ks * 32, 16, 1024), bo, IDESC_ACC, 1u);
-          mma_ss(t_dk, sw128_desc(s_dst + ks * 32, 16, 1024), bq, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dk, sw128_desc(s_dst + T128 + ks * 32, 16, 1024), bq, IDESC_ACC, 1u);
+          const uint64_t bq = dQm + sg + ks * 128, bo = dOm + sg + ks * 128;  // + ks * 2048 bytes
+          mma_ss(t_dv, dPT + ks * 2, bo, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dv, dPT + T128 / 16 + ks * 2, bo, IDESC_ACC, 1u);
+          mma_ss(t_dk, dST + ks * 2, bq, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dk, dST + T128 / 16 + ks * 2, bq, IDESC_ACC, 1u);
         }
         mma_commit(bar + 9 + (it & 1));
       };
@@ -157,20 +164,20 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
-        tc_fence_after();
-        issue_acc(it);
         if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
           if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
           load_stage(it + 2);
         }
+        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
+        tc_fence_after();
+        issue_acc(it);
       }
     }
   } else {
     // ------------------------------------------------------------------ compute warps
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
     const int row = (warp % 4) * 32 + (tid % 32);  // key row within the block = TMEM lane
-    const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
+    const int qtr = warp / 4;                       // this thread's 16 of the step's 64 columns
     const int kj = k0 + row;
     auto wait_all = [&](uint64_t* b, uint32_t parity) {
       bool ok = mbar_wait(b, parity, abort_flag, status);
@@ -180,26 +187,27 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
       if (!wait_all(bar + 1 + it % 3, (it / 3) & 1)) break;  // lse, D of this step (visibility)
       tc_fence_after();
-      float st[32], dpt[32];
+      float st[16], dpt[16];
       {
-        uint32_t r0[32], r2[32];
+        uint32_t r0[16], r2[16];
         const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
-        tmem_ld32(t_st + lane_off + half * 32, r0);
-        tmem_ld32(t_dpt + lane_off + half * 32, r2);
+        tmem_ld16(t_st + lane_off + qtr * 16, r0);
+        tmem_ld16(t_dpt + lane_off + qtr * 16, r2);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           st[e] = __uint_as_float(r0[e]);
           dpt[e] = __uint_as_float(r2[e]);
         }
       }
       tc_fence_before();
-      mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
-      const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512) + half * 8;
-      const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512 + 256) + half * 8;
-      const int q0 = k0 + it * 64 + half * 32;
+      __syncwarp();
+      if ((tid % 32) == 0) mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
+      const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512) + qtr * 4;
+      const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512 + 256) + qtr * 4;
+      const int q0 = k0 + it * 64 + qtr * 16;
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
+      for (int c4 = 0; c4 < 4; ++c4) {
         const float4 lv = lv4[c4], dv = dv4[c4];
         const float la[4] = {lv.x * kLog2e, lv.y * kLog2e, lv.z * kLog2e, lv.w * kLog2e};
         const float da[4] = {dv.x, dv.y, dv.z, dv.w};
@@ -213,14 +221,14 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       }
       if (q0 < k0 + 128) {  // steps that reach the diagonal: keys after the query are invisible
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
+        for (int c = 0; c < 16; ++c)
           if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
       }
       // the accumulate MMAs of the previous step read P^T and dS^T
       if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {  // this half's 4 chunks of 8 queries, K-major, 128B swizzle
-        const int c = half * 4 + cc;
+      for (int cc = 0; cc < 2; ++cc) {  // this quarter's 2 chunks of 8 queries, K-major, 128B swizzle
+        const int c = qtr * 2 + cc;
         uint32_t wp[4], wq[4], wh[4], wl[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -234,7 +242,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         store_pair4(s_dst + T128 + off, wl);
       }
       fence_async_smem();
-      mbar_arrive(bar + 8);  // P^T, dS^T of step it are written
+      __syncwarp();
+      if ((tid % 32) == 0) mbar_arrive(bar + 8);  // P^T, dS^T of step it are written
     }
     // ---- epilogue: dV, dK rows
     const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
@@ -242,22 +251,22 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     if (ok_end) {
       float* dvrow = dV + (size_t)(g0 + kj) * D;
       float* dkrow = dK + (size_t)(g0 + kj) * D;
-      uint32_t r[32];
+      uint32_t r[16];
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int c = half * (D / 64) + cc;
-        tmem_ld32(t_dv + lane_off + c * 32, r);
+      for (int cc = 0; cc < D / 64; ++cc) {  // this quarter's D/4 columns, 16 at a time
+        const int c = qtr * (D / 64) + cc;
+        tmem_ld16(t_dv + lane_off + c * 16, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dvrow + c * 32 + e) =
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(dvrow + c * 16 + e) =
               make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
                           __uint_as_float(r[e + 3]));
-        tmem_ld32(t_dk + lane_off + c * 32, r);
+        tmem_ld16(t_dk + lane_off + c * 16, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dkrow + c * 32 + e) =
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(dkrow + c * 16 + e) =
               make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
                           __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
       }
@@ -304,14 +313,14 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / 128;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // heaviest first
-  const int bh = blockIdx.y;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // heads vary fastest; heaviest blocks first
+  const int bh = blockIdx.x;
   const int g0 = bh * S;
   const int q0 = qb * 128;
   const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
 
   if (tid == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute : 1);
+    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -328,7 +337,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
-  if (warp == 8) {
+  if (warp == kCompute / 32) {
     // ------------------------------------------------------------------ producer
     if ((tid % 32) == 0) {
       prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
@@ -341,24 +350,27 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           tma_load_2d(sm + Ly::V + sg * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
         }
       };
+      const uint64_t dQ_ = desc_base(16, 1024) + (s_q >> 4), dO_ = desc_base(16, 1024) + (s_do >> 4);
+      const uint64_t dKk = desc_base(16, 1024) + (s_k >> 4), dVk = desc_base(16, 1024) + (s_v >> 4);
+      const uint64_t dKm = desc_base(T64, 1024) + (s_k >> 4), dDS = desc_base(16, 1024) + (s_ds >> 4);
       auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T into TMEM buffer it & 1
-        const uint32_t kbs = s_k + (it % 3) * KB * T64, vbs = s_v + (it % 3) * KB * T64;
+        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
         const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t offA = (ks / 4) * T128 + (ks % 4) * 32, offB = (ks / 4) * T64 + (ks % 4) * 32;
-          mma_ss(t_s, sw128_desc(s_q + offA, 16, 1024), sw128_desc(kbs + offB, 16, 1024), IDESC_S, ks > 0);
-          mma_ss(t_dp, sw128_desc(s_do + offA, 16, 1024), sw128_desc(vbs + offB, 16, 1024), IDESC_S, ks > 0);
+          const uint32_t offA = ((ks / 4) * T128 + (ks % 4) * 32) >> 4, offB = ((ks / 4) * T64 + (ks % 4) * 32) >> 4;
+          mma_ss(t_s, dQ_ + offA, dKk + sg + offB, IDESC_S, ks > 0);
+          mma_ss(t_dp, dO_ + offA, dVk + sg + offB, IDESC_S, ks > 0);
         }
         mma_commit(bar + 4 + (it & 1));
       };
       auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
-        const uint32_t kbs = s_k + (it % 3) * KB * T64;
+        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bk = sw128_desc(kbs + ks * 2048, T64, 1024);
-          mma_ss(t_dq, sw128_desc(s_ds + ks * 32, 16, 1024), bk, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dq, sw128_desc(s_ds + T128 + ks * 32, 16, 1024), bk, IDESC_ACC, 1u);
+          const uint64_t bk = dKm + sg + ks * 128;  // + ks * 2048 bytes
+          mma_ss(t_dq, dDS + ks * 2, bk, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dq, dDS + T128 / 16 + ks * 2, bk, IDESC_ACC, 1u);
         }
         mma_commit(bar + 9 + (it & 1));
       };
@@ -379,20 +391,20 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // dS of step it
-        tc_fence_after();
-        issue_acc(it);
         if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
           if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
           load_kv(it + 2);
         }
+        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // dS of step it
+        tc_fence_after();
+        issue_acc(it);
       }
     }
   } else {
     // ------------------------------------------------------------------ compute warps
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
     const int row = (warp % 4) * 32 + (tid % 32);  // query row within the block = TMEM lane
-    const int half = warp / 4;                      // this thread's 32 of the step's 64 columns
+    const int qtr = warp / 4;                       // this thread's 16 of the step's 64 columns
     const int qi = q0 + row;
     const float l2 = lse[g0 + qi] * kLog2e;
     const float dl = delta[g0 + qi];
@@ -403,33 +415,34 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     for (int it = 0; it < nit; ++it) {
       if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
       tc_fence_after();
-      float s[32], dp[32];
+      float s[16], dp[16];
       {
-        uint32_t r0[32], r2[32];
+        uint32_t r0[16], r2[16];
         const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
-        tmem_ld32(t_s + lane_off + half * 32, r0);
-        tmem_ld32(t_dp + lane_off + half * 32, r2);
+        tmem_ld16(t_s + lane_off + qtr * 16, r0);
+        tmem_ld16(t_dp + lane_off + qtr * 16, r2);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           s[e] = __uint_as_float(r0[e]);
           dp[e] = __uint_as_float(r2[e]);
         }
       }
       tc_fence_before();
-      mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
-      const int kj0 = it * 64 + half * 32;
+      __syncwarp();
+      if ((tid % 32) == 0) mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
+      const int kj0 = it * 64 + qtr * 16;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
-      if (kj0 + 32 > q0) {  // steps that reach the diagonal: keys after the query are invisible
+      for (int c = 0; c < 16; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
+      if (kj0 + 16 > q0) {  // steps that reach the diagonal: keys after the query are invisible
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
+        for (int c = 0; c < 16; ++c)
           if (kj0 + c > qi) dp[c] = 0.f;
       }
       if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
-        const int c = half * 4 + cc;
+      for (int cc = 0; cc < 2; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
+        const int c = qtr * 2 + cc;
         uint32_t wh[4], wl[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) split_bf16x2(dp[cc * 8 + 2 * h], dp[cc * 8 + 2 * h + 1], wh[h], wl[h]);
@@ -438,21 +451,22 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         store_pair4(s_ds + T128 + off, wl);
       }
       fence_async_smem();
-      mbar_arrive(bar + 8);  // dS of step it is written
+      __syncwarp();
+      if ((tid % 32) == 0) mbar_arrive(bar + 8);  // dS of step it is written
     }
     const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
     tc_fence_after();
     if (ok_end) {
       float* dqrow = dQ + (size_t)(g0 + qi) * D;
-      uint32_t r[32];
+      uint32_t r[16];
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int c = half * (D / 64) + cc;
-        tmem_ld32(t_dq + lane_off + c * 32, r);
+      for (int cc = 0; cc < D / 64; ++cc) {  // this quarter's D/4 columns, 16 at a time
+        const int c = qtr * (D / 64) + cc;
+        tmem_ld16(t_dq + lane_off + c * 16, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dqrow + c * 32 + e) =
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(dqrow + c * 16 + e) =
               make_float4(__uint_as_float(r[e]) * sigma, __uint_as_float(r[e + 1]) * sigma,
                           __uint_as_float(r[e + 2]) * sigma, __uint_as_float(r[e + 3]) * sigma);
       }
@@ -510,13 +524,13 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
   const int smem1 = LayDKV<D>::BYTES + 1024 > 120 * 1024 ? LayDKV<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem1, st>>>(
+  attn_bwd_dkdv_tc<D><<<dim3((unsigned)g.BH, (unsigned)(g.S / 128)), kThreads, smem1, st>>>(
       k128, v128, q64, do64, lse, delta, dk, dv, g.S, sigma, scale_log2, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int smem2 = LayDQ<D>::BYTES + 1024 > 120 * 1024 ? LayDQ<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_tc<D><<<dim3((unsigned)(g.S / 128), (unsigned)g.BH), kThreads, smem2, st>>>(
+  attn_bwd_dq_tc<D><<<dim3((unsigned)g.BH, (unsigned)(g.S / 128)), kThreads, smem2, st>>>(
       q128, do128, k64, v64, lse, delta, dq, g.S, sigma, scale_log2, status);
   return cudaGetLastError();
 }

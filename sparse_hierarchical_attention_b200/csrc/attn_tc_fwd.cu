@@ -57,8 +57,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / BM;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // heaviest tiles first
-  const int bh = blockIdx.y;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // heads vary fastest; heaviest tiles first
+  const int bh = blockIdx.x;
   const int grow0 = bh * S;                  // first row of this (b,h) in the [BH*S, D] view
   const int nkb = qb + 1;
 
@@ -309,7 +309,7 @@ cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, con
       !make_tmap_rows(&mv, vs, rows, g.d))
     return cudaErrorInvalidValue;
   const float scale_log2 = (1.0f / sqrtf((float)g.d)) * 1.4426950408889634f;
-  dim3 grid((unsigned)(g.S / BM), (unsigned)g.BH);
+  dim3 grid((unsigned)g.BH, (unsigned)(g.S / BM));
   cudaError_t e;
   if (g.d == 128) {
     const int smem = Layout<128>::BYTES + 1024;

@@ -134,6 +134,16 @@ __device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ inline void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -159,6 +169,14 @@ __device__ inline uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32
   d |= (uint64_t)1 << 46;  // version
   d |= (uint64_t)2 << 61;  // 128-byte swizzle
   return d;
+}
+
+// The same descriptor with the start-address field left for the caller: shared-memory
+// addresses stay below 2^18, so desc_base(lbo, sbo) + (addr >> 4) is sw128_desc(addr, lbo, sbo),
+// and a constant byte offset o is added as (o >> 4).
+__host__ __device__ constexpr uint64_t desc_base(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
 // kind::f16 instruction descriptor: bf16 x bf16 -> f32, M x N, operand majors.
