@@ -11,9 +11,10 @@
 //   dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
 //           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K.
 // Warp roles: warps 0-15 compute (warp w owns TMEM lanes 32(w%4)..+31 and column quarter w/4 of
-// each step); warp 16, lane 0, is the producer: it issues every TMA load and every MMA. The two sides
-// meet only at mbarriers (S ready, S buffer free, P written, accumulation done; one arrival
-// per warp), so the tensor
+// each step); warp 16 (one lane) issues the TMA loads; warp 17 (one lane) issues the MMAs, so that
+// an MMA issue that waits for room in the tensor pipe never delays a load, and the accumulation of
+// a step is issued as soon as its P lands. The sides meet only at mbarriers (stage loaded, stage
+// free, S ready, S buffer free, P written, accumulation done; one arrival per warp), so the tensor
 // cores work on step it+1's S/dP and step it-1's accumulation while the warps do step it.
 // Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, with lse and D riding along as
 // 1-D bulk copies; S/dP are double-buffered in TMEM; accumulators stay in TMEM until the
@@ -36,7 +37,7 @@ namespace {
 using namespace tc;
 
 constexpr int kCompute = 512;              // warps 0-15
-constexpr int kThreads = kCompute + 32;    // + the producer warp
+constexpr int kThreads = kCompute + 64;    // + the TMA warp and the MMA warp
 constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -63,6 +64,7 @@ struct LayDKV {
 };
 
 // bars: 0 K+V | 1-3 Q/dO stages | 4-5 S buffers | 6-7 S buffers free | 8 P written | 9-10 acc
+//       | 11-13 Q/dO stages free
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -75,8 +77,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
   // grid (BH, blocks): heads vary fastest, so every head's heaviest blocks launch first
@@ -87,7 +89,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
 
   if (tid == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
+    for (int i = 0; i < 14; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -105,7 +107,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
   if (warp == kCompute / 32) {
-    // ------------------------------------------------------------------ producer
+    // ------------------------------------------------------------------ TMA warp
     if ((tid % 32) == 0) {
       prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
       auto load_stage = [&](int it) {  // Q, dO, lse, D of query block it into stage it % 3
@@ -119,6 +121,20 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + k0 + it * 64, 256, b);
         bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + k0 + it * 64, 256, b);
       };
+      mbar_expect_tx(bar, 2 * KB * T128);
+      for (int c = 0; c < KB; ++c) {
+        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
+        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
+      }
+      for (int i = 0; i < 3 && i < nit; ++i) load_stage(i);
+      for (int it = 3; it < nit; ++it) {  // step it reuses the stage of step it-3
+        if (!mbar_wait(bar + 11 + it % 3, ((it - 3) / 3) & 1, abort_flag, status)) break;
+        load_stage(it);
+      }
+    }
+  } else if (warp == kCompute / 32 + 1) {
+    // ------------------------------------------------------------------ MMA warp
+    if ((tid % 32) == 0) {
       // K-major operands: LBO 16, SBO 1024; MN-major Q/dO stages: LBO = one [64][64] sub-tile
       const uint64_t dK_ = desc_base(16, 1024) + (s_k >> 4), dV_ = desc_base(16, 1024) + (s_v >> 4);
       const uint64_t dQk = desc_base(16, 1024) + (s_q >> 4), dOk = desc_base(16, 1024) + (s_do >> 4);
@@ -146,13 +162,8 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
           mma_ss(t_dk, dST + T128 / 16 + ks * 2, bq, IDESC_ACC, 1u);
         }
         mma_commit(bar + 9 + (it & 1));
+        mma_commit(bar + 11 + it % 3);  // the stage of step it is free once this completes
       };
-      mbar_expect_tx(bar, 2 * KB * T128);
-      for (int c = 0; c < KB; ++c) {
-        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
-        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
-      }
-      for (int i = 0; i < 3 && i < nit; ++i) load_stage(i);
       bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
       if (ok) issue_s(0);
       for (int it = 0; it < nit && ok; ++it) {
@@ -163,10 +174,6 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
-        }
-        if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
-          if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
-          load_stage(it + 2);
         }
         if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
         tc_fence_after();
@@ -297,6 +304,7 @@ struct LayDQ {
 };
 
 // bars: 0 Q+dO | 1-3 K/V stages | 4-5 S buffers | 6-7 S buffers free | 8 dS written | 9-10 acc
+//       | 11-13 K/V stages free
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -308,8 +316,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / 128;
@@ -320,7 +328,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
 
   if (tid == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
+    for (int i = 0; i < 14; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -338,7 +346,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
   if (warp == kCompute / 32) {
-    // ------------------------------------------------------------------ producer
+    // ------------------------------------------------------------------ TMA warp
     if ((tid % 32) == 0) {
       prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
       auto load_kv = [&](int it) {  // K, V of key block it into stage it % 3
@@ -350,6 +358,20 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           tma_load_2d(sm + Ly::V + sg * KB * T64 + c * T64, &tv, c * 64, g0 + it * 64, b);
         }
       };
+      mbar_expect_tx(bar, 2 * KB * T128);
+      for (int c = 0; c < KB; ++c) {
+        tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
+        tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
+      }
+      for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
+      for (int it = 3; it < nit; ++it) {  // step it reuses the stage of step it-3
+        if (!mbar_wait(bar + 11 + it % 3, ((it - 3) / 3) & 1, abort_flag, status)) break;
+        load_kv(it);
+      }
+    }
+  } else if (warp == kCompute / 32 + 1) {
+    // ------------------------------------------------------------------ MMA warp
+    if ((tid % 32) == 0) {
       const uint64_t dQ_ = desc_base(16, 1024) + (s_q >> 4), dO_ = desc_base(16, 1024) + (s_do >> 4);
       const uint64_t dKk = desc_base(16, 1024) + (s_k >> 4), dVk = desc_base(16, 1024) + (s_v >> 4);
       const uint64_t dKm = desc_base(T64, 1024) + (s_k >> 4), dDS = desc_base(16, 1024) + (s_ds >> 4);
@@ -373,13 +395,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           mma_ss(t_dq, dDS + T128 / 16 + ks * 2, bk, IDESC_ACC, 1u);
         }
         mma_commit(bar + 9 + (it & 1));
+        mma_commit(bar + 11 + it % 3);  // the stage of step it is free once this completes
       };
-      mbar_expect_tx(bar, 2 * KB * T128);
-      for (int c = 0; c < KB; ++c) {
-        tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
-        tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
-      }
-      for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
       bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
       if (ok) issue_s(0);
       for (int it = 0; it < nit && ok; ++it) {
@@ -390,10 +407,6 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
-        }
-        if (it >= 1 && it + 2 < nit) {  // stage (it-1) % 3 is free once acc(it-1) is done
-          if (!mbar_wait(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, status)) break;
-          load_kv(it + 2);
         }
         if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // dS of step it
         tc_fence_after();
