@@ -43,21 +43,32 @@ struct PoolArgs {
   int64_t N, R, S, T, m, C;
   int64_t off[16];    // row id offsets of levels
   float inv[16];      // fl32(1 / p^l)
+  int wdiv[8];        // W / p^l for l = 1..A: level-l cells per stream
   int p, L, W, A2, U;
   int do_pyr, do_score;
 };
 
-// fp32 l2 norm in the SPEC section 2 order: each lane sums the squares of its 16-byte group in
-// ascending order (products rounded on their own), then a butterfly over the LPR lanes of the
-// row realises the halving tree (lane i pairs with i+s for s = LPR/2 .. 1).
-template <int VEC, int LPR>
-__device__ inline float row_norm(const float* x) {
+// fp32 l2 norm in the SPEC section 2 order. Each lane of a row sums the squares of its 16-byte
+// group in ascending order (products rounded on their own) and leaves that partial in shared
+// memory; one lane then folds the LPR partials of the row with the halving tree (partial i
+// pairs with i + s for s = LPR/2 .. 1, the pairs a lane butterfly would form) and takes the root.
+template <int VEC>
+__device__ inline float group_sumsq(const float* x) {
   float a = 0.f;
 #pragma unroll
   for (int e = 0; e < VEC; ++e) a = __fadd_rn(a, __fmul_rn(x[e], x[e]));
+  return a;
+}
+template <int LPR>
+__device__ inline float tree_norm(const float* part) {
+  float t[LPR];
 #pragma unroll
-  for (int s = LPR / 2; s >= 1; s >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, s));
-  return __fsqrt_rn(a);
+  for (int i = 0; i < LPR; ++i) t[i] = part[i];
+#pragma unroll
+  for (int s = LPR / 2; s >= 1; s >>= 1)
+#pragma unroll
+    for (int i = 0; i < s; ++i) t[i] = __fadd_rn(t[i], t[i + s]);
+  return __fsqrt_rn(t[0]);
 }
 
 // Row id -> level and cell index, from the level offsets.
@@ -75,9 +86,16 @@ __global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const
   constexpr int VEC = V::N, LPR = D / VEC, STREAMS = kThreads / LPR;
   constexpr int NX = MODE == MODE_PYRAMID ? 3 : 1;
   constexpr int AR = A > 0 ? A : 1;
+  constexpr bool NORMS = MODE == MODE_PYRAMID;
+  constexpr int PSTR = LPR + 1;  // partials row stride (conflict-free column reads)
   __shared__ float stage[NX][STREAMS][D];
   __shared__ float smax[2][STREAMS];
   __shared__ int smap[MODE == MODE_SPANSUM ? 2 * STREAMS * 16 + 64 : 1];  // (level, cell) -> row
+  // norms: per-lane partial sums of squares [2][STREAMS][16 rows][PSTR], then per stream the row
+  // norms and the level maxima [2][STREAMS][32] (W + W/p + ... + 1 <= 32 entries)
+  extern __shared__ float dyn[];
+  float* const part = dyn;
+  float* const lev = dyn + 2 * STREAMS * 16 * PSTR;
 
   const int tid = threadIdx.x, col = tid % LPR, s = tid / LPR;
   const int64_t bh = blockIdx.y;
@@ -121,45 +139,29 @@ __global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const
   }
 
   float acc[NX][AR][VEC];
-  float mq[AR], mk[AR];
 #pragma unroll
-  for (int l = 0; l < AR; ++l) {
-    mq[l] = 0.f; mk[l] = 0.f;
+  for (int l = 0; l < AR; ++l)
 #pragma unroll
     for (int xi = 0; xi < NX; ++xi)
 #pragma unroll
       for (int e = 0; e < VEC; ++e) acc[xi][l][e] = 0.f;
+  // Level l+1 completes after p completions of level l (level 0: rows); cellj[l] is the global
+  // index of the level-(l+1) cell being summed. W = p^A divides the tile, so the first cell of
+  // a stream is a product of small integers.
+  int left[AR];
+  int64_t cellj[AR];
+#pragma unroll
+  for (int l = 0; l < AR; ++l) {
+    left[l] = p;
+    cellj[l] = ((int64_t)blockIdx.x * STREAMS + s) * (A > 0 ? a.wdiv[l] : 0);
   }
-
-  // Stores one finished cell (level l, global cell j) from registers.
-  auto store_cell = [&](int l, int64_t j, float (*src)[VEC], float sq, float sk) {
-    if constexpr (MODE == MODE_PYRAMID) {
-      if (a.do_pyr) {
-        const int64_t row = bh * a.R + (a.off[l] - a.N) + j;
-#pragma unroll
-        for (int xi = 0; xi < NX; ++xi) {
-          float o[VEC];
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) o[e] = __fmul_rn(src[xi][e], a.inv[l]);
-          stg16(static_cast<E*>(a.px[xi]) + row * D + col * VEC, V::pack(o));
-        }
-      }
-      if (a.do_score && col == 0) a.score[bh * NR + a.off[l] + j] = __fadd_rn(sq, sk);
-    } else {
-      const int64_t first = t_tile;
-      int64_t pw = 1;
-      for (int q = 0; q < l; ++q) pw *= p;
-      const int r = smap[map_base[l] + (int)(j - first / pw)];
-      if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(src[0]));
-    }
-  };
 
   const E* X[NX];
 #pragma unroll
-  for (int xi = 0; xi < NX; ++xi) X[xi] = static_cast<const E*>(a.x[xi]);
+  for (int xi = 0; xi < NX; ++xi) X[xi] = static_cast<const E*>(a.x[xi]) + (bh * a.N + tok0) * D + col * VEC;
 
-  // Rows are fetched U at a time (3U x 16 bytes in flight per thread), then processed.
-  constexpr int U = LH_POOL_UNROLL;
+  // Rows are fetched U at a time (NX x U x 16 bytes in flight per thread), then processed.
+  constexpr int U = NX == 1 ? 2 * LH_POOL_UNROLL : LH_POOL_UNROLL;
 #pragma unroll 1
   for (int row0 = 0; row0 < W; row0 += U) {
     uint4 raw[U][NX];
@@ -168,70 +170,113 @@ __global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const
 #pragma unroll
       for (int xi = 0; xi < NX; ++xi) {
         raw[u][xi] = make_uint4(0, 0, 0, 0);
-        if (active && xi < nx && row0 + u < W)
-          raw[u][xi] = ldg16(X[xi] + (bh * a.N + tok0 + row0 + u) * D + col * VEC);
+        if (active && xi < nx && row0 + u < W) raw[u][xi] = ldg16(X[xi] + (int64_t)(row0 + u) * D);
       }
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int row = row0 + u;
-    if (row >= W) break;  // the same for every thread of the CTA
-    const int64_t t = tok0 + row;
-    float x[NX][VEC];
+    for (int u = 0; u < U; ++u) {
+      const int row = row0 + u;
+      if (row >= W) break;  // the same for every thread of the CTA
+      float x[NX][VEC];
 #pragma unroll
-    for (int xi = 0; xi < NX; ++xi) V::unpack(raw[u][xi], x[xi]);
-    float nq = 0.f, nk = 0.f;
-    if (MODE == MODE_PYRAMID && a.do_score) {
-      nq = row_norm<VEC, LPR>(x[0]);
-      nk = row_norm<VEC, LPR>(x[1]);
-      if (active && col == 0) a.score[bh * NR + t] = __fadd_rn(nq, nk);
-    }
-    if constexpr (MODE == MODE_SPANSUM) {
-      if (active) {
-        const int r = smap[(int)(t - t_tile)];
-        if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(x[0]));
-      }
-    }
-    if constexpr (A > 0) {
-#pragma unroll
-      for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[xi][0][e] += x[xi][e];
-      mq[0] = fmaxf(mq[0], nq);
-      mk[0] = fmaxf(mk[0], nk);
-      int pw = 1;
-#pragma unroll
-      for (int l = 1; l <= A; ++l) {
-        pw *= p;
-        if ((row + 1) % pw != 0) break;
-        float cur[NX][VEC];
-#pragma unroll
-        for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) cur[xi][e] = acc[xi][l - 1][e];
-        if (active) store_cell(l, (t + 1) / pw - 1, cur, mq[l - 1], mk[l - 1]);
-        if (l < A) {
-#pragma unroll
-          for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[xi][l < A ? l : 0][e] += cur[xi][e];
-          mq[l < A ? l : 0] = fmaxf(mq[l < A ? l : 0], mq[l - 1]);
-          mk[l < A ? l : 0] = fmaxf(mk[l < A ? l : 0], mk[l - 1]);
-        } else {
-#pragma unroll
-          for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = cur[xi][e];
-          if (col == 0) { smax[0][s] = mq[l - 1]; smax[1][s] = mk[l - 1]; }
+      for (int xi = 0; xi < NX; ++xi) V::unpack(raw[u][xi], x[xi]);
+      if constexpr (NORMS) {
+        if (a.do_score) {
+          float* pr = part + (s * 16 + row) * PSTR + col;
+          pr[0] = group_sumsq<VEC>(x[0]);
+          pr[STREAMS * 16 * PSTR] = group_sumsq<VEC>(x[1]);
         }
+      }
+      if constexpr (MODE == MODE_SPANSUM) {
+        if (active) {
+          const int r = smap[s * W + row];
+          if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(x[0]));
+        }
+      }
+      if constexpr (A > 0) {
 #pragma unroll
         for (int xi = 0; xi < NX; ++xi)
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[xi][l - 1][e] = 0.f;
-        mq[l - 1] = 0.f;
-        mk[l - 1] = 0.f;
+          for (int e = 0; e < VEC; ++e) acc[xi][0][e] += x[xi][e];
+#pragma unroll
+        for (int l = 0; l < A; ++l) {  // a finished level-l cell may finish level l+1, and so on
+          if (--left[l] != 0) break;
+          left[l] = p;
+          const int lv = l + 1;
+          if (active) {
+            if constexpr (MODE == MODE_PYRAMID) {
+              if (a.do_pyr) {
+                const int64_t prow = bh * a.R + (a.off[lv] - a.N) + cellj[l];
+#pragma unroll
+                for (int xi = 0; xi < NX; ++xi) {
+                  float o[VEC];
+#pragma unroll
+                  for (int e = 0; e < VEC; ++e) o[e] = __fmul_rn(acc[xi][l][e], a.inv[lv]);
+                  stg16(static_cast<E*>(a.px[xi]) + prow * D + col * VEC, V::pack(o));
+                }
+              }
+            } else {
+              const int local = (int)(cellj[l] - (int64_t)blockIdx.x * STREAMS * a.wdiv[l]);
+              const int r = smap[map_base[lv] + local];
+              if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(acc[0][l]));
+            }
+          }
+          ++cellj[l];
+          if (l + 1 < A) {
+#pragma unroll
+            for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) acc[xi][l + 1 < A ? l + 1 : l][e] += acc[xi][l][e];
+          } else {
+#pragma unroll
+            for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = acc[xi][l][e];
+          }
+#pragma unroll
+          for (int xi = 0; xi < NX; ++xi)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[xi][l][e] = 0.f;
+        }
       }
     }
   }
+
+  // Norms of the stream's W rows (lane c takes rows c, c + LPR, ...), the level-0 scores, and the
+  // max-pooled scores of levels 1..A.
+  if constexpr (NORMS) {
+    if (a.do_score) {
+      __syncwarp();
+      float* const lq = lev + s * 32;
+      float* const lk = lev + (STREAMS + s) * 32;
+      for (int r = col; r < W; r += LPR) {
+        const float nq = tree_norm<LPR>(part + (s * 16 + r) * PSTR);
+        const float nk = tree_norm<LPR>(part + ((STREAMS + s) * 16 + r) * PSTR);
+        if (active) a.score[bh * NR + tok0 + r] = __fadd_rn(nq, nk);
+        lq[r] = nq;
+        lk[r] = nk;
+      }
+      __syncwarp();
+      int base = 0, n = W;
+#pragma unroll 1
+      for (int l = 1; l <= A; ++l) {
+        const int nc = n / p;
+        const int64_t first = ((int64_t)blockIdx.x * STREAMS + s) * a.wdiv[l - 1];
+        for (int c = col; c < nc; c += LPR) {
+          float mq = 0.f, mk = 0.f;
+          for (int ch = 0; ch < p; ++ch) {
+            mq = fmaxf(mq, lq[base + c * p + ch]);
+            mk = fmaxf(mk, lk[base + c * p + ch]);
+          }
+          lq[base + n + c] = mq;
+          lk[base + n + c] = mk;
+          if (active) a.score[bh * NR + a.off[l] + first + c] = __fadd_rn(mq, mk);
+        }
+        base += n;
+        n = nc;
+        __syncwarp();
+      }
+      if (A > 0 && col == 0) { smax[0][s] = lq[base]; smax[1][s] = lk[base]; }
+    }
   }
   if (A == 0 || (a.U == 0 && a.A2 >= a.L - 1)) return;
   __syncthreads();
@@ -423,18 +468,28 @@ Plan make_plan(const Geo& g) {
   return pl;
 }
 
+template <typename E, int D, int A, int MODE>
+cudaError_t launch_tile_a(dim3 grid, const PoolArgs& a, cudaStream_t st) {
+  constexpr int LPR = D / Vec<E>::N, STREAMS = kThreads / LPR;
+  const size_t smem = MODE == MODE_PYRAMID ? (size_t)(2 * STREAMS * 16 * (LPR + 1) + 2 * STREAMS * 32) * sizeof(float) : 0;
+  cudaError_t e = cudaFuncSetAttribute(pool_tile_kernel<E, D, A, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  pool_tile_kernel<E, D, A, MODE><<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename E, int D, int MODE>
 cudaError_t launch_tile(const Plan& pl, const PoolArgs& a, int64_t BH, cudaStream_t st) {
   const int64_t tile = (int64_t)pl.W * pl.streams;
   dim3 grid((unsigned)((a.N + tile - 1) / tile), (unsigned)BH);
   switch (pl.A) {
-    case 0: pool_tile_kernel<E, D, 0, MODE><<<grid, kThreads, 0, st>>>(a); break;
-    case 1: pool_tile_kernel<E, D, 1, MODE><<<grid, kThreads, 0, st>>>(a); break;
-    case 2: pool_tile_kernel<E, D, 2, MODE><<<grid, kThreads, 0, st>>>(a); break;
-    case 3: pool_tile_kernel<E, D, 3, MODE><<<grid, kThreads, 0, st>>>(a); break;
-    default: pool_tile_kernel<E, D, 4, MODE><<<grid, kThreads, 0, st>>>(a); break;
+    case 0: return launch_tile_a<E, D, 0, MODE>(grid, a, st);
+    case 1: return launch_tile_a<E, D, 1, MODE>(grid, a, st);
+    case 2: return launch_tile_a<E, D, 2, MODE>(grid, a, st);
+    case 3: return launch_tile_a<E, D, 3, MODE>(grid, a, st);
+    default: return launch_tile_a<E, D, 4, MODE>(grid, a, st);
   }
-  return cudaGetLastError();
 }
 
 template <int MODE>
@@ -442,6 +497,10 @@ cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
   const Plan pl = make_plan(g);
   a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C;
   a.p = g.p; a.L = g.L; a.W = pl.W; a.A2 = pl.A2; a.U = pl.U;
+  for (int l = 0, w = pl.W; l < 8; ++l) {  // level-(l+1) cells per stream
+    w = l < pl.A ? w / g.p : 0;
+    a.wdiv[l] = w;
+  }
   for (int l = 0; l < 16; ++l) {
     a.off[l] = l < g.L ? g.off[l] : 0;
     double pw = 1.0;
