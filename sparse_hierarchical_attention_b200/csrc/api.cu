@@ -209,7 +209,7 @@ int lh_launches(const lh_shape* shape, int* fwd, int* bwd) {
   // forward: pyramid (+coarse), select, gather, attention, scatter
   if (fwd) *fwd = pool_launches(g) + 1 + 1 + attn_fwd_launches(g) + 1;
   // backward: span sums (+coarse), attention backward, gather backward
-  if (bwd) *bwd = pool_launches(g) + attn_bwd_launches(g) + 1;
+  if (bwd) *bwd = span_sum_launches(g) + attn_bwd_launches(g) + 1;
   return LH_OK;
 }
 

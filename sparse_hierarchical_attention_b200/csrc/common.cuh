@@ -86,6 +86,7 @@ cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool fr
 cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, void* do_sub,
                             void* tmp, uint32_t* status, cudaStream_t st);
 size_t span_sum_tmp_bytes(const Geo& g);
+int span_sum_launches(const Geo& g);  // 1 or 2, as pool_launches
 bool attn_tc_eligible(const Geo& g);  // bf16, d in {64,128}, S % 128 == 0
 cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
                                float* os, float* lse, uint32_t* status, cudaStream_t st);

@@ -25,6 +25,9 @@ namespace {
 
 constexpr int kThreads = 256;
 enum { MODE_PYRAMID = 0, MODE_SPANSUM = 1 };
+// Rows one stream walks with register carries: p^A <= 16 for the three-tensor pyramid, <= 64 for
+// the one-tensor span sums (fewer live registers, so longer streams and fewer tile setups).
+constexpr int kWMaxPyr = 16, kWMaxSpan = 64;
 // Rows fetched ahead per thread, and the CTAs per SM the register budget is sized for.
 #ifndef LH_POOL_UNROLL
 #define LH_POOL_UNROLL 4
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const
   constexpr int PSTR = LPR + 1;  // partials row stride (conflict-free column reads)
   __shared__ float stage[NX][STREAMS][D];
   __shared__ float smax[2][STREAMS];
-  __shared__ int smap[MODE == MODE_SPANSUM ? 2 * STREAMS * 16 + 64 : 1];  // (level, cell) -> row
+  __shared__ int smap[MODE == MODE_SPANSUM ? 2 * STREAMS * kWMaxSpan + 64 : 1];  // (level, cell) -> row
   // norms: per-lane partial sums of squares [2][STREAMS][16 rows][PSTR], then per stream the row
   // norms and the level maxima [2][STREAMS][32] (W + W/p + ... + 1 <= 32 entries)
   extern __shared__ float dyn[];
@@ -441,10 +444,10 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
   }
 }
 
-// Register levels A for a pooling factor: the largest A <= min(L-1, 4) with p^A <= 16.
-int pick_A(int p, int L) {
+// Register levels A for a pooling factor: the largest A <= min(L-1, 4) with p^A <= wmax.
+int pick_A(int p, int L, int wmax) {
   int A = 0, pw = 1;
-  while (A < L - 1 && A < 4 && pw * p <= 16) { pw *= p; ++A; }
+  while (A < L - 1 && A < 4 && pw * p <= wmax) { pw *= p; ++A; }
   return A;
 }
 
@@ -452,9 +455,9 @@ struct Plan {
   int A, W, streams, U, A2;
 };
 
-Plan make_plan(const Geo& g) {
+Plan make_plan(const Geo& g, int wmax) {
   Plan pl;
-  pl.A = pick_A(g.p, g.L);
+  pl.A = pick_A(g.p, g.L, wmax);
   pl.W = 1;
   for (int i = 0; i < pl.A; ++i) pl.W *= g.p;
   const int vec = 16 / g.esize, lpr = g.d / vec;
@@ -494,7 +497,7 @@ cudaError_t launch_tile(const Plan& pl, const PoolArgs& a, int64_t BH, cudaStrea
 
 template <int MODE>
 cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
-  const Plan pl = make_plan(g);
+  const Plan pl = make_plan(g, MODE == MODE_SPANSUM ? kWMaxSpan : kWMaxPyr);
   a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C;
   a.p = g.p; a.L = g.L; a.W = pl.W; a.A2 = pl.A2; a.U = pl.U;
   for (int l = 0, w = pl.W; l < 8; ++l) {  // level-(l+1) cells per stream
@@ -529,8 +532,8 @@ cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-size_t tmp_bytes(const Geo& g, int nx) {
-  const Plan pl = make_plan(g);
+size_t tmp_bytes(const Geo& g, int nx, int wmax) {
+  const Plan pl = make_plan(g, wmax);
   if (pl.A2 >= g.L - 1) return 0;
   int64_t pw = 1;
   for (int l = 0; l < pl.A2; ++l) pw *= g.p;
@@ -540,9 +543,10 @@ size_t tmp_bytes(const Geo& g, int nx) {
 
 }  // namespace
 
-size_t pyramid_tmp_bytes(const Geo& g) { return tmp_bytes(g, 3); }
-int pool_launches(const Geo& g) { return make_plan(g).A2 >= g.L - 1 ? 1 : 2; }
-size_t span_sum_tmp_bytes(const Geo& g) { return tmp_bytes(g, 1); }
+size_t pyramid_tmp_bytes(const Geo& g) { return tmp_bytes(g, 3, kWMaxPyr); }
+int pool_launches(const Geo& g) { return make_plan(g, kWMaxPyr).A2 >= g.L - 1 ? 1 : 2; }
+size_t span_sum_tmp_bytes(const Geo& g) { return tmp_bytes(g, 1, kWMaxSpan); }
+int span_sum_launches(const Geo& g) { return make_plan(g, kWMaxSpan).A2 >= g.L - 1 ? 1 : 2; }
 
 cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,
                            void* pk, void* pv, float* score, void* tmp, cudaStream_t st) {
