@@ -6,19 +6,21 @@
 //   dkdv: one CTA per 128-key block steps through the 64-row query blocks that can see the keys:
 //           S^T = K Q^T and dP^T = V dO^T;
 //           P^T = exp2(S^T c - lse2) and dS^T = P^T (dP^T - D) in fp32 registers;
-//           dV += P^T dO and dK += dS^T Q (A operands from shared memory, K-major; B = dO or Q
-//           read as MN-major operands).
+//           dV += P^T dO and dK += dS^T Q, with P^T and dS^T written to tensor memory by the
+//           warps and read from there as the A operand (B = dO or Q, MN-major, from shared memory).
 //   dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
-//           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K.
+//           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K (dS from tensor memory).
 // Warp roles: warps 0-15 compute (warp w owns TMEM lanes 32(w%4)..+31 and column quarter w/4 of
 // each step); warp 16 (one lane) issues the TMA loads; warp 17 (one lane) issues the MMAs, so that
 // an MMA issue that waits for room in the tensor pipe never delays a load, and the accumulation of
 // a step is issued as soon as its P lands. The sides meet only at mbarriers (stage loaded, stage
 // free, S ready, S buffer free, P written, accumulation done; one arrival per warp), so the tensor
 // cores work on step it+1's S/dP and step it-1's accumulation while the warps do step it.
-// Q/dO (dkdv) and K/V (dq) come through three-stage TMA rings, with lse and D riding along as
-// 1-D bulk copies; S/dP are double-buffered in TMEM; accumulators stay in TMEM until the
-// epilogue writes fp32 results.
+// Q/dO (dkdv) and K/V (dq) come through four-stage TMA rings, with lse and D riding along as
+// 1-D bulk copies. Tensor memory holds S/dP (single-buffered in dkdv, whose warps read it at the
+// start of a step; double-buffered in dq), the P/dS operands in their own columns (so that no MMA
+// writes columns an earlier MMA may still read), and the accumulators until the epilogue writes
+// fp32 results.
 // dQ, dK and dV all sum P or dS against rows with mixed signs. Coarse rows carry dO_sub that
 // sums thousands of tokens, and there those sums cancel by orders of magnitude. So P^T, dS^T and
 // dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That is
@@ -42,29 +44,25 @@ constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ inline void store_pair4(uint32_t addr, const uint32_t (&w)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-               "r"(w[3])
-               : "memory");
-}
-
 // ------------------------------------------------------------------------------------ dK, dV
+constexpr int kStQ = 4;  // Q/dO stages of the dK/dV kernel
+
 template <int D>
 struct LayDKV {
   static constexpr int KB = D / 64;
   static constexpr int K = 0;                     // [128][D]
   static constexpr int V = K + KB * T128;         // [128][D]
-  static constexpr int Q = V + KB * T128;         // 3 stages of [64][D]
-  static constexpr int DO = Q + 3 * KB * T64;     // 3 stages of [64][D]
-  static constexpr int PT = DO + 3 * KB * T64;    // hi, lo: [128 keys][64 queries] each
-  static constexpr int DST = PT + 2 * T128;       // hi, lo: [128 keys][64 queries] each
-  static constexpr int VEC = DST + 2 * T128;      // 3 stages of lse[64], delta[64]
-  static constexpr int BAR = VEC + 3 * 512;
+  static constexpr int Q = V + KB * T128;         // kStQ stages of [64][D]
+  static constexpr int DO = Q + kStQ * KB * T64;  // kStQ stages of [64][D]
+  static constexpr int VEC = DO + kStQ * KB * T64;  // kStQ stages of lse[64], delta[64]
+  static constexpr int BAR = VEC + kStQ * 512;
   static constexpr int BYTES = BAR + 128;
 };
 
-// bars: 0 K+V | 1-3 Q/dO stages | 4-5 S buffers | 6-7 S buffers free | 8 P written | 9-10 acc
-//       | 11-13 Q/dO stages free
+// bars: 0 K+V | 1-4 Q/dO stages loaded | 5 S ready | 6 S read | 7 P written | 8 acc done
+//       | 9-12 Q/dO stages free
+// TMEM columns: S^T 0-63, dP^T 64-127, dV 128.., dK 128+D.., P^T hi 384, lo 416, dS^T hi 448,
+// lo 480 (64 queries as bf16 pairs: 32 columns each)
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -74,11 +72,19 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
                  float scale_log2, uint32_t* status) {
   using Ly = LayDKV<D>;
   constexpr int KB = Ly::KB;
+  constexpr int kBars = 9 + kStQ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + kBars) + 1;
+  uint64_t* const bar_kv = bar;
+  uint64_t* const bar_st = bar + 1;        // + stage
+  uint64_t* const bar_s = bar + 5;
+  uint64_t* const bar_sfree = bar + 6;
+  uint64_t* const bar_p = bar + 7;
+  uint64_t* const bar_acc = bar + 8;
+  uint64_t* const bar_stfree = bar + 9;    // + stage
 
   const int tid = threadIdx.x, warp = tid / 32;
   // grid (BH, blocks): heads vary fastest, so every head's heaviest blocks launch first
@@ -89,7 +95,7 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
 
   if (tid == 0) {
-    for (int i = 0; i < 14; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
+    for (int i = 0; i < kBars; ++i) mbar_init(bar + i, (i == 6 || i == 7) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -98,11 +104,10 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  // S^T / dP^T buffer b at columns 128b / 128b + 64; dV at 256, dK at 256 + D
-  const uint32_t t_dv = tbase + 256, t_dk = tbase + 256 + D;
+  const uint32_t t_st = tbase, t_dpt = tbase + 64, t_dv = tbase + 128, t_dk = tbase + 128 + D;
+  const uint32_t t_pt = tbase + 384, t_dst = tbase + 448;
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
-  const uint32_t s_pt = smem_u32(sm + Ly::PT), s_dst = smem_u32(sm + Ly::DST);
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
@@ -110,9 +115,9 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     // ------------------------------------------------------------------ TMA warp
     if ((tid % 32) == 0) {
       prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
-      auto load_stage = [&](int it) {  // Q, dO, lse, D of query block it into stage it % 3
-        const int sg = it % 3;
-        uint64_t* b = bar + 1 + sg;
+      auto load_stage = [&](int it) {  // Q, dO, lse, D of query block it into stage it % kStQ
+        const int sg = it % kStQ;
+        uint64_t* b = bar_st + sg;
         mbar_expect_tx(b, 2 * KB * T64 + 512);
         for (int c = 0; c < KB; ++c) {
           tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
@@ -121,14 +126,13 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + k0 + it * 64, 256, b);
         bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + k0 + it * 64, 256, b);
       };
-      mbar_expect_tx(bar, 2 * KB * T128);
+      mbar_expect_tx(bar_kv, 2 * KB * T128);
       for (int c = 0; c < KB; ++c) {
-        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar);
-        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar);
+        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar_kv);
+        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar_kv);
       }
-      for (int i = 0; i < 3 && i < nit; ++i) load_stage(i);
-      for (int it = 3; it < nit; ++it) {  // step it reuses the stage of step it-3
-        if (!mbar_wait(bar + 11 + it % 3, ((it - 3) / 3) & 1, abort_flag, status)) break;
+      for (int it = 0; it < nit; ++it) {  // step it reuses the stage of step it - kStQ
+        if (it >= kStQ && !mbar_wait(bar_stfree + it % kStQ, ((it - kStQ) / kStQ) & 1, abort_flag, status)) break;
         load_stage(it);
       }
     }
@@ -139,43 +143,41 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       const uint64_t dK_ = desc_base(16, 1024) + (s_k >> 4), dV_ = desc_base(16, 1024) + (s_v >> 4);
       const uint64_t dQk = desc_base(16, 1024) + (s_q >> 4), dOk = desc_base(16, 1024) + (s_do >> 4);
       const uint64_t dQm = desc_base(T64, 1024) + (s_q >> 4), dOm = desc_base(T64, 1024) + (s_do >> 4);
-      const uint64_t dPT = desc_base(16, 1024) + (s_pt >> 4), dST = desc_base(16, 1024) + (s_dst >> 4);
-      auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T into TMEM buffer it & 1
-        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
-        const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
+      auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T
+        const uint32_t sg = (uint32_t)((it % kStQ) * KB * T64) >> 4;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t offA = ((ks / 4) * T128 + (ks % 4) * 32) >> 4, offB = ((ks / 4) * T64 + (ks % 4) * 32) >> 4;
           mma_ss(t_st, dK_ + offA, dQk + sg + offB, IDESC_S, ks > 0);
           mma_ss(t_dpt, dV_ + offA, dOk + sg + offB, IDESC_S, ks > 0);
         }
-        mma_commit(bar + 4 + (it & 1));
+        mma_commit(bar_s);
       };
       auto issue_acc = [&](int it) {  // dV += (P^T_hi + P^T_lo) dO, dK += (dS^T_hi + dS^T_lo) Q
-        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
+        const uint32_t sg = (uint32_t)((it % kStQ) * KB * T64) >> 4;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t bq = dQm + sg + ks * 128, bo = dOm + sg + ks * 128;  // + ks * 2048 bytes
-          mma_ss(t_dv, dPT + ks * 2, bo, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dv, dPT + T128 / 16 + ks * 2, bo, IDESC_ACC, 1u);
-          mma_ss(t_dk, dST + ks * 2, bq, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dk, dST + T128 / 16 + ks * 2, bq, IDESC_ACC, 1u);
+          mma_ts(t_dv, t_pt + ks * 8, bo, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(t_dv, t_pt + 32 + ks * 8, bo, IDESC_ACC, 1u);
+          mma_ts(t_dk, t_dst + ks * 8, bq, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(t_dk, t_dst + 32 + ks * 8, bq, IDESC_ACC, 1u);
         }
-        mma_commit(bar + 9 + (it & 1));
-        mma_commit(bar + 11 + it % 3);  // the stage of step it is free once this completes
+        mma_commit(bar_acc);
+        mma_commit(bar_stfree + it % kStQ);  // the stage of step it is free once this completes
       };
-      bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, status) && mbar_wait(bar_st, 0, abort_flag, status);
       if (ok) issue_s(0);
       for (int it = 0; it < nit && ok; ++it) {
-        if (it + 1 < nit) {  // next step's S/dP into the other buffer once it is free
+        if (it + 1 < nit) {  // next step's S^T/dP^T once the warps have read this step's
           const int n = it + 1;
-          ok = mbar_wait(bar + 1 + n % 3, (n / 3) & 1, abort_flag, status);
-          if (ok && n >= 2) ok = mbar_wait(bar + 6 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
+          ok = mbar_wait(bar_st + n % kStQ, (n / kStQ) & 1, abort_flag, status) &&
+               mbar_wait(bar_sfree, it & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
+        if (!mbar_wait(bar_p, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
         tc_fence_after();
         issue_acc(it);
       }
@@ -191,13 +193,12 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       return __all_sync(0xffffffffu, ok);
     };
     for (int it = 0; it < nit; ++it) {
-      if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
-      if (!wait_all(bar + 1 + it % 3, (it / 3) & 1)) break;  // lse, D of this step (visibility)
+      if (!wait_all(bar_s, it & 1)) break;
+      if (!wait_all(bar_st + it % kStQ, (it / kStQ) & 1)) break;  // lse, D of this step (visibility)
       tc_fence_after();
       float st[16], dpt[16];
       {
         uint32_t r0[16], r2[16];
-        const uint32_t t_st = tbase + (it & 1) * 128, t_dpt = t_st + 64;
         tmem_ld16(t_st + lane_off + qtr * 16, r0);
         tmem_ld16(t_dpt + lane_off + qtr * 16, r2);
         tmem_wait_ld();
@@ -209,9 +210,9 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       }
       tc_fence_before();
       __syncwarp();
-      if ((tid % 32) == 0) mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
-      const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512) + qtr * 4;
-      const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % 3) * 512 + 256) + qtr * 4;
+      if ((tid % 32) == 0) mbar_arrive(bar_sfree);  // S^T / dP^T may be overwritten
+      const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStQ) * 512) + qtr * 4;
+      const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStQ) * 512 + 256) + qtr * 4;
       const int q0 = k0 + it * 64 + qtr * 16;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -231,29 +232,26 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         for (int c = 0; c < 16; ++c)
           if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
       }
-      // the accumulate MMAs of the previous step read P^T and dS^T
-      if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
+      uint32_t wp[8], wq[8], wh[8], wl[8];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {  // this quarter's 2 chunks of 8 queries, K-major, 128B swizzle
-        const int c = qtr * 2 + cc;
-        uint32_t wp[4], wq[4], wh[4], wl[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          split_bf16x2(st[cc * 8 + 2 * h], st[cc * 8 + 2 * h + 1], wp[h], wq[h]);
-          split_bf16x2(dpt[cc * 8 + 2 * h], dpt[cc * 8 + 2 * h + 1], wh[h], wl[h]);
-        }
-        const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
-        store_pair4(s_pt + off, wp);
-        store_pair4(s_pt + T128 + off, wq);
-        store_pair4(s_dst + off, wh);
-        store_pair4(s_dst + T128 + off, wl);
+      for (int h = 0; h < 8; ++h) {
+        split_bf16x2(st[2 * h], st[2 * h + 1], wp[h], wq[h]);
+        split_bf16x2(dpt[2 * h], dpt[2 * h + 1], wh[h], wl[h]);
       }
-      fence_async_smem();
+      // the accumulate MMAs of the previous step read P^T and dS^T
+      if (it > 0 && !wait_all(bar_acc, (it - 1) & 1)) break;
+      tc_fence_after();
+      tmem_st8(t_pt + lane_off + qtr * 8, wp);
+      tmem_st8(t_pt + lane_off + 32 + qtr * 8, wq);
+      tmem_st8(t_dst + lane_off + qtr * 8, wh);
+      tmem_st8(t_dst + lane_off + 32 + qtr * 8, wl);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if ((tid % 32) == 0) mbar_arrive(bar + 8);  // P^T, dS^T of step it are written
+      if ((tid % 32) == 0) mbar_arrive(bar_p);  // P^T, dS^T of step it are written
     }
     // ---- epilogue: dV, dK rows
-    const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
+    const bool ok_end = !*abort_flag && wait_all(bar_acc, (nit - 1) & 1);
     tc_fence_after();
     if (ok_end) {
       float* dvrow = dV + (size_t)(g0 + kj) * D;
@@ -291,20 +289,22 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
 }
 
 // ------------------------------------------------------------------------------------ dQ
+constexpr int kStK = 4;  // K/V stages of the dQ kernel
+
 template <int D>
 struct LayDQ {
   static constexpr int KB = D / 64;
   static constexpr int Q = 0;                    // [128][D]
   static constexpr int DO = Q + KB * T128;       // [128][D]
-  static constexpr int K = DO + KB * T128;       // 3 stages of [64][D]
-  static constexpr int V = K + 3 * KB * T64;     // 3 stages of [64][D]
-  static constexpr int DS = V + 3 * KB * T64;    // hi, lo: [128 queries][64 keys] each
-  static constexpr int BAR = DS + 2 * T128;
-  static constexpr int BYTES = BAR + 128;
+  static constexpr int K = DO + KB * T128;       // kStK stages of [64][D]
+  static constexpr int V = K + kStK * KB * T64;  // kStK stages of [64][D]
+  static constexpr int BAR = V + kStK * KB * T64;
+  static constexpr int BYTES = BAR + 256;
 };
 
-// bars: 0 Q+dO | 1-3 K/V stages | 4-5 S buffers | 6-7 S buffers free | 8 dS written | 9-10 acc
-//       | 11-13 K/V stages free
+// bars: 0 Q+dO | 1-4 K/V stages | 5-6 S buffers | 7-8 S buffers free | 9 dS written | 10-11 acc
+//       | 12-15 K/V stages free
+// TMEM columns: S / dP buffer b at 128b / 128b + 64, dQ at 256, dS hi at 384, lo at 416
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
@@ -316,8 +316,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14) + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 16) + 1;
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / 128;
@@ -328,7 +328,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
 
   if (tid == 0) {
-    for (int i = 0; i < 14; ++i) mbar_init(bar + i, (i == 6 || i == 7 || i == 8) ? kCompute / 32 : 1);
+    for (int i = 0; i < 16; ++i) mbar_init(bar + i, (i == 7 || i == 8 || i == 9) ? kCompute / 32 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -337,11 +337,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  // S / dP buffer b at columns 128b / 128b + 64; dQ at 256
-  const uint32_t t_dq = tbase + 256;
+  const uint32_t t_dq = tbase + 256, t_ds = tbase + 384;
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
-  const uint32_t s_ds = smem_u32(sm + Ly::DS);
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
 
@@ -349,8 +347,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     // ------------------------------------------------------------------ TMA warp
     if ((tid % 32) == 0) {
       prefetch_tmap(&tq); prefetch_tmap(&tdo); prefetch_tmap(&tk); prefetch_tmap(&tv);
-      auto load_kv = [&](int it) {  // K, V of key block it into stage it % 3
-        const int sg = it % 3;
+      auto load_kv = [&](int it) {  // K, V of key block it into stage it % kStK
+        const int sg = it % kStK;
         uint64_t* b = bar + 1 + sg;
         mbar_expect_tx(b, 2 * KB * T64);
         for (int c = 0; c < KB; ++c) {
@@ -363,9 +361,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tma_load_2d(sm + Ly::Q + c * T128, &tq, c * 64, g0 + q0, bar);
         tma_load_2d(sm + Ly::DO + c * T128, &tdo, c * 64, g0 + q0, bar);
       }
-      for (int i = 0; i < 3 && i < nit; ++i) load_kv(i);
-      for (int it = 3; it < nit; ++it) {  // step it reuses the stage of step it-3
-        if (!mbar_wait(bar + 11 + it % 3, ((it - 3) / 3) & 1, abort_flag, status)) break;
+      for (int it = 0; it < nit; ++it) {  // step it reuses the stage of step it - kStK
+        if (it >= kStK && !mbar_wait(bar + 12 + it % kStK, ((it - kStK) / kStK) & 1, abort_flag, status)) break;
         load_kv(it);
       }
     }
@@ -374,9 +371,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     if ((tid % 32) == 0) {
       const uint64_t dQ_ = desc_base(16, 1024) + (s_q >> 4), dO_ = desc_base(16, 1024) + (s_do >> 4);
       const uint64_t dKk = desc_base(16, 1024) + (s_k >> 4), dVk = desc_base(16, 1024) + (s_v >> 4);
-      const uint64_t dKm = desc_base(T64, 1024) + (s_k >> 4), dDS = desc_base(16, 1024) + (s_ds >> 4);
+      const uint64_t dKm = desc_base(T64, 1024) + (s_k >> 4);
       auto issue_s = [&](int it) {  // S = Q K^T, dP = dO V^T into TMEM buffer it & 1
-        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
+        const uint32_t sg = (uint32_t)((it % kStK) * KB * T64) >> 4;
         const uint32_t t_s = tbase + (it & 1) * 128, t_dp = t_s + 64;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -384,31 +381,31 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
           mma_ss(t_s, dQ_ + offA, dKk + sg + offB, IDESC_S, ks > 0);
           mma_ss(t_dp, dO_ + offA, dVk + sg + offB, IDESC_S, ks > 0);
         }
-        mma_commit(bar + 4 + (it & 1));
+        mma_commit(bar + 5 + (it & 1));
       };
-      auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K
-        const uint32_t sg = (uint32_t)((it % 3) * KB * T64) >> 4;
+      auto issue_acc = [&](int it) {  // dQ += (dS_hi + dS_lo) K, dS from tensor memory
+        const uint32_t sg = (uint32_t)((it % kStK) * KB * T64) >> 4;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t bk = dKm + sg + ks * 128;  // + ks * 2048 bytes
-          mma_ss(t_dq, dDS + ks * 2, bk, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
-          mma_ss(t_dq, dDS + T128 / 16 + ks * 2, bk, IDESC_ACC, 1u);
+          mma_ts(t_dq, t_ds + ks * 8, bk, IDESC_ACC, (it > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(t_dq, t_ds + 32 + ks * 8, bk, IDESC_ACC, 1u);
         }
-        mma_commit(bar + 9 + (it & 1));
-        mma_commit(bar + 11 + it % 3);  // the stage of step it is free once this completes
+        mma_commit(bar + 10 + (it & 1));
+        mma_commit(bar + 12 + it % kStK);  // the stage of step it is free once this completes
       };
       bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
       if (ok) issue_s(0);
       for (int it = 0; it < nit && ok; ++it) {
         if (it + 1 < nit) {
           const int n = it + 1;
-          ok = mbar_wait(bar + 1 + n % 3, (n / 3) & 1, abort_flag, status);
-          if (ok && n >= 2) ok = mbar_wait(bar + 6 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
+          ok = mbar_wait(bar + 1 + n % kStK, (n / kStK) & 1, abort_flag, status);
+          if (ok && n >= 2) ok = mbar_wait(bar + 7 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar + 8, it & 1, abort_flag, status)) break;  // dS of step it
+        if (!mbar_wait(bar + 9, it & 1, abort_flag, status)) break;  // dS of step it
         tc_fence_after();
         issue_acc(it);
       }
@@ -426,7 +423,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       return __all_sync(0xffffffffu, ok);
     };
     for (int it = 0; it < nit; ++it) {
-      if (!wait_all(bar + 4 + (it & 1), (it >> 1) & 1)) break;
+      if (!wait_all(bar + 5 + (it & 1), (it >> 1) & 1)) break;
       tc_fence_after();
       float s[16], dp[16];
       {
@@ -443,7 +440,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       }
       tc_fence_before();
       __syncwarp();
-      if ((tid % 32) == 0) mbar_arrive(bar + 6 + (it & 1));  // this S buffer may be overwritten
+      if ((tid % 32) == 0) mbar_arrive(bar + 7 + (it & 1));  // this S buffer may be overwritten
       const int kj0 = it * 64 + qtr * 16;
 #pragma unroll
       for (int c = 0; c < 16; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
@@ -452,22 +449,20 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int c = 0; c < 16; ++c)
           if (kj0 + c > qi) dp[c] = 0.f;
       }
-      if (it > 0 && !wait_all(bar + 9 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
+      uint32_t wh[8], wl[8];  // dS = hi + lo: this quarter's 16 keys as 8 columns of pairs each
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {  // dS = hi + lo, K-major, 128-byte swizzle
-        const int c = qtr * 2 + cc;
-        uint32_t wh[4], wl[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) split_bf16x2(dp[cc * 8 + 2 * h], dp[cc * 8 + 2 * h + 1], wh[h], wl[h]);
-        const uint32_t off = row * 128 + ((c ^ (row % 8)) * 16);
-        store_pair4(s_ds + off, wh);
-        store_pair4(s_ds + T128 + off, wl);
-      }
-      fence_async_smem();
+      for (int h = 0; h < 8; ++h) split_bf16x2(dp[2 * h], dp[2 * h + 1], wh[h], wl[h]);
+      // the accumulate MMAs of the previous step read dS
+      if (it > 0 && !wait_all(bar + 10 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
+      tc_fence_after();
+      tmem_st8(t_ds + lane_off + qtr * 8, wh);
+      tmem_st8(t_ds + lane_off + 32 + qtr * 8, wl);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if ((tid % 32) == 0) mbar_arrive(bar + 8);  // dS of step it is written
+      if ((tid % 32) == 0) mbar_arrive(bar + 9);  // dS of step it is written
     }
-    const bool ok_end = !*abort_flag && wait_all(bar + 9 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
+    const bool ok_end = !*abort_flag && wait_all(bar + 10 + ((nit - 1) & 1), ((nit - 1) >> 1) & 1);
     tc_fence_after();
     if (ok_end) {
       float* dqrow = dQ + (size_t)(g0 + qi) * D;

@@ -4,9 +4,11 @@
 // 2.C: dense causal attention on the S selected rows; row j visible to row i iff j <= i).
 //
 // One CTA = 128 query rows of one (b,h). Warp roles:
-//  - warps 0-3 (softmax): thread t owns query row t = TMEM lane t;
-//  - warp 4, one lane: TMA loads (Q once; K and V through three-stage rings);
-//  - warp 5, one lane: every MMA.
+//  - warps 0-7 (softmax): warps w and w+4 share the TMEM lanes 32(w%4)..+31 (query rows); warp w
+//    takes keys 0-63 of every block and warp w+4 keys 64-127, and the pair swaps row maxima
+//    through shared memory (a 64-thread named barrier) so that both halves use one max;
+//  - warp 8, one lane: TMA loads (Q once; K through a three-stage ring, V through two or three);
+//  - warp 9, one lane: every MMA.
 // Tensor memory (512 columns) holds four disjoint regions, so that no MMA writes columns that
 // an earlier MMA may still read:
 //   S buffers at 0 and 128 (S_{j+1} = Q K_{j+1}^T runs while the softmax of S_j does),
@@ -21,8 +23,8 @@
 //  - Key blocks above the diagonal are skipped; the diagonal block is masked.
 // Tensor-core order: S_0, S_1, PV_0, S_2, PV_1, ... The softmax of S_j therefore overlaps PV_{j-1}
 // and S_{j+1}; it writes P_j only after PV_{j-1} has finished reading P and O.
-// The output is fp32 O_sub and the natural-log lse. Shared memory per CTA: Q + 3 K + 3 V tiles
-// of 128 rows (224 KB at d = 128), one CTA per SM.
+// The output is fp32 O_sub and the natural-log lse. Shared memory per CTA: Q + 3 K + 2 V tiles of
+// 128 rows at d = 128 (192 KB; 3 V tiles at d = 64), one CTA per SM.
 #include <mutex>
 
 #include "tc.cuh"
@@ -33,8 +35,9 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kSoftmax = 128, kThreads = kSoftmax + 64;  // + the TMA warp and the MMA warp
-constexpr int kStages = 3;
+constexpr int kSoftmax = 256, kThreads = kSoftmax + 64;  // + the TMA warp and the MMA warp
+constexpr int kStages = 3;  // K ring
+template <int D> constexpr int v_stages() { return D == 128 ? 2 : 3; }
 constexpr int TILE = 128 * 128;  // bytes of one [128 rows][64 bf16] 128B-swizzled sub-tile
 
 template <int D>
@@ -43,8 +46,9 @@ struct Layout {
   static constexpr int Q = 0;
   static constexpr int K = Q + KB * TILE;            // stage s at K + s * KB * TILE
   static constexpr int V = K + kStages * KB * TILE;  // stage s at V + s * KB * TILE
-  static constexpr int BAR = V + kStages * KB * TILE;
-  static constexpr int BYTES = BAR + 256;
+  static constexpr int BAR = V + v_stages<D>() * KB * TILE;
+  static constexpr int XCH = BAR + 256;              // [2 parities][2 halves][128 rows] floats
+  static constexpr int BYTES = XCH + 2 * 2 * 128 * 4;
 };
 
 // bars: 0 Q | 1-3 K loaded | 4-6 V loaded | 7-9 K free | 10-12 V free | 13-14 S ready
@@ -58,6 +62,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             int S, float scale_log2, uint32_t* status) {
   using Ly = Layout<D>;
   constexpr int KB = Ly::KB;
+  constexpr int kStV = v_stages<D>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
@@ -82,7 +87,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
   if (tid == 0) {
     for (int i = 0; i < kBars; ++i)
-      mbar_init(bar + i, (i == 15 || i == 16 || i == 17) ? kSoftmax / 32 : 1);
+      mbar_init(bar + i, (i == 15 || i == 16 || i == 17) ? kSoftmax / 32 : 1);  // one arrival per warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -104,19 +109,17 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           tma_load_2d(sm + Ly::K + (j % kStages) * KB * TILE + c * TILE, &tk, c * 64, grow0 + j * BN, b);
       };
       auto load_v = [&](int j) {
-        uint64_t* b = bar_v + j % kStages;
+        uint64_t* b = bar_v + j % kStV;
         mbar_expect_tx(b, KB * TILE);
         for (int c = 0; c < KB; ++c)
-          tma_load_2d(sm + Ly::V + (j % kStages) * KB * TILE + c * TILE, &tv, c * 64, grow0 + j * BN, b);
+          tma_load_2d(sm + Ly::V + (j % kStV) * KB * TILE + c * TILE, &tv, c * 64, grow0 + j * BN, b);
       };
       mbar_expect_tx(bar_q, KB * TILE);
       for (int c = 0; c < KB; ++c) tma_load_2d(sm + Ly::Q + c * TILE, &tq, c * 64, grow0 + qb * BM, bar_q);
-      for (int j = 0; j < kStages && j < nkb; ++j) { load_k(j); load_v(j); }
-      for (int j = kStages; j < nkb; ++j) {  // block j reuses the stages of block j - 3
-        const uint32_t par = ((j - kStages) / kStages) & 1;
-        if (!mbar_wait(bar_kfree + j % kStages, par, abort_flag, status)) break;
+      for (int j = 0; j < nkb; ++j) {  // block j reuses the K stage of block j - 3, the V stage of j - kStV
+        if (j >= kStages && !mbar_wait(bar_kfree + j % kStages, ((j - kStages) / kStages) & 1, abort_flag, status)) break;
         load_k(j);
-        if (!mbar_wait(bar_vfree + j % kStages, par, abort_flag, status)) break;
+        if (j >= kStV && !mbar_wait(bar_vfree + j % kStV, ((j - kStV) / kStV) & 1, abort_flag, status)) break;
         load_v(j);
       }
     }
@@ -139,7 +142,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         mma_commit(bar_kfree + j % kStages);
       };
       auto issue_pv = [&](int j) {  // O += hi_j V_j + lo_j V_j
-        const uint32_t sg = (uint32_t)((j % kStages) * KB * TILE) >> 4;
+        const uint32_t sg = (uint32_t)((j % kStV) * KB * TILE) >> 4;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
@@ -148,7 +151,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                    (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(bar_pv);
-        mma_commit(bar_vfree + j % kStages);
+        mma_commit(bar_vfree + j % kStV);
       };
       bool ok = mbar_wait(bar_q, 0, abort_flag, status) && mbar_wait(bar_k, 0, abort_flag, status);
       if (ok) { tc_fence_after(); issue_s(0); }
@@ -162,7 +165,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           issue_s(n);
         }
         ok = mbar_wait(bar_p, j & 1, abort_flag, status) &&
-             mbar_wait(bar_v + j % kStages, (j / kStages) & 1, abort_flag, status);
+             mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status);
         if (!ok) break;
         tc_fence_after();
         issue_pv(j);
@@ -170,98 +173,114 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    constexpr int DH = D / 2;  // O columns each half rescales and stores
+    const int q4 = warp % 4, half = warp / 4;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const int row = q4 * 32 + (tid % 32);  // query row within the tile = TMEM lane
+    float* const xch = reinterpret_cast<float*>(sm + Ly::XCH);
+    // Warps w and w+4 meet here every block, so both always reach it: a failed wait clears `ok`
+    // and the loop goes on without touching tensor memory.
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
     // all lanes of a warp wait together, so that the warp stays converged for tcgen05.ld/st
     auto wait_all = [&](uint64_t* b, uint32_t parity) {
       bool ok = mbar_wait(b, parity, abort_flag, status);
       return __all_sync(0xffffffffu, ok);
     };
-    const int row = tid;  // query row within the tile = TMEM lane
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkb; ++j) {
-      if (!wait_all(bar_s + (j & 1), (j >> 1) & 1)) { ok = false; break; }
+      ok = ok && wait_all(bar_s + (j & 1), (j >> 1) & 1);
       tc_fence_after();
-      float s[BN];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ts = tbase + (j & 1) * 128 + lane_off;
+      float s[64];
+      if (ok) {
+        uint32_t r0[32], r1[32];
+        const uint32_t ts = tbase + (j & 1) * 128 + half * 64 + lane_off;
         tmem_ld32(ts, r0);
         tmem_ld32(ts + 32, r1);
-        tmem_ld32(ts + 64, r2);
-        tmem_ld32(ts + 96, r3);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if ((tid % 32) == 0) mbar_arrive(bar_sfree + (j & 1));
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           s[e] = __uint_as_float(r0[e]) * scale_log2;
           s[32 + e] = __uint_as_float(r1[e]) * scale_log2;
-          s[64 + e] = __uint_as_float(r2[e]) * scale_log2;
-          s[96 + e] = __uint_as_float(r3[e]) * scale_log2;
         }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) s[e] = 0.f;
       }
+      tc_fence_before();
+      __syncwarp();
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_sfree + (j & 1));
       if (j == qb) {  // diagonal block: key column > query row is invisible
 #pragma unroll
-        for (int e = 0; e < BN; ++e)
-          if (e > row) s[e] = -INFINITY;
+        for (int e = 0; e < 64; ++e)
+          if (half * 64 + e > row) s[e] = -INFINITY;
       }
-      float mt = -INFINITY;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int e = 0; e < BN; ++e) mt = fmaxf(mt, s[e]);
+      for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], s[e]);
+      const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      xch[((j & 1) * 2 + half) * 128 + row] = mloc;
+      pair_sync();
+      const float mt = fmaxf(mloc, xch[((j & 1) * 2 + (half ^ 1)) * 128 + row]);
       const bool grow = mt > m_used + 8.0f;
       const float m_new = grow ? mt : m_used;
       const float alpha = grow ? exp2f(m_used - m_new) : 1.0f;
-      float sum = 0.f;
-      uint32_t ph[BN / 2], pl[BN / 2];
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t ph[32], pl[32];
 #pragma unroll
-      for (int e = 0; e < BN; e += 2) {
-        const float a = ex2(s[e] - m_new), b = ex2(s[e + 1] - m_new);
-        sum += a + b;
-        split_bf16x2(a, b, ph[e / 2], pl[e / 2]);
+      for (int e = 0; e < 64; e += 2) {
+        const float x0 = ex2(s[e] - m_new), x1 = ex2(s[e + 1] - m_new);
+        sum4[(e >> 1) & 3] += x0 + x1;
+        split_bf16x2(x0, x1, ph[e / 2], pl[e / 2]);
       }
-      l = l * alpha + sum;
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m_used = m_new;
       // PV_{j-1} must be done before P and O are touched again
       if (j > 0) {
-        if (!wait_all(bar_pv, (j - 1) & 1)) { ok = false; break; }
+        ok = ok && wait_all(bar_pv, (j - 1) & 1);
         tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {  // rescale this warp's O rows
+        if (ok && __any_sync(0xffffffffu, grow)) {  // rescale this warp's rows of its O half
           uint32_t r[32];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(t_o + lane_off + c * 32, r);
+          for (int c = 0; c < DH / 32; ++c) {
+            const uint32_t to = t_o + lane_off + half * DH + c * 32;
+            tmem_ld32(to, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(t_o + lane_off + c * 32, r);
+            tmem_st32(to, r);
           }
         }
       }
+      if (ok) {
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {  // 16 columns of packed pairs per 32 keys
-        uint32_t h[16], w[16];
+        for (int c = 0; c < 2; ++c) {  // keys 64 half + 32c .. : 16 columns of packed pairs
+          uint32_t h[16], w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) { h[e] = ph[c * 16 + e]; w[e] = pl[c * 16 + e]; }
-        tmem_st16(t_p + lane_off + c * 16, h);
-        tmem_st16(t_p + lane_off + 64 + c * 16, w);
+          for (int e = 0; e < 16; ++e) { h[e] = ph[c * 16 + e]; w[e] = pl[c * 16 + e]; }
+          tmem_st16(t_p + lane_off + half * 32 + c * 16, h);
+          tmem_st16(t_p + lane_off + 64 + half * 32 + c * 16, w);
+        }
+        tmem_wait_st();
       }
-      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if ((tid % 32) == 0) mbar_arrive(bar_p);
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_p);
     }
-    // ---- epilogue: O / l and lse
+    // ---- epilogue: O / l and lse (the pair adds its two partial sums of l)
     ok = ok && wait_all(bar_pv, (nkb - 1) & 1);
     tc_fence_after();
+    xch[((nkb & 1) * 2 + half) * 128 + row] = l;
+    pair_sync();
+    const float lo = xch[((nkb & 1) * 2 + (half ^ 1)) * 128 + row];
+    const float lt = half == 0 ? l + lo : lo + l;
     if (ok) {
-      const float inv = 1.0f / l;
-      float* orow = O + (size_t)(grow0 + qb * BM + row) * D;
+      const float inv = 1.0f / lt;
+      float* orow = O + (size_t)(grow0 + qb * BM + row) * D + half * DH;
       uint32_t r[32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(t_o + lane_off + c * 32, r);
+      for (int c = 0; c < DH / 32; ++c) {
+        tmem_ld32(t_o + lane_off + half * DH + c * 32, r);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -270,7 +289,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           *reinterpret_cast<float4*>(orow + c * 32 + e) = v;
         }
       }
-      lse[grow0 + qb * BM + row] = (m_used + log2f(l)) * 0.69314718055994531f;
+      if (half == 0) lse[grow0 + qb * BM + row] = (m_used + log2f(lt)) * 0.69314718055994531f;
     }
   }
   tc_fence_before();
