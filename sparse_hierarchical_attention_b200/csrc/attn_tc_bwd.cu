@@ -39,7 +39,7 @@ namespace {
 using namespace tc;
 
 constexpr int kCompute = 512;              // warps 0-15
-constexpr int kThreads = kCompute + 64;    // + the TMA warp and the MMA warp
+constexpr int kThreads = kCompute + 96;    // + the TMA warp and two MMA warps (S/dP, accumulate)
 constexpr int T128 = 128 * 128;  // [128 rows][64 bf16] sub-tile bytes
 constexpr int T64 = 64 * 128;    // [64 rows][64 bf16] sub-tile bytes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -136,9 +136,11 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         load_stage(it);
       }
     }
-  } else if (warp == kCompute / 32 + 1) {
-    // ------------------------------------------------------------------ MMA warp
+  } else if (warp == kCompute / 32 + 1 || warp == kCompute / 32 + 2) {
+    // ------------------------------------------------------------------ MMA warps
+    // warp 17 issues S^T/dP^T, warp 18 the accumulations; neither waits on the other's barriers
     if ((tid % 32) == 0) {
+      const bool s_issuer = warp == kCompute / 32 + 1;
       // K-major operands: LBO 16, SBO 1024; MN-major Q/dO stages: LBO = one [64][64] sub-tile
       const uint64_t dK_ = desc_base(16, 1024) + (s_k >> 4), dV_ = desc_base(16, 1024) + (s_v >> 4);
       const uint64_t dQk = desc_base(16, 1024) + (s_q >> 4), dOk = desc_base(16, 1024) + (s_do >> 4);
@@ -166,20 +168,21 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
         mma_commit(bar_acc);
         mma_commit(bar_stfree + it % kStQ);  // the stage of step it is free once this completes
       };
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, status) && mbar_wait(bar_st, 0, abort_flag, status);
-      if (ok) issue_s(0);
-      for (int it = 0; it < nit && ok; ++it) {
-        if (it + 1 < nit) {  // next step's S^T/dP^T once the warps have read this step's
-          const int n = it + 1;
+      if (s_issuer) {
+        bool ok = mbar_wait(bar_kv, 0, abort_flag, status);
+        for (int n = 0; n < nit && ok; ++n) {  // S^T/dP^T of step n once the warps have read step n-1's
           ok = mbar_wait(bar_st + n % kStQ, (n / kStQ) & 1, abort_flag, status) &&
-               mbar_wait(bar_sfree, it & 1, abort_flag, status);
+               (n == 0 || mbar_wait(bar_sfree, (n - 1) & 1, abort_flag, status));
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar_p, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
-        tc_fence_after();
-        issue_acc(it);
+      } else {
+        for (int it = 0; it < nit; ++it) {
+          if (!mbar_wait(bar_p, it & 1, abort_flag, status)) break;  // P^T, dS^T of step it
+          tc_fence_after();
+          issue_acc(it);  // its stage-free commit also covers S(it): P(it) exists only after S(it)
+        }
       }
     }
   } else {
@@ -366,9 +369,11 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         load_kv(it);
       }
     }
-  } else if (warp == kCompute / 32 + 1) {
-    // ------------------------------------------------------------------ MMA warp
+  } else if (warp == kCompute / 32 + 1 || warp == kCompute / 32 + 2) {
+    // ------------------------------------------------------------------ MMA warps
+    // warp 17 issues S/dP, warp 18 the accumulations
     if ((tid % 32) == 0) {
+      const bool s_issuer = warp == kCompute / 32 + 1;
       const uint64_t dQ_ = desc_base(16, 1024) + (s_q >> 4), dO_ = desc_base(16, 1024) + (s_do >> 4);
       const uint64_t dKk = desc_base(16, 1024) + (s_k >> 4), dVk = desc_base(16, 1024) + (s_v >> 4);
       const uint64_t dKm = desc_base(T64, 1024) + (s_k >> 4);
@@ -394,20 +399,21 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         mma_commit(bar + 10 + (it & 1));
         mma_commit(bar + 12 + it % kStK);  // the stage of step it is free once this completes
       };
-      bool ok = mbar_wait(bar, 0, abort_flag, status) && mbar_wait(bar + 1, 0, abort_flag, status);
-      if (ok) issue_s(0);
-      for (int it = 0; it < nit && ok; ++it) {
-        if (it + 1 < nit) {
-          const int n = it + 1;
+      if (s_issuer) {
+        bool ok = mbar_wait(bar, 0, abort_flag, status);
+        for (int n = 0; n < nit && ok; ++n) {  // S/dP of step n into buffer n & 1 once it is free
           ok = mbar_wait(bar + 1 + n % kStK, (n / kStK) & 1, abort_flag, status);
           if (ok && n >= 2) ok = mbar_wait(bar + 7 + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        if (!mbar_wait(bar + 9, it & 1, abort_flag, status)) break;  // dS of step it
-        tc_fence_after();
-        issue_acc(it);
+      } else {
+        for (int it = 0; it < nit; ++it) {
+          if (!mbar_wait(bar + 9, it & 1, abort_flag, status)) break;  // dS of step it
+          tc_fence_after();
+          issue_acc(it);  // its stage-free commit also covers S(it): dS(it) exists only after S(it)
+        }
       }
     }
   } else {
