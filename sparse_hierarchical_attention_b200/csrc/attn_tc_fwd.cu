@@ -8,7 +8,8 @@
 //    takes keys 0-63 of every block and warp w+4 keys 64-127, and the pair swaps row maxima
 //    through shared memory (a 64-thread named barrier) so that both halves use one max;
 //  - warp 8, one lane: TMA loads (Q once; K through a three-stage ring, V through two or three);
-//  - warp 9, one lane: every MMA.
+//  - warp 9, one lane: the S MMAs; warp 10, one lane: the PV MMAs. Two issuers keep the tensor
+//    queue fed while either waits on its own barriers.
 // Tensor memory (512 columns) holds four disjoint regions, so that no MMA writes columns that
 // an earlier MMA may still read:
 //   S buffers at 0 and 128 (S_{j+1} = Q K_{j+1}^T runs while the softmax of S_j does),
@@ -35,7 +36,7 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kSoftmax = 256, kThreads = kSoftmax + 64;  // + the TMA warp and the MMA warp
+constexpr int kSoftmax = 256, kThreads = kSoftmax + 96;  // + the TMA warp and two MMA warps
 constexpr int kStages = 3;  // K ring
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 3; }
 constexpr int TILE = 128 * 128;  // bytes of one [128 rows][64 bf16] 128B-swizzled sub-tile
@@ -123,9 +124,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         load_v(j);
       }
     }
-  } else if (warp == kSoftmax / 32 + 1) {
-    // ------------------------------------------------------------------ MMA warp
+  } else if (warp == kSoftmax / 32 + 1 || warp == kSoftmax / 32 + 2) {
+    // ------------------------------------------------------------------ MMA warps
     if ((tid % 32) == 0) {
+      const bool s_issuer = warp == kSoftmax / 32 + 1;
       const uint32_t s_q = smem_u32(sm + Ly::Q), s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
       const uint64_t dQ = desc_base(16, 1024) + (s_q >> 4), dK = desc_base(16, 1024) + (s_k >> 4);
       const uint64_t dV = desc_base(TILE, 1024) + (s_v >> 4);  // MN-major: LBO = one sub-tile
@@ -153,22 +155,23 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         mma_commit(bar_pv);
         mma_commit(bar_vfree + j % kStV);
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, status) && mbar_wait(bar_k, 0, abort_flag, status);
-      if (ok) { tc_fence_after(); issue_s(0); }
-      for (int j = 0; j < nkb && ok; ++j) {
-        if (j + 1 < nkb) {  // S_{j+1} into the other buffer once the softmax has read S_{j-1}
-          const int n = j + 1;
+      if (s_issuer) {
+        bool ok = mbar_wait(bar_q, 0, abort_flag, status);
+        for (int n = 0; n < nkb && ok; ++n) {  // S_n into buffer n & 1 once the softmax has read S_{n-2}
           ok = mbar_wait(bar_k + n % kStages, (n / kStages) & 1, abort_flag, status);
           if (ok && n >= 2) ok = mbar_wait(bar_sfree + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        ok = mbar_wait(bar_p, j & 1, abort_flag, status) &&
-             mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(j);
+      } else {
+        for (int j = 0; j < nkb; ++j) {
+          const bool ok = mbar_wait(bar_p, j & 1, abort_flag, status) &&
+                          mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j);
+        }
       }
     }
   } else {
