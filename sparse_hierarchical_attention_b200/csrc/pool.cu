@@ -28,13 +28,13 @@ enum { MODE_PYRAMID = 0, MODE_SPANSUM = 1 };
 // Rows one stream walks with register carries: p^A <= 16 for the three-tensor pyramid, <= 64 for
 // the one-tensor span sums (fewer live registers, so longer streams and fewer tile setups).
 constexpr int kWMaxPyr = 16, kWMaxSpan = 64;
-// Rows fetched ahead per thread, and the CTAs per SM the register budget is sized for.
-#ifndef LH_POOL_UNROLL
-#define LH_POOL_UNROLL 4
-#endif
-#ifndef LH_POOL_MINB
-#define LH_POOL_MINB 2
-#endif
+// Rows fetched ahead per thread, and the CTAs per SM the register budget is sized for (a sweep
+// of 4 or 8 rows against 2, 3 or 4 CTAs per SM at 128K picked these; A >= 3, which only p = 2
+// or 3 reaches, carries more level sums and gets a larger budget).
+template <int MODE> constexpr int rows_ahead() { return MODE == 0 ? 8 : 4; }
+template <int MODE, int A> constexpr int ctas_per_sm() {
+  return MODE == 0 ? (A >= 3 ? 2 : 3) : (A >= 4 ? 3 : 4);
+}
 
 struct PoolArgs {
   const void* x[3];  // q, k, v (pyramid) or d_o (span sums)
@@ -84,7 +84,7 @@ __device__ inline void decode_rid(int64_t rid, const int64_t* off, int L, int& l
 }
 
 template <typename E, int D, int A, int MODE>
-__global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_kernel(const PoolArgs a) {
   using V = Vec<E>;
   constexpr int VEC = V::N, LPR = D / VEC, STREAMS = kThreads / LPR;
   constexpr int NX = MODE == MODE_PYRAMID ? 3 : 1;
@@ -141,104 +141,84 @@ __global__ void __launch_bounds__(kThreads, LH_POOL_MINB) pool_tile_kernel(const
     __syncthreads();
   }
 
-  float acc[NX][AR][VEC];
-#pragma unroll
-  for (int l = 0; l < AR; ++l)
-#pragma unroll
-    for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[xi][l][e] = 0.f;
-  // Level l+1 completes after p completions of level l (level 0: rows); cellj[l] is the global
-  // index of the level-(l+1) cell being summed. W = p^A divides the tile, so the first cell of
-  // a stream is a product of small integers.
-  int left[AR];
-  int64_t cellj[AR];
-#pragma unroll
-  for (int l = 0; l < AR; ++l) {
-    left[l] = p;
-    cellj[l] = ((int64_t)blockIdx.x * STREAMS + s) * (A > 0 ? a.wdiv[l] : 0);
-  }
-
-  const E* X[NX];
-#pragma unroll
-  for (int xi = 0; xi < NX; ++xi) X[xi] = static_cast<const E*>(a.x[xi]) + (bh * a.N + tok0) * D + col * VEC;
-
-  // Rows are fetched U at a time (NX x U x 16 bytes in flight per thread), then processed.
-  constexpr int U = NX == 1 ? 2 * LH_POOL_UNROLL : LH_POOL_UNROLL;
+  // The tensors go through the tile one after another, so that the registers hold the level
+  // partial sums and the fetched rows of one tensor only (more CTAs per SM, more rows in flight).
+  constexpr int U = rows_ahead<MODE>();
 #pragma unroll 1
-  for (int row0 = 0; row0 < W; row0 += U) {
-    uint4 raw[U][NX];
+  for (int xi = 0; xi < nx; ++xi) {
+    float acc[AR][VEC];
 #pragma unroll
-    for (int u = 0; u < U; ++u)
+    for (int l = 0; l < AR; ++l)
 #pragma unroll
-      for (int xi = 0; xi < NX; ++xi) {
-        raw[u][xi] = make_uint4(0, 0, 0, 0);
-        if (active && xi < nx && row0 + u < W) raw[u][xi] = ldg16(X[xi] + (int64_t)(row0 + u) * D);
+      for (int e = 0; e < VEC; ++e) acc[l][e] = 0.f;
+    // Level l+1 completes after p completions of level l (level 0: rows); cellj[l] is the global
+    // index of the level-(l+1) cell being summed. W = p^A divides the tile, so the first cell of
+    // a stream is a product of small integers.
+    int left[AR];
+    int64_t cellj[AR];
+#pragma unroll
+    for (int l = 0; l < AR; ++l) {
+      left[l] = p;
+      cellj[l] = ((int64_t)blockIdx.x * STREAMS + s) * (A > 0 ? a.wdiv[l] : 0);
+    }
+    const E* const X = static_cast<const E*>(a.x[xi]) + (bh * a.N + tok0) * D + col * VEC;
+    E* const PX = static_cast<E*>(a.px[MODE == MODE_PYRAMID ? xi : 0]);
+    const bool norm_of = NORMS && a.do_score && xi < 2;  // Q and K rows feed the score
+#pragma unroll 1
+    for (int row0 = 0; row0 < W; row0 += U) {
+      uint4 raw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        raw[u] = make_uint4(0, 0, 0, 0);
+        if (active && row0 + u < W) raw[u] = ldg16(X + (int64_t)(row0 + u) * D);
       }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int row = row0 + u;
-      if (row >= W) break;  // the same for every thread of the CTA
-      float x[NX][VEC];
-#pragma unroll
-      for (int xi = 0; xi < NX; ++xi) V::unpack(raw[u][xi], x[xi]);
-      if constexpr (NORMS) {
-        if (a.do_score) {
-          float* pr = part + (s * 16 + row) * PSTR + col;
-          pr[0] = group_sumsq<VEC>(x[0]);
-          pr[STREAMS * 16 * PSTR] = group_sumsq<VEC>(x[1]);
-        }
-      }
-      if constexpr (MODE == MODE_SPANSUM) {
-        if (active) {
-          const int r = smap[s * W + row];
-          if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(x[0]));
-        }
-      }
-      if constexpr (A > 0) {
-#pragma unroll
-        for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[xi][0][e] += x[xi][e];
-#pragma unroll
-        for (int l = 0; l < A; ++l) {  // a finished level-l cell may finish level l+1, and so on
-          if (--left[l] != 0) break;
-          left[l] = p;
-          const int lv = l + 1;
+      for (int u = 0; u < U; ++u) {
+        const int row = row0 + u;
+        if (row >= W) break;  // the same for every thread of the CTA
+        float x[VEC];
+        V::unpack(raw[u], x);
+        if (norm_of) part[((xi * STREAMS + s) * 16 + row) * PSTR + col] = group_sumsq<VEC>(x);
+        if constexpr (MODE == MODE_SPANSUM) {
           if (active) {
-            if constexpr (MODE == MODE_PYRAMID) {
-              if (a.do_pyr) {
-                const int64_t prow = bh * a.R + (a.off[lv] - a.N) + cellj[l];
+            const int r = smap[s * W + row];
+            if (r >= 0) stg16(PX + (bh * a.S + r) * D + col * VEC, V::pack(x));
+          }
+        }
+        if constexpr (A > 0) {
 #pragma unroll
-                for (int xi = 0; xi < NX; ++xi) {
+          for (int e = 0; e < VEC; ++e) acc[0][e] += x[e];
+#pragma unroll
+          for (int l = 0; l < A; ++l) {  // a finished level-l cell may finish level l+1, and so on
+            if (--left[l] != 0) break;
+            left[l] = p;
+            const int lv = l + 1;
+            if (active) {
+              if constexpr (MODE == MODE_PYRAMID) {
+                if (a.do_pyr) {
+                  const int64_t prow = bh * a.R + (a.off[lv] - a.N) + cellj[l];
                   float o[VEC];
 #pragma unroll
-                  for (int e = 0; e < VEC; ++e) o[e] = __fmul_rn(acc[xi][l][e], a.inv[lv]);
-                  stg16(static_cast<E*>(a.px[xi]) + prow * D + col * VEC, V::pack(o));
+                  for (int e = 0; e < VEC; ++e) o[e] = __fmul_rn(acc[l][e], a.inv[lv]);
+                  stg16(PX + prow * D + col * VEC, V::pack(o));
                 }
+              } else {
+                const int local = (int)(cellj[l] - (int64_t)blockIdx.x * STREAMS * a.wdiv[l]);
+                const int r = smap[map_base[lv] + local];
+                if (r >= 0) stg16(PX + (bh * a.S + r) * D + col * VEC, V::pack(acc[l]));
               }
-            } else {
-              const int local = (int)(cellj[l] - (int64_t)blockIdx.x * STREAMS * a.wdiv[l]);
-              const int r = smap[map_base[lv] + local];
-              if (r >= 0) stg16(static_cast<E*>(a.px[0]) + (bh * a.S + r) * D + col * VEC, V::pack(acc[0][l]));
             }
+            ++cellj[l];
+            if (l + 1 < A) {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) acc[l + 1 < A ? l + 1 : l][e] += acc[l][e];
+            } else {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = acc[l][e];
+            }
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[l][e] = 0.f;
           }
-          ++cellj[l];
-          if (l + 1 < A) {
-#pragma unroll
-            for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-              for (int e = 0; e < VEC; ++e) acc[xi][l + 1 < A ? l + 1 : l][e] += acc[xi][l][e];
-          } else {
-#pragma unroll
-            for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-              for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = acc[xi][l][e];
-          }
-#pragma unroll
-          for (int xi = 0; xi < NX; ++xi)
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[xi][l][e] = 0.f;
         }
       }
     }
