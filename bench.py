@@ -52,15 +52,18 @@ def parse():
 
 
 # ----------------------------------------------------------------------------- process group
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU (torchrun env). `gloo` serves the CPU tests of this host logic."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {"timeout": datetime.timedelta(seconds=300)}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, **kw)
     return world, rank, local
 
 
@@ -74,9 +77,18 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def throughput(total_ms_local, steps, tokens_per_rank, world):
+    """Whole-job tokens/s and ms per step. Every rank runs its own replica (weak scaling); the
+    slowest rank's device time over the timed steps sets the job's time."""
+    total_ms = max_over_ranks(total_ms_local, world)
+    ms_step = total_ms / steps
+    return tokens_per_rank * world / (ms_step / 1e3), ms_step
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -212,10 +224,7 @@ def run_ours(args, world, rank, local):
     total_ms = sum(ev[s][0].elapsed_time(ev[s][-1]) for s in range(K))
     per_stage = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)) / K
                  for i, (name, _) in enumerate(stages)}
-    total_ms = max_over_ranks(total_ms, world)
-    ms_step = total_ms / K
-    tokens = B * N * world
-    value = tokens / (ms_step / 1e3)
+    value, ms_step = throughput(total_ms, K, B * N, world)
 
     pk_, src = peaks()
     work = stage_work(w, geo)
