@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sdpa", action="store_true",
+                    help="skip the dense causal SDPA context timing (run when N <= 128K)")
     return ap.parse_args()
 
 
@@ -237,6 +239,8 @@ def run_ours(args, world, rank, local):
             ach, peak, unit = amount / (ms / 1e3) / 1e12, pk_["bf16_tflops"], "TFLOP/s"
         stage_report[name] = {"ms": round(ms, 4), "achieved": round(ach, 2), "unit": unit,
                               "frac": round(ach / peak, 4), "bound": kind}
+        if kind != "hbm":  # against the sustained (power-capped) GEMM figure as well
+            stage_report[name]["frac_sustained"] = round(ach / pk_["bf16_tflops_sustained"], 4)
     dom = max(per_stage, key=per_stage.get)
     kind, amount = work[dom]
     rf = stage_report[dom]
@@ -250,6 +254,9 @@ def run_ours(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world)
+    context = None
+    if world == 1 and not args.no_sdpa and N <= 131072 and dt == torch.bfloat16:
+        context = dense_sdpa_context(q, k, v, d_o, ms_step)
     for t in (pq, pk, pv, score, qs, ks, vs, os_, dos, dqs, dks, dvs, dq, dk, dv, o):
         del t
     out = {
@@ -266,7 +273,40 @@ def run_ours(args, world, rank, local):
     }
     if e2e:
         out["e2e"] = e2e
+    if context:
+        out["context"] = context
     return out
+
+
+def dense_sdpa_context(q, k, v, d_o, ms_layer):
+    """Dense causal SDPA (torch's fused backends) fwd+bwd on the layer's own Q, K, V and dO, for
+    context only: what full attention over all N tokens costs on the same GPU."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    qq, kk, vv = (t.detach().clone().requires_grad_(True) for t in (q, k, v))
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION):
+        try:
+            with sdpa_kernel([backend]):
+                def step():
+                    o = F.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+                    o.backward(d_o)
+                step()
+                torch.cuda.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(2):
+                    step()
+                b.record()
+                torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / 2
+            B, H, N, d = q.shape
+            return {"what": "dense causal SDPA fwd+bwd over all N tokens, same shape and GPU",
+                    "backend": backend.name, "ms_per_step": round(ms, 3),
+                    "tflops": round(7 * B * H * N * N * d / (ms / 1e3) / 1e12, 1),  # causal: 2+5 N^2 d
+                    "layer_speedup": round(ms / ms_layer, 2)}
+        except RuntimeError:
+            continue
+    return {"what": "dense causal SDPA fwd+bwd", "unavailable": "no torch SDPA backend ran"}
 
 
 def run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world):
