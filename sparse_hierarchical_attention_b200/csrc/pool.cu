@@ -74,6 +74,16 @@ __device__ inline float tree_norm(const float* part) {
   return __fsqrt_rn(t[0]);
 }
 
+// Two-lane fp32 add (sm_100 f32x2): each lane rounds to nearest exactly as __fadd_rn does. Products
+// stay scalar (__fmul_rn): a packed multiply feeding a packed add did not reproduce the separately
+// rounded scalar pair on fp32 inputs.
+__device__ inline void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
 // Row id -> level and cell index, from the level offsets.
 __device__ inline void decode_rid(int64_t rid, const int64_t* off, int L, int& lvl, int64_t& cell) {
   lvl = 0;
@@ -172,13 +182,8 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
         raw[u] = make_uint4(0, 0, 0, 0);
         if (active && row0 + u < W) raw[u] = ldg16(X + (int64_t)(row0 + u) * D);
       }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int row = row0 + u;
-        if (row >= W) break;  // the same for every thread of the CTA
-        float x[VEC];
-        V::unpack(raw[u], x);
-        if (norm_of) part[((xi * STREAMS + s) * 16 + row) * PSTR + col] = group_sumsq<VEC>(x);
+      // one row: the span-sum level-0 store, the level sums, and the cells they complete
+      auto take_row = [&](int row, const float (&x)[VEC]) {
         if constexpr (MODE == MODE_SPANSUM) {
           if (active) {
             const int r = smap[s * W + row];
@@ -186,8 +191,13 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
           }
         }
         if constexpr (A > 0) {
+          if constexpr (MODE == MODE_PYRAMID) {
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[0][e] += x[e];
+            for (int e = 0; e < VEC; e += 2) add2(acc[0][e], acc[0][e + 1], x[e], x[e + 1]);
+          } else {  // scalar adds measured faster for the one-tensor span sums
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[0][e] += x[e];
+          }
 #pragma unroll
           for (int l = 0; l < A; ++l) {  // a finished level-l cell may finish level l+1, and so on
             if (--left[l] != 0) break;
@@ -211,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
             ++cellj[l];
             if (l + 1 < A) {
 #pragma unroll
-              for (int e = 0; e < VEC; ++e) acc[l + 1 < A ? l + 1 : l][e] += acc[l][e];
+              for (int e = 0; e < VEC; e += 2)
+                add2(acc[l + 1 < A ? l + 1 : l][e], acc[l + 1 < A ? l + 1 : l][e + 1], acc[l][e], acc[l][e + 1]);
             } else {
 #pragma unroll
               for (int e = 0; e < VEC; ++e) stage[xi][s][col * VEC + e] = acc[l][e];
@@ -220,6 +231,35 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
             for (int e = 0; e < VEC; ++e) acc[l][e] = 0.f;
           }
         }
+      };
+      if constexpr (MODE == MODE_SPANSUM) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int row = row0 + u;
+          if (row >= W) break;  // the same for every thread of the CTA
+          float x[VEC];
+          V::unpack(raw[u], x);
+          take_row(row, x);
+        }
+      } else {
+#pragma unroll
+      for (int u = 0; u < U; u += 2) {  // rows in pairs: their sums of squares run as f32x2
+        const int row = row0 + u;
+        if (row >= W) break;  // the same for every thread of the CTA
+        const bool second = row + 1 < W;
+        float x0[VEC], x1[VEC];
+        V::unpack(raw[u], x0);
+        V::unpack(raw[u + 1], x1);
+        if (norm_of) {
+          float a0 = 0.f, a1 = 0.f;  // each row's group in ascending order (SPEC section 2)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) add2(a0, a1, __fmul_rn(x0[e], x0[e]), __fmul_rn(x1[e], x1[e]));
+          part[((xi * STREAMS + s) * 16 + row) * PSTR + col] = a0;
+          if (second) part[((xi * STREAMS + s) * 16 + row + 1) * PSTR + col] = a1;
+        }
+        take_row(row, x0);
+        if (second) take_row(row + 1, x1);
+      }
       }
     }
   }
