@@ -76,8 +76,11 @@ const char* lh_status_string(int status);
 const char* lh_version(void);
 
 /* Validates a shape for the GPU path and fills `out` (may be NULL).
- * Method constraints: N % p^(L-1) == 0, S % C == 0, 1 <= S/C <= M+1.
- * GPU constraints: d in {64, 128}, 2 <= p <= 16, L <= 12, p^(L-1) <= 2^20, B*H <= 65535*... */
+ * Method constraints (LH_ERR_INVALID_ARG): B, H, N, d, S >= 1, p >= 2, L >= 1, dtype f32 or
+ *   bf16, N % p^(L-1) == 0, S % C == 0, 1 <= S/C <= M+1.
+ * GPU constraints (LH_ERR_UNSUPPORTED): d in {64, 128}; p <= 16; L <= 12; p^(L-1) <= 2^20;
+ *   B*H <= 65535; N + R < 2^31; (M + k) * 8 <= 200 KiB, because a chunk's candidate keys are
+ *   ranked in shared memory (at p = 4 this allows L <= 8). */
 int lh_validate(const lh_shape* shape, lh_sizes* out);
 
 /* Bytes of the workspace `ws` that the entry points below take. The first 256 bytes hold the

@@ -47,6 +47,18 @@ def test_unsupported_head_dim():
     assert _lib.lh_validate_status(Shape(1, 2, 4096, 96, 4, 3, 256 * 4)) == 2
 
 
+@pytest.mark.parametrize("shape,status", [
+    (Shape(1, 1, 32768, 128, 4, 8, 2 * 64), 0),      # M + k = 21907 keys: inside the limit
+    (Shape(1, 1, 131072, 128, 4, 9, 2 * 64), 2),     # M + k = 87443 keys: over 200 KiB
+    (Shape(1, 1, 2 * 17 * 17, 64, 17, 3, 2), 2),     # p = 17
+    (Shape(1, 1, 2 * 2 ** 12, 64, 2, 13, 2), 2),     # L = 13
+    (Shape(1, 1, 2 * 16 ** 2, 64, 16, 3, 2 * 17), 0),  # p = 16, L = 3
+    (Shape(1, 1, 2 * 2 ** 11, 64, 2, 12, 2 * 64), 0),  # p = 2, L = 12
+])
+def test_gpu_path_limits(shape, status):
+    assert _lib.lh_validate_status(shape) == status
+
+
 def test_null_pointers_rejected_before_launch():
     s = Shape(1, 2, 4096, 128, 4, 3, 1024).c()
     rc = _lib._lib.lh_layer_fwd(ctypes.byref(s), None, None, None, None, None, None, None)

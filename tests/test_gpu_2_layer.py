@@ -83,6 +83,9 @@ def test_unit_variance_literal_thresholds(name, B, H, N, S, dtype):
     (1, 2, 2048, 64, 2, 8, 128),        # p = 2
     (1, 1, 2187, 128, 3, 4, 81 * 4),    # p = 3
     (1, 1, 1280, 64, 4, 4, 20 * 7),     # C = 20, S = 140: ragged attention tiles
+    (1, 1, 2048, 64, 16, 3, 8 * 17),    # p = 16, the largest pooling factor
+    (1, 1, 4096, 64, 2, 12, 2 * 64),    # L = 12, the most levels: five tree levels and a coarse pass
+    (1, 1, 32768, 128, 4, 8, 2 * 64),   # M = 21844 candidates per chunk, near the shared-memory limit
 ])
 def test_layer_edge_cases(B, H, N, d, p, L, S, dtype):
     shape = Shape(B, H, N, d, p, L, S, dtype)
