@@ -310,42 +310,70 @@ def dense_sdpa_context(q, k, v, d_o, ms_layer):
 
 
 def run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world):
-    """Same metric through the public layer API from pinned host buffers: per step, copy Q,K,V,dO
-    in, run lh_layer_fwd + lh_layer_bwd, copy O, dQ, dK, dV out."""
+    """Same metric through the public layer API from pinned host buffers. Every step copies its
+    Q, K, V, dO in, runs lh_layer_fwd + lh_layer_bwd and copies O, dQ, dK, dV out. Two buffer
+    sets and two copy streams pipeline the steps: step t+1's inputs cross the host link while step
+    t's outputs cross it the other way (the link is full duplex) and while the GPU computes."""
     from sparse_hierarchical_attention_b200 import LighthouseLayer
     layer = LighthouseLayer(shape, dev)
     h_in = [t.cpu().pin_memory() for t in (q, k, v, d_o)]
-    h_out = [torch.empty_like(h_in[0]).pin_memory() for _ in range(4)]
-    d_in = [torch.empty_like(q) for _ in range(4)]
-    d_out = [torch.empty_like(q) for _ in range(4)]
+    h_out = [[torch.empty_like(h_in[0]).pin_memory() for _ in range(4)] for _ in range(2)]
+    d_in = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
+    d_out = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
     saved = layer.new_saved()
-    stream = torch.cuda.current_stream()
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    state = {"computed": [None, None], "copied": [None, None]}
 
-    def step():
-        for h, dbuf in zip(h_in, d_in):
-            dbuf.copy_(h, non_blocking=True)
-        layer.forward(d_in[0], d_in[1], d_in[2], o=d_out[0], saved=saved)
-        layer.backward(saved, d_in[3], dq=d_out[1], dk=d_out[2], dv=d_out[3])
-        for h, dbuf in zip(h_out, d_out):
-            h.copy_(dbuf, non_blocking=True)
+    def step(t, after=None):
+        b = t % 2
+        if after is not None:
+            s_in.wait_event(after)
+        if state["computed"][b] is not None:  # d_in[b] is free once the step before last computed
+            s_in.wait_event(state["computed"][b])
+        with torch.cuda.stream(s_in):
+            for h, dbuf in zip(h_in, d_in[b]):
+                dbuf.copy_(h, non_blocking=True)
+        ev_in = torch.cuda.Event()
+        ev_in.record(s_in)
+        main.wait_event(ev_in)
+        if state["copied"][b] is not None:  # d_out[b] is free once its outputs left
+            main.wait_event(state["copied"][b])
+        layer.forward(d_in[b][0], d_in[b][1], d_in[b][2], o=d_out[b][0], saved=saved)
+        layer.backward(saved, d_in[b][3], dq=d_out[b][1], dk=d_out[b][2], dv=d_out[b][3])
+        ev_c = torch.cuda.Event()
+        ev_c.record(main)
+        state["computed"][b] = ev_c
+        s_out.wait_event(ev_c)
+        with torch.cuda.stream(s_out):
+            for h, dbuf in zip(h_out[b], d_out[b]):
+                h.copy_(dbuf, non_blocking=True)
+        ev_o = torch.cuda.Event()
+        ev_o.record(s_out)
+        state["copied"][b] = ev_o
 
-    for _ in range(W):
-        step()
+    for t in range(W):
+        step(t)
     torch.cuda.synchronize()
+    state["computed"], state["copied"] = [None, None], [None, None]
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
+    a.record(main)
+    for t in range(K):
+        step(t, after=a if t == 0 else None)
+    for ev in state["copied"]:  # the last outputs have reached the host
+        if ev is not None:
+            main.wait_event(ev)
+    b.record(main)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world) / K
     layer.check()
     nbytes = sum(t.numel() * t.element_size() for t in h_in)
     return {"value": round(w.B * w.N * world / (ms / 1e3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": nbytes,
-            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out),
-            "api": "LighthouseLayer.forward/backward -> lh_layer_fwd/lh_layer_bwd"}
+            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out[0]),
+            "api": "LighthouseLayer.forward/backward -> lh_layer_fwd/lh_layer_bwd",
+            "pipelining": "two buffer sets; copies in, compute and copies out on three streams"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
