@@ -223,7 +223,8 @@ def run_ours(args, world, rank, local):
     wall = time.perf_counter() - t_wall
     barrier(world)
     clk = clocks.stop()
-    total_ms = sum(ev[s][0].elapsed_time(ev[s][-1]) for s in range(K))
+    step_ms = [ev[s][0].elapsed_time(ev[s][-1]) for s in range(K)]
+    total_ms = sum(step_ms)
     per_stage = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)) / K
                  for i, (name, _) in enumerate(stages)}
     value, ms_step = throughput(total_ms, K, B * N, world)
@@ -261,7 +262,8 @@ def run_ours(args, world, rank, local):
         del t
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4),
+        "ms_per_step_median_rank0": round(statistics.median(step_ms), 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic (seeded N(0,1) Q/K/V with the workload's row-scale recipe; dO N(0,1))",
         "config": {"workload": w.name, "describe": w.describe, "B": B, "H": H, "N": N, "d": d,
