@@ -128,6 +128,40 @@ def test_deterministic_bits():
         assert torch.equal(x, y)
 
 
+def test_layer_replays_as_one_cuda_graph():
+    """The layer allocates nothing and never synchronises, so a whole forward + backward step
+    captures into one CUDA graph; replays with new inputs give the eager results bit for bit."""
+    w = WORKLOADS["128k"]
+    shape = Shape(1, 2, 8192, w.d, w.p, w.L, 512, w.dtype)
+    layer = LighthouseLayer(shape)
+    saved = layer.new_saved()
+    ins = [torch.empty(1, 2, 8192, w.d, dtype=w.dtype, device="cuda") for _ in range(4)]
+    outs = [torch.empty_like(ins[0]) for _ in range(4)]
+
+    def step():
+        layer.forward(ins[0], ins[1], ins[2], o=outs[0], saved=saved)
+        layer.backward(saved, ins[3], dq=outs[1], dk=outs[2], dv=outs[3])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()  # warm the launch paths outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for seed in (3, 4):
+        for dst, src in zip(ins, make_inputs(w, "cuda", seed=seed, B=1, H=2, N=8192)):
+            dst.copy_(src)
+        g.replay()
+        got = [t.clone() for t in outs]
+        want = run_layer(shape, *ins)
+        assert torch.equal(got[0], want[0])
+        for x, y in zip(got[1:], want[2]):
+            assert torch.equal(x, y)
+    layer.check()
+
+
 def test_future_chunks_do_not_change_the_past():
     w = WORKLOADS["llama530m-98k"]
     N, S = 8192, 8 * 64
