@@ -11,9 +11,10 @@
 //   dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
 //           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K (dS from tensor memory).
 // Warp roles: warps 0-15 compute (warp w owns TMEM lanes 32(w%4)..+31 and column quarter w/4 of
-// each step); warp 16 (one lane) issues the TMA loads; warp 17 (one lane) issues the MMAs, so that
-// an MMA issue that waits for room in the tensor pipe never delays a load, and the accumulation of
-// a step is issued as soon as its P lands. The sides meet only at mbarriers (stage loaded, stage
+// each step); warp 16 (one lane) issues the TMA loads; warp 17 (one lane) issues the S/dP MMAs and
+// warp 18 (one lane) the accumulation MMAs, so that an MMA issue that waits for room in the tensor
+// pipe never delays a load or the other stream, and the accumulation of a step is issued as soon
+// as its P lands. The sides meet only at mbarriers (stage loaded, stage
 // free, S ready, S buffer free, P written, accumulation done; one arrival per warp), so the tensor
 // cores work on step it+1's S/dP and step it-1's accumulation while the warps do step it.
 // Q/dO (dkdv) and K/V (dq) come through four-stage TMA rings, with lse and D riding along as
@@ -26,6 +27,9 @@
 // dS each enter their product as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi). That is
 // one extra MMA per product and keeps the operand to ~16 bits. With one bf16 term, single dV
 // elements were off by 34% of their size.
+// The warps' element arithmetic runs on key (or query) pairs with packed f32x2 FMA, subtract and
+// multiply, each lane rounded as the scalar instruction is, so the results are those of the scalar
+// sequence exp2(s c - lse2), (dP - D) p, hi/lo split, with half the issue slots.
 // Every barrier that could run two phases ahead of a waiter is doubled, so that no parity wait
 // is ambiguous. All waits are bounded and report through the status word.
 #include "tc.cuh"
@@ -217,29 +221,40 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
       const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStQ) * 512) + qtr * 4;
       const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStQ) * 512 + 256) + qtr * 4;
       const int q0 = k0 + it * 64 + qtr * 16;
+      uint64_t p2[8], ds2[8];  // column pairs (2h, 2h+1), one f32x2 instruction per pair
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         const float4 lv = lv4[c4], dv = dv4[c4];
-        const float la[4] = {lv.x * kLog2e, lv.y * kLog2e, lv.z * kLog2e, lv.w * kLog2e};
-        const float da[4] = {dv.x, dv.y, dv.z, dv.w};
+        const uint64_t nla[2] = {f2_pack(-(lv.x * kLog2e), -(lv.y * kLog2e)),
+                                 f2_pack(-(lv.z * kLog2e), -(lv.w * kLog2e))};
+        const uint64_t da[2] = {f2_pack(dv.x, dv.y), f2_pack(dv.z, dv.w)};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c4 * 4 + e;
-          const float p = ex2(fmaf(st[c], scale_log2, -la[e]));
-          st[c] = p;
-          dpt[c] = p * (dpt[c] - da[e]);
+        for (int e = 0; e < 2; ++e) {
+          const int h = c4 * 2 + e;
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(st[2 * h], st[2 * h + 1]), c2, nla[e]), a0, a1);
+          p2[h] = f2_pack(ex2(a0), ex2(a1));
+          ds2[h] = f2_mul(p2[h], f2_sub(f2_pack(dpt[2 * h], dpt[2 * h + 1]), da[e]));
         }
       }
       if (q0 < k0 + 128) {  // steps that reach the diagonal: keys after the query are invisible
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (kj > q0 + c) { st[c] = 0.f; dpt[c] = 0.f; }
+        for (int h = 0; h < 8; ++h) {
+          float x0, x1, y0, y1;
+          f2_unpack(p2[h], x0, x1);
+          f2_unpack(ds2[h], y0, y1);
+          if (kj > q0 + 2 * h) { x0 = 0.f; y0 = 0.f; }
+          if (kj > q0 + 2 * h + 1) { x1 = 0.f; y1 = 0.f; }
+          p2[h] = f2_pack(x0, x1);
+          ds2[h] = f2_pack(y0, y1);
+        }
       }
       uint32_t wp[8], wq[8], wh[8], wl[8];
 #pragma unroll
       for (int h = 0; h < 8; ++h) {
-        split_bf16x2(st[2 * h], st[2 * h + 1], wp[h], wq[h]);
-        split_bf16x2(dpt[2 * h], dpt[2 * h + 1], wh[h], wl[h]);
+        split_bf16x2_f2(p2[h], wp[h], wq[h]);
+        split_bf16x2_f2(ds2[h], wh[h], wl[h]);
       }
       // the accumulate MMAs of the previous step read P^T and dS^T
       if (it > 0 && !wait_all(bar_acc, (it - 1) & 1)) break;
@@ -448,16 +463,29 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
       __syncwarp();
       if ((tid % 32) == 0) mbar_arrive(bar + 7 + (it & 1));  // this S buffer may be overwritten
       const int kj0 = it * 64 + qtr * 16;
+      uint64_t ds2[8];  // key pairs (2h, 2h+1), one f32x2 instruction per pair
+      {
+        const uint64_t c2 = f2_pack(scale_log2, scale_log2), nl2 = f2_pack(-l2, -l2), dl2 = f2_pack(dl, dl);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) dp[c] = ex2(fmaf(s[c], scale_log2, -l2)) * (dp[c] - dl);
+        for (int h = 0; h < 8; ++h) {
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(s[2 * h], s[2 * h + 1]), c2, nl2), a0, a1);
+          ds2[h] = f2_mul(f2_pack(ex2(a0), ex2(a1)), f2_sub(f2_pack(dp[2 * h], dp[2 * h + 1]), dl2));
+        }
+      }
       if (kj0 + 16 > q0) {  // steps that reach the diagonal: keys after the query are invisible
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (kj0 + c > qi) dp[c] = 0.f;
+        for (int h = 0; h < 8; ++h) {
+          float y0, y1;
+          f2_unpack(ds2[h], y0, y1);
+          if (kj0 + 2 * h > qi) y0 = 0.f;
+          if (kj0 + 2 * h + 1 > qi) y1 = 0.f;
+          ds2[h] = f2_pack(y0, y1);
+        }
       }
       uint32_t wh[8], wl[8];  // dS = hi + lo: this quarter's 16 keys as 8 columns of pairs each
 #pragma unroll
-      for (int h = 0; h < 8; ++h) split_bf16x2(dp[2 * h], dp[2 * h + 1], wh[h], wl[h]);
+      for (int h = 0; h < 8; ++h) split_bf16x2_f2(ds2[h], wh[h], wl[h]);
       // the accumulate MMAs of the previous step read dS
       if (it > 0 && !wait_all(bar + 10 + ((it - 1) & 1), ((it - 1) >> 1) & 1)) break;
       tc_fence_after();

@@ -21,6 +21,10 @@
 //    thousands of tokens.
 //  - The running max is updated lazily: O and l are rescaled only when a row's max grows by more
 //    than 2^8, which keeps every exponent bounded and skips most TMEM round trips.
+//  - The softmax warps are bound by instruction issue and the ex2 unit, so their arithmetic is
+//    counted: the row max is taken over the raw scores with three-input max (exact, as the scale is
+//    positive), the scale enters the exponent through one packed f32x2 FMA per pair of keys, and
+//    the row sums and the lo residuals are packed f32x2 adds and subtracts.
 //  - Key blocks above the diagonal are skipped; the diagonal block is masked.
 // Tensor-core order: S_0, S_1, PV_0, S_2, PV_1, ... The softmax of S_j therefore overlaps PV_{j-1}
 // and S_{j+1}; it writes P_j only after PV_{j-1} has finished reading P and O.
@@ -203,8 +207,8 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(r0[e]) * scale_log2;
-          s[32 + e] = __uint_as_float(r1[e]) * scale_log2;
+          s[e] = __uint_as_float(r0[e]);  // raw scores: the scale goes into the exponent's FMA
+          s[32 + e] = __uint_as_float(r1[e]);
         }
       } else {
 #pragma unroll
@@ -218,25 +222,36 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         for (int e = 0; e < 64; ++e)
           if (half * 64 + e > row) s[e] = -INFINITY;
       }
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float m4[4];
 #pragma unroll
-      for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], s[e]);
-      const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      for (int c = 0; c < 4; ++c) {  // four chains of 16; the scale is positive, so max commutes with it
+        m4[c] = max3(s[16 * c], s[16 * c + 1], s[16 * c + 2]);
+#pragma unroll
+        for (int e = 16 * c + 3; e < 16 * c + 15; e += 2) m4[c] = max3(m4[c], s[e], s[e + 1]);
+        m4[c] = fmaxf(m4[c], s[16 * c + 15]);
+      }
+      const float mloc = max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;
       xch[((j & 1) * 2 + half) * 128 + row] = mloc;
       pair_sync();
       const float mt = fmaxf(mloc, xch[((j & 1) * 2 + (half ^ 1)) * 128 + row]);
       const bool grow = mt > m_used + 8.0f;
       const float m_new = grow ? mt : m_used;
       const float alpha = grow ? exp2f(m_used - m_new) : 1.0f;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
+      uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
       uint32_t ph[32], pl[32];
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        const float x0 = ex2(s[e] - m_new), x1 = ex2(s[e + 1] - m_new);
-        sum4[(e >> 1) & 3] += x0 + x1;
-        split_bf16x2(x0, x1, ph[e / 2], pl[e / 2]);
+      for (int e = 0; e < 64; e += 2) {  // p = 2^(s * scale - m), a pair per instruction
+        float a0, a1;
+        f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nm2), a0, a1);
+        const uint64_t x = f2_pack(ex2(a0), ex2(a1));
+        sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], x);
+        split_bf16x2_f2(x, ph[e / 2], pl[e / 2]);
       }
-      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      float sa0, sa1, sb0, sb1;
+      f2_unpack(sum2[0], sa0, sa1);
+      f2_unpack(sum2[1], sb0, sb1);
+      l = l * alpha + ((sa0 + sa1) + (sb0 + sb1));
       m_used = m_new;
       // PV_{j-1} must be done before P and O are touched again
       if (j > 0) {

@@ -245,5 +245,53 @@ __device__ inline void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
+// Two-lane fp32 arithmetic (sm_100 f32x2): one instruction for a pair, each lane rounded to
+// nearest as the scalar instruction rounds it.
+__device__ inline uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ inline void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ inline uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ inline uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ inline uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ inline uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three: sm_100's three-input max, which issues at the two-input rate
+__device__ inline float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// split_bf16x2 for a packed pair (a in the low lane): the residual is one packed subtract.
+__device__ inline void split_bf16x2_f2(uint64_t ab, uint32_t& hi, uint32_t& lo) {
+  float a, b;
+  f2_unpack(ab, a, b);
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  float la, lb;
+  f2_unpack(f2_sub(ab, f2_pack(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u))), la, lb);
+  __nv_bfloat162 l = __floats2bfloat162_rn(la, lb);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 }  // namespace tc
 }  // namespace lh
