@@ -37,6 +37,12 @@ from sparse_hierarchical_attention_b200.workloads import WORKLOADS, make_inputs 
 METRIC = "Lighthouse layer fwd+bwd tokens/s at N=128K, 1 B200; % of HBM / tensor roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of this command with
+# `-k regex:"attn_|delta_kernel"`) of one attention-backward call (D, dK/dV and dQ launches) of the
+# current kernels, per workload. Writes still in L2 when a launch ends are not counted. These are
+# the roofline's `traffic` for that stage; any change to those kernels makes them stale.
+MEASURED_TRAFFIC = {("32k", "attn_bwd"): 205012992, ("llama530m-98k", "attn_bwd"): 142262784,
+                    ("128k", "attn_bwd"): 1073160960, ("1m", "attn_bwd"): 654756864}
 
 
 def parse():
@@ -247,7 +253,9 @@ def run_ours(args, world, rank, local):
     rf = stage_report[dom]
     roofline = {"kernel": dom, "bound": "hbm" if kind == "hbm" else "tensor",
                 "achieved": rf["achieved"], "peak": pk_["hbm_gbs"] if kind == "hbm" else pk_["bf16_tflops"],
-                "unit": rf["unit"], "frac": rf["frac"], "traffic": None,
+                "unit": rf["unit"], "frac": rf["frac"],
+                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)),
+                "traffic_scope": "bytes of one stage call (all its launches), like achieved",
                 "peak_source": f"{src} ({'hbm_gbs' if kind == 'hbm' else 'bf16_tflops'})",
                 "units_per_launch": amount}
     nf, nb = lh.lh_launches(shape)

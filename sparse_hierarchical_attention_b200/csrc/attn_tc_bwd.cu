@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                  const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                  const float* __restrict__ lse, const float* __restrict__ delta,
-                 float* __restrict__ dK, float* __restrict__ dV, int S, float sigma,
+                 float* __restrict__ dK, float* __restrict__ dV, int S, int BH, float sigma,
                  float scale_log2, uint32_t* status) {
   using Ly = LayDKV<D>;
   constexpr int KB = Ly::KB;
@@ -91,9 +91,9 @@ attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__
   uint64_t* const bar_stfree = bar + 9;    // + stage
 
   const int tid = threadIdx.x, warp = tid / 32;
-  // grid (BH, blocks): heads vary fastest, so every head's heaviest blocks launch first
-  const int kb = blockIdx.y;  // low key blocks see the most queries
-  const int bh = blockIdx.x;
+  const int kb = blockIdx.y;  // low key blocks see the most queries: heaviest first in a group
+  const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
+  if (bh >= BH) return;  // the last group may be partial
   const int g0 = bh * S;
   const int k0 = kb * 128;
   const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                const float* __restrict__ lse, const float* __restrict__ delta,
-               float* __restrict__ dQ, int S, float sigma, float scale_log2, uint32_t* status) {
+               float* __restrict__ dQ, int S, int BH, float sigma, float scale_log2, uint32_t* status) {
   using Ly = LayDQ<D>;
   constexpr int KB = Ly::KB;
   extern __shared__ uint8_t smem_raw[];
@@ -339,8 +339,9 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / 128;
-  const int qb = nqb - 1 - (int)blockIdx.y;  // heads vary fastest; heaviest blocks first
-  const int bh = blockIdx.x;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // heaviest blocks first within a head group
+  const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
+  if (bh >= BH) return;  // the last group may be partial
   const int g0 = bh * S;
   const int q0 = qb * 128;
   const int nit = (q0 + 128) / 64;  // 64-row key blocks up to the diagonal
@@ -566,14 +567,16 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
   const int smem1 = LayDKV<D>::BYTES + 1024 > 120 * 1024 ? LayDKV<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dkdv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1);
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc<D><<<dim3((unsigned)g.BH, (unsigned)(g.S / 128)), kThreads, smem1, st>>>(
-      k128, v128, q64, do64, lse, delta, dk, dv, g.S, sigma, scale_log2, status);
+  const dim3 grid((unsigned)(g.BH < kHeadGroup ? g.BH : kHeadGroup), (unsigned)(g.S / 128),
+                  (unsigned)((g.BH + kHeadGroup - 1) / kHeadGroup));
+  attn_bwd_dkdv_tc<D><<<grid, kThreads, smem1, st>>>(
+      k128, v128, q64, do64, lse, delta, dk, dv, g.S, (int)g.BH, sigma, scale_log2, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int smem2 = LayDQ<D>::BYTES + 1024 > 120 * 1024 ? LayDQ<D>::BYTES + 1024 : 120 * 1024;
   e = cudaFuncSetAttribute(attn_bwd_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_tc<D><<<dim3((unsigned)g.BH, (unsigned)(g.S / 128)), kThreads, smem2, st>>>(
-      q128, do128, k64, v64, lse, delta, dq, g.S, sigma, scale_log2, status);
+  attn_bwd_dq_tc<D><<<grid, kThreads, smem2, st>>>(
+      q128, do128, k64, v64, lse, delta, dq, g.S, (int)g.BH, sigma, scale_log2, status);
   return cudaGetLastError();
 }
 

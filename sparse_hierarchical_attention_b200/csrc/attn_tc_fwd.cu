@@ -64,7 +64,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, float* __restrict__ O, float* __restrict__ lse,
-            int S, float scale_log2, uint32_t* status) {
+            int S, int BH, float scale_log2, uint32_t* status) {
   using Ly = Layout<D>;
   constexpr int KB = Ly::KB;
   constexpr int kStV = v_stages<D>();
@@ -85,8 +85,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
   const int tid = threadIdx.x, warp = tid / 32;
   const int nqb = S / BM;
-  const int qb = nqb - 1 - (int)blockIdx.y;  // heads vary fastest; heaviest tiles first
-  const int bh = blockIdx.x;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // heaviest tiles first within a head group
+  const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
+  if (bh >= BH) return;  // the last group may be partial
   const int grow0 = bh * S;                  // first row of this (b,h) in the [BH*S, D] view
   const int nkb = qb + 1;
 
@@ -372,19 +373,20 @@ cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, con
       !make_tmap_rows(&mv, vs, rows, g.d))
     return cudaErrorInvalidValue;
   const float scale_log2 = (1.0f / sqrtf((float)g.d)) * 1.4426950408889634f;
-  dim3 grid((unsigned)g.BH, (unsigned)(g.S / BM));
+  const unsigned gx = g.BH < kHeadGroup ? (unsigned)g.BH : (unsigned)kHeadGroup;
+  dim3 grid(gx, (unsigned)(g.S / BM), (unsigned)((g.BH + kHeadGroup - 1) / kHeadGroup));
   cudaError_t e;
   if (g.d == 128) {
     const int smem = Layout<128>::BYTES + 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, scale_log2, status);
+      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status);
   } else {
     // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
     const int smem = Layout<64>::BYTES + 1024 > 120 * 1024 ? Layout<64>::BYTES + 1024 : 120 * 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, scale_log2, status);
+      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status);
   }
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -23,6 +23,14 @@ namespace tc {
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
+// Attention grids: blockIdx.x = head within a group of kHeadGroup heads, blockIdx.y = row block
+// (heaviest first), blockIdx.z = head group. CTAs are dispatched x fastest, so the CTAs in flight
+// cover one or two groups, whose K/V (or Q/dO) tiles stay in L2 (8 heads at S = 8192, d = 128:
+// 32 MB). Ordering heads fastest over all heads instead re-read those tiles from DRAM 3-4 times
+// at 32 heads (128 MB in flight); within a group the heaviest-first order still balances the
+// causal tail.
+constexpr int kHeadGroup = 8;
+
 __device__ inline uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
