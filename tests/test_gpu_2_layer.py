@@ -81,6 +81,7 @@ def test_unit_variance_literal_thresholds(name, B, H, N, S, dtype):
     (2, 2, 1024, 128, 4, 4, 16 * 85),   # m = M + 1: everything selected
     (1, 2, 4096, 128, 4, 6, 4),         # m = 1: only the coarsest cells
     (1, 2, 2048, 64, 2, 8, 128),        # p = 2
+    (1, 2, 4096, 128, 2, 3, 1024 * 3),  # p = 2, L = 3 (the pages' best ablation): 4-token chunks, M = 6
     (1, 1, 2187, 128, 3, 4, 81 * 4),    # p = 3
     (1, 1, 1280, 64, 4, 4, 20 * 7),     # C = 20, S = 140: ragged attention tiles
     (1, 1, 2048, 64, 16, 3, 8 * 17),    # p = 16, the largest pooling factor
