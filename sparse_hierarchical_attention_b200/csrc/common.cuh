@@ -65,6 +65,11 @@ template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 }
 
 __device__ inline uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, size a multiple of 16); a hint that
+// holds no registers and changes no result.
+__device__ inline void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ inline void stg16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
 __device__ inline void raise_fault(uint32_t* status, uint32_t bit) {

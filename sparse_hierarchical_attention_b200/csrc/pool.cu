@@ -174,8 +174,18 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
     const E* const X = static_cast<const E*>(a.x[xi]) + (bh * a.N + tok0) * D + col * VEC;
     E* const PX = static_cast<E*>(a.px[MODE == MODE_PYRAMID ? xi : 0]);
     const bool norm_of = NORMS && a.do_score && xi < 2;  // Q and K rows feed the score
+    // L2 prefetch ahead of the loads. The kernel waits mostly on load latency, and the rows a
+    // warp holds in flight are capped by its registers (the span-sum kernel sits at the register
+    // limit of 4 CTAs per SM). A bulk prefetch into L2 holds no registers: one lane of the group
+    // asks for the stream's rows PF ahead (contiguous, U rows per request), so the loads then hit
+    // L2. Measured per mode: PF = 16 for the pyramid (U = 8), PF = 4 for the span sums (U = 4).
+    constexpr int PF = MODE == MODE_PYRAMID ? 16 : 4;
+    if (active && col == 0)
+      prefetch_l2(X, (uint32_t)((W < PF ? W : PF) * D * sizeof(E)));
 #pragma unroll 1
     for (int row0 = 0; row0 < W; row0 += U) {
+      if (active && col == 0 && row0 + PF < W)  // an active stream's W rows all lie inside x
+        prefetch_l2(X + (int64_t)(row0 + PF) * D, (uint32_t)(min(U, W - (row0 + PF)) * D * sizeof(E)));
       uint4 raw[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
