@@ -184,7 +184,7 @@ def test_future_chunks_do_not_change_the_past():
 def test_full_size_sampled_heads(name, unit):
     """Full-size workload in the benchmark's launch; the oracle checks the last head whole.
 
-    unit=True drops the row scales, so the benchmark spec's unit-variance limits apply literally.
+    unit=True drops the row scales, so the unit-variance acceptance limits apply literally.
     """
     w = WORKLOADS[name]
     shape = Shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S, w.dtype)
