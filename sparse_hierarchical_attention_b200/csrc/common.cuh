@@ -71,6 +71,12 @@ __device__ inline void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 __device__ inline void stg16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+// Store with the evict-first (streaming) policy, for final outputs that no later kernel of the
+// step reads back: the L2 then keeps the lines that are reused (the covering rows in the spread).
+__device__ inline void stg16_stream(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w) : "memory");
+}
 
 __device__ inline void raise_fault(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);

@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
               for (int e = 0; e < VEC; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(x[e], w));
             }
           }
-          stg16(dst + (int64_t)t * D, Vec<E>::pack(out));
+          stg16_stream(dst + (int64_t)t * D, Vec<E>::pack(out));  // O or dQ/dK/dV: final outputs
         }
       }
     }
