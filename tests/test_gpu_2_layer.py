@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     import sparse_hierarchical_attention_b200 as lh
-    from sparse_hierarchical_attention_b200 import LighthouseLayer, Shape, saved_views
+    from sparse_hierarchical_attention_b200 import LighthouseAttention, LighthouseLayer, Shape, saved_views
     from sparse_hierarchical_attention_b200.workloads import WORKLOADS, make_inputs
 
 from gpu_util import assert_close, g_of, np64, store_of
@@ -202,3 +202,24 @@ def test_full_size_sampled_heads(name, unit):
     assert_close(np64(o[sl]), wo, w.dtype, "O", mode="literal" if unit else "scaled")
     for got, want, n in zip(grads, wgrads, ("dQ", "dK", "dV")):
         assert_close(np64(got[sl]), want, w.dtype, n)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_autograd_module_matches_layer_calls(dtype):
+    """LighthouseAttention (nn.Module over a torch.autograd.Function) returns the O, dQ, dK and dV
+    of explicit LighthouseLayer forward/backward calls on the same inputs, bit for bit: the same
+    kernels run, and the layer is deterministic."""
+    name, B, H, N, S = SMALL[1] if dtype == torch.bfloat16 else SMALL[0]
+    w = WORKLOADS[name]
+    shape = Shape(B, H, N, w.d, w.p, w.L, S, dtype)
+    q, k, v, d_o = (t.to(dtype) for t in make_inputs(w, "cuda", seed=3, B=B, H=H, N=N))
+    o_ref, _, (dq_ref, dk_ref, dv_ref) = run_layer(shape, q, k, v, d_o)
+    attn = LighthouseAttention(w.p, w.L, S)
+    qq, kk, vv = (x.clone().requires_grad_() for x in (q, k, v))
+    o = attn(qq, kk, vv)
+    o.backward(d_o)
+    assert o.dtype == dtype and o.shape == q.shape
+    assert torch.equal(o.detach(), o_ref)
+    assert torch.equal(qq.grad, dq_ref)
+    assert torch.equal(kk.grad, dk_ref)
+    assert torch.equal(vv.grad, dv_ref)
