@@ -32,17 +32,45 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_hierarchical_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+from workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "Lighthouse layer fwd+bwd tokens/s at N=128K, 1 B200; % of HBM / tensor roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of this command with
-# `-k regex:"attn_|delta_kernel"`) of one attention-backward call (D, dK/dV and dQ launches) of the
-# current kernels, per workload. Writes still in L2 when a launch ends are not counted. These are
-# the roofline's `traffic` for that stage; any change to those kernels makes them stale.
-MEASURED_TRAFFIC = {("32k", "attn_bwd"): 205012992, ("llama530m-98k", "attn_bwd"): 142262784,
-                    ("128k", "attn_bwd"): 1073160960, ("1m", "attn_bwd"): 654756864}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one call of a stage, from one ncu
+# capture, with the digest of the kernel sources the capture ran. `roofline.traffic` reports them
+# only while those sources are unchanged; after any change it is null and `traffic_stale` true.
+# (workload, stage) -> (bytes per call, source digest, how the bytes were obtained)
+MEASURED_TRAFFIC = {}
+# the sources whose kernels run in each stage
+STAGE_SOURCES = {
+    "pyramid_score": ["pool.cu"], "select": ["select.cu"], "gather": ["gather_scatter.cu"],
+    "attn_fwd": ["attn_tc_fwd.cu", "tc.cuh"], "scatter": ["gather_scatter.cu"],
+    "scatter_bwd": ["pool.cu"], "attn_bwd": ["attn_tc_bwd.cu", "tc.cuh"],
+    "gather_bwd": ["gather_scatter.cu"],
+}
+
+
+def source_digest(stage):
+    """sha256 (first 16 hex digits) of the CUDA sources of a stage's kernels, plus common.cuh."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_hierarchical_attention_b200", "csrc")
+    for name in STAGE_SOURCES[stage] + ["common.cuh"]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_of(workload, stage):
+    """(bytes or None, stale flag, note) of the measured DRAM traffic of one stage call."""
+    rec = MEASURED_TRAFFIC.get((workload, stage))
+    if rec is None:
+        return None, False, "not captured for this workload"
+    nbytes, digest, how = rec
+    if digest != source_digest(stage):
+        return None, True, "kernel sources changed since the capture"
+    return nbytes, False, how
 
 
 def parse():
@@ -254,7 +282,9 @@ def run_ours(args, world, rank, local):
     roofline = {"kernel": dom, "bound": "hbm" if kind == "hbm" else "tensor",
                 "achieved": rf["achieved"], "peak": pk_["hbm_gbs"] if kind == "hbm" else pk_["bf16_tflops"],
                 "unit": rf["unit"], "frac": rf["frac"],
-                "traffic": MEASURED_TRAFFIC.get((args.workload, dom)),
+                "traffic": traffic_of(args.workload, dom)[0],
+                "traffic_stale": traffic_of(args.workload, dom)[1],
+                "traffic_note": traffic_of(args.workload, dom)[2],
                 "traffic_scope": "bytes of one stage call (all its launches), like achieved",
                 "peak_source": f"{src} ({'hbm_gbs' if kind == 'hbm' else 'bf16_tflops'})",
                 "units_per_launch": amount}
@@ -274,10 +304,7 @@ def run_ours(args, world, rank, local):
         "ms_per_step_median_rank0": round(statistics.median(step_ms), 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic (seeded N(0,1) Q/K/V with the workload's row-scale recipe; dO N(0,1))",
-        "config": {"workload": w.name, "describe": w.describe, "B": B, "H": H, "N": N, "d": d,
-                   "p": w.p, "L": w.L, "S": S, "global_batch": B * world, "seq_len": N,
-                   "parallelism": f"replicas x{world} (independent heads, no collective)",
-                   "l2": "inputs larger than L2 (each input tensor > 126 MB); no flush"},
+        "config": workload_config(w, world),
         "stages": stage_report, "roofline": roofline, "gpu_launches": (nf + nb) * K,
         "clocks": clk, "wall_s_timed": round(wall, 3),
     }
@@ -387,6 +414,14 @@ def run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
+def workload_config(w, world):
+    """The `config` object of both arms' JSON lines: the workload, named by what it is."""
+    return {"workload": w.name, "describe": w.describe, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "p": w.p, "L": w.L, "S": w.S, "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": f"replicas x{world} (independent heads, no collective)",
+            "l2": "inputs larger than L2 (each input tensor > 126 MB); no flush"}
+
+
 def oracle_sample(w, frac, seed=0):
     """One head, the first N/frac tokens (same p, L and rows per chunk), on the host."""
     N, S = w.N // frac, w.S // frac
@@ -394,7 +429,15 @@ def oracle_sample(w, frac, seed=0):
     return [t.to(torch.float64).numpy() for t in (q, k, v, d_o)], N, S
 
 
+def single_threaded():
+    """Limits the BLAS thread pools to one thread while the oracle is timed; returns the
+    limiter (a context manager) and the number of threads the timing then uses."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1), 1
+
+
 def time_oracle(w, frac, steps=1):
+    """Seconds of one oracle forward + backward over one head of N/frac tokens."""
     import oracle as O
     (q, k, v, d_o), N, S = oracle_sample(w, frac)
     geo = O.Geometry(N, w.p, w.L, S).check()
@@ -410,54 +453,64 @@ def time_oracle(w, frac, steps=1):
     return value, dt, N, S
 
 
-def cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
-    except Exception:
-        return os.cpu_count() or 1
+def pick_sample(w, budget_s, runs):
+    """Largest head prefix (1, 1/4 or 1/16 of the tokens) whose `runs` oracle passes are
+    projected to fit `budget_s`, from one timed pass at 1/16. The oracle's time grows about as
+    the sample's tokens to the power 1.5 (its attention is quadratic in the kept rows)."""
+    _, t16, _, _ = time_oracle(w, 16)
+    for frac in (1, 4):
+        if runs * t16 * (16 / frac) ** 1.5 <= budget_s:
+            return frac, t16
+    return 16, t16
 
 
-def cpu_baseline(w, budget_s=25.0):
-    """The oracle on one head: the whole head if it fits the budget, else a prefix."""
-    frac = 16
-    value, dt, N, S = time_oracle(w, frac)
-    for f in (4, 1):  # grow the sample while the projected time (about linear in N) fits
-        if dt * (frac / f) * 1.3 <= budget_s:
-            frac = f
-            value, dt, N, S = time_oracle(w, frac)
-        else:
-            break
-    return {"value": round(value, 2), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"head 0 of {w.B * w.H}, first {N} of {w.N} tokens (S={S}, same p, L, "
-                      f"rows per chunk), fwd+bwd in {dt:.2f}s; tokens/s = {N}/({dt:.2f}s x "
-                      f"{w.B * w.H} heads)." + ("" if N == w.N else " A prefix has cheaper "
-                      "attention per token than the whole sequence, so this overstates the "
-                      "oracle's full-workload rate.")}
+def sample_note(w, N, S):
+    return (f"head 0 of {w.B * w.H}, first {N} of {w.N} tokens (S={S}, same p, L, rows per "
+            f"chunk)" + ("" if N == w.N else "; a prefix has cheaper attention per token than "
+            "the whole sequence, so this overstates the oracle's full-workload rate"))
 
 
-def run_reference(args, world, rank):
+def cpu_baseline(w, budget_s=30.0):
+    """The oracle, single-threaded, on one head: the whole head if it fits the budget, else the
+    longest prefix that does."""
+    limiter, cores = single_threaded()
+    with limiter:
+        frac, _ = pick_sample(w, budget_s, 1)
+        value, dt, N, S = time_oracle(w, frac)
+    return {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{sample_note(w, N, S)}; fwd+bwd in {dt:.2f}s on one thread; tokens/s = "
+                      f"{N}/({dt:.2f}s x {w.B * w.H} heads)"}
+
+
+def run_reference(args, world, rank, budget_s=180.0):
+    """The reference arm: the CPU oracle as it stands, single-threaded, on the GPU arm's
+    workload and config. Each step is a bounded sample of it: one head (every head is the same
+    problem), whole if all warm-up and timed steps fit about three minutes, else its longest
+    prefix that does. The value is the layer's tokens/s if the B*H heads ran one after another
+    on this core. This process imports only the oracle and the input generator, never the CUDA
+    library."""
     w = WORKLOADS[args.workload]
     if rank != 0:
         return None
-    frac = 16
-    for _ in range(args.warmup):
-        time_oracle(w, frac)
-    t0 = time.perf_counter()
-    vals = [time_oracle(w, frac)[1] for _ in range(args.steps)]
-    total = time.perf_counter() - t0
-    dt = sum(vals) / len(vals)
-    N = w.N // frac
+    limiter, cores = single_threaded()
+    with limiter:
+        frac, _ = pick_sample(w, budget_s, args.steps + args.warmup)
+        for _ in range(args.warmup):
+            time_oracle(w, frac)
+        t0 = time.perf_counter()
+        runs = [time_oracle(w, frac) for _ in range(args.steps)]
+        total = time.perf_counter() - t0
+    dt = sum(r[1] for r in runs) / len(runs)
+    N, S = runs[0][2], runs[0][3]
     value = N / (dt * w.H * w.B)
-    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-          "sample": f"each step: head 0 of {w.B * w.H}, first {N} of {w.N} tokens, fwd+bwd"}
+    cb = {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+          "sample": f"each step: {sample_note(w, N, S)}; fwd+bwd on one thread; tokens/s = "
+                    f"{N}/(seconds per step x {w.B * w.H} heads)"}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * dt, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe as our arm)",
-            "config": {"workload": w.name, "describe": w.describe, "sample_tokens": N},
-            "cpu_baseline": cb, "wall_s": round(total, 2),
+            "config": workload_config(w, world), "cpu_baseline": cb, "wall_s": round(total, 2),
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -30,8 +30,10 @@
  *  - Row ids (idx) are int32 ids into the concatenated pyramid of each (b, h): tokens have ids
  *    0..N-1; cell j of level l >= 1 has id N + off_l + j with off_l = sum_{l'=1}^{l-1} N/p^l'.
  *    Levels 1..L-1 are stored in one [B, H, R, d] tensor per X in Q, K, V, level 1 first.
- *  - Numerics follow SPEC.md: fp32 accumulation everywhere, scores in a fixed fp32 order so
- *    the selection is reproducible bit for bit, one rounding to the storage dtype.
+ *  - Numerics: fp32 accumulation everywhere; scores in one fixed fp32 order (16-byte groups of
+ *    separately rounded squares in ascending order, a halving tree over the groups, a correctly
+ *    rounded square root) so that the selection is reproducible bit for bit; one rounding to the
+ *    storage dtype.
  */
 #ifndef LIGHTHOUSE_LH_H
 #define LIGHTHOUSE_LH_H
@@ -62,7 +64,7 @@ typedef struct {
   int dtype; /* lh_dtype */
 } lh_shape;
 
-/* Sizes derived from a shape (SPEC.md section 0). */
+/* Sizes derived from a shape (the pages' notation: p, L, N per level, budget S). */
 typedef struct {
   int64_t R;  /* pooled rows per (b,h): sum_{l=1}^{L-1} N/p^l */
   int64_t C;  /* chunks = coarsest cells = N/p^(L-1) */
@@ -163,17 +165,25 @@ int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void
  *  - The per-row scratch (D_i = do_sub[i] . o_sub[i]) lives in a file-scope device array of
  *    256 + 4 * LH_STATIC_SCRATCH_ROWS bytes (about 4 MiB). Every GPU that loads the library
  *    holds it until the process exits. The call itself allocates and frees nothing.
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *    with that device current. Make that first call before any stream capture.
+ *  - The first call on a device (or of lh_check_static) looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and clears its status word with a
+ *    synchronous memset. Make that first call before any stream capture.
  *  - Returns LH_ERR_WORKSPACE, launching nothing, when B*H*S > LH_STATIC_SCRATCH_ROWS.
- *  - All calls share the one array, which keeps the previous call's contents. Calls that
- *    overlap on the GPU (different streams, no ordering between them) race on it.
+ *  - All calls share the one array, which keeps the previous call's contents. D is rewritten
+ *    in full by every call before it is read. Calls that overlap on the GPU (different
+ *    streams, no ordering between them) race on it.
+ *  - Device faults (bounded wait ran out) latch in the array's status word; lh_check_static
+ *    reads and clears it.
  *  - Other arguments, layouts and errors as lh_attn_bwd. */
 #define LH_STATIC_SCRATCH_ROWS (1 << 20)
 int lh_attn_bwd_static(const lh_shape* shape, const void* q_sub, const void* k_sub,
                        const void* v_sub, const float* o_sub, const float* lse,
                        const void* do_sub, float* dq_sub, float* dk_sub, float* dv_sub,
                        void* stream);
+/* The status word of lh_attn_bwd_static's static scratch on the current device: synchronises
+ * `stream`, reads and clears the word. Returns LH_OK or LH_ERR_DEVICE (then *flags, if
+ * non-NULL, holds the fault bits as in lh_check). Allocates nothing. */
+int lh_check_static(void* stream, uint32_t* flags);
 
 /* Number of kernel launches one lh_layer_fwd (*fwd) and one lh_layer_bwd (*bwd) make for this
  * shape (either pointer may be NULL). Host-side plan only; launches nothing. */

@@ -4,9 +4,10 @@ This module is the checker, not the product. Only the tests, the smoke check and
 baseline leg of the benchmark may import it. The CUDA library never calls it, and it calls
 nothing of the CUDA library.
 
-It computes exactly what SPEC.md fixes, step by step, in float64 from the exact input values.
-The one exception is the ranking score, which decides an integer result. It is computed in
-float32 in the order SPEC.md section 2 states, so that the GPU path can match it bit for bit.
+It computes the layer step by step, in float64 from the exact input values, with every
+convention the pages leave open fixed as stated next to the step that takes it. The one
+exception is the ranking score, which decides an integer result. It is computed in float32 in
+one fixed order (row_norm_f32), so that the GPU path can match it bit for bit.
 
 Sources: *Long Context Pre-Training with Lighthouse Attention* (gist.science summary,
 technical summary section 2.A-2.D and section 5), and the Nous Research article on
@@ -30,11 +31,12 @@ import numpy as np
 
 
 # ---------------------------------------------------------------------------------------
-# Shape bookkeeping (SPEC section 0)
+# Shape bookkeeping (the pages' notation: p, L, N_l = N / p^l, budget S)
 # ---------------------------------------------------------------------------------------
 @dataclass(frozen=True)
 class Geometry:
-    """Derived sizes of one layer call; see the notation table of SPEC section 0."""
+    """Derived sizes of one layer call: R pooled rows, C chunks of T = p^(L-1) tokens,
+    m = S / C rows and k = m - 1 picks per chunk, M candidates per chunk."""
 
     N: int
     p: int
@@ -116,11 +118,11 @@ def build_pyramid(x, geo: Geometry):
 
 
 # ---------------------------------------------------------------------------------------
-# 2. Scores: l2 norms of Q and K per head, max-pooled upward, summed (SPEC section 2;
-#    Lighthouse summary, section 2.B; the article's "two scalar scores per cell").
+# 2. Scores: l2 norms of Q and K per head, max-pooled upward, summed (Lighthouse summary,
+#    section 2.B; the article's "two scalar scores per cell").
 # ---------------------------------------------------------------------------------------
 def row_norm_f32(x, g):
-    """fp32 l2 norm of each row of x[..., d] in the SPEC section 2 order.
+    """fp32 l2 norm of each row of x[..., d] in one fixed order.
 
     Groups of g consecutive coordinates are summed in ascending order, each square rounded
     on its own; the group sums are then combined by a halving tree; then a rounded sqrt.
@@ -154,8 +156,8 @@ def score(q, k, geo: Geometry, g):
 
 
 # ---------------------------------------------------------------------------------------
-# 3.-4. Stratified top-K and the causal order of the subsequence (SPEC sections 3-4;
-#    Lighthouse summary, sections 2.B-2.C; the article keeps the coarsest level always).
+# 3.-4. Stratified top-K and the causal order of the subsequence (Lighthouse summary,
+#    sections 2.B-2.C; the article keeps the coarsest level always).
 # ---------------------------------------------------------------------------------------
 def select_topk(r, geo: Geometry):
     """r: float32 [B,H,N+R] -> idx int32 [B,H,S] (row ids, in subsequence order)."""
@@ -200,14 +202,14 @@ def select_topk(r, geo: Geometry):
 
 
 def gather(x, px, idx):
-    """X_sub[i] = row idx[i] of the concatenated pyramid [x | px] (SPEC section 4)."""
+    """X_sub[i] = row idx[i] of the concatenated pyramid [x | px] (Lighthouse summary, 2.C)."""
     full = np.concatenate([np.asarray(x, dtype=np.float64), np.asarray(px, dtype=np.float64)],
                           axis=2)
     return np.take_along_axis(full, idx[..., None].astype(np.int64), axis=2)
 
 
 # ---------------------------------------------------------------------------------------
-# 5. Dense causal attention on the subsequence (SPEC section 5; Lighthouse summary, 2.C).
+# 5. Dense causal attention on the subsequence (Lighthouse summary, 2.C).
 # ---------------------------------------------------------------------------------------
 _ROW_BLOCK = 2048
 
@@ -237,7 +239,7 @@ def attn_fwd(qs, ks, vs):
 
 
 def attn_bwd(qs, ks, vs, os_, lse, dos):
-    """Gradients of attn_fwd w.r.t. Q_sub, K_sub, V_sub (SPEC section 7)."""
+    """Gradients of attn_fwd w.r.t. Q_sub, K_sub, V_sub (Lighthouse summary, 2.B)."""
     B, H, S, d = qs.shape
     sigma = 1.0 / np.sqrt(d)
     dq, dk, dv = np.zeros_like(qs), np.zeros_like(ks), np.zeros_like(vs)
@@ -258,8 +260,8 @@ def attn_bwd(qs, ks, vs, os_, lse, dos):
 
 
 # ---------------------------------------------------------------------------------------
-# 6. Scatter-back: every output row is added to each token of its span (SPEC section 6;
-#    Lighthouse summary, 2.C).
+# 6. Scatter-back: every output row is added to each token of its span (Lighthouse
+#    summary, 2.C).
 # ---------------------------------------------------------------------------------------
 def scatter(idx, os_, geo: Geometry):
     """O[t] = sum of O_sub[i] over subsequence rows whose span covers t."""
@@ -278,7 +280,7 @@ def scatter(idx, os_, geo: Geometry):
 
 
 # ---------------------------------------------------------------------------------------
-# 7. Backward through scatter and gather/pooling (SPEC section 7; Lighthouse summary, 2.B).
+# 7. Backward through scatter and gather/pooling (Lighthouse summary, 2.B).
 # ---------------------------------------------------------------------------------------
 def scatter_bwd(idx, d_o, geo: Geometry):
     """dO_sub[i] = sum of dO over the tokens of span(i)."""
@@ -308,8 +310,7 @@ def gather_bwd(idx, dx_sub, geo: Geometry):
 
 
 # ---------------------------------------------------------------------------------------
-# Storage rounding (SPEC section 9): the layer stores the pyramid, O_sub and dO_sub in its
-# dtype. Round to nearest, ties to even, from the exact value.
+# Storage rounding: the layer stores the pyramid and dO_sub in its dtype (O_sub stays fp32). Round to nearest, ties to even, from the exact value.
 # ---------------------------------------------------------------------------------------
 def round_to(x, store):
     """Exact value -> nearest value of the storage type ("bf16", "f32" or None = keep)."""
@@ -325,7 +326,7 @@ def round_to(x, store):
 
 
 def pool_stored(x, geo: Geometry, store, mean=True):
-    """The stored pooled levels 1..L-1 of x, [B,H,R,d] (SPEC sections 1 and 9).
+    """The stored pooled levels 1..L-1 of x, [B,H,R,d], as the layer rounds them.
 
     Rounding a pooled value to the storage type is a quantisation, so it is decided on the same
     fp32 value that the layer rounds: each level adds its p children's unrounded fp32 sums from
@@ -355,8 +356,8 @@ def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
     """Forward of the layer. g is the score group size (8 for bf16 inputs, 4 for fp32).
 
     idx may be given to force a selection (used for the dense recovery identity). store names
-    the storage type of the stored intermediates, SPEC section 9: the pooled cells (and, in
-    layer_bwd, the span sums dO_sub) are then the fp32 sums of SPEC section 1 rounded to it.
+    the storage type of the stored intermediates: the pooled cells (and, in layer_bwd, the
+    span sums dO_sub) are then the fp32 children sums of pool_stored rounded to it.
     Returns (O [B,H,N,d] float64, saved dict for layer_bwd).
     """
     geo.check()

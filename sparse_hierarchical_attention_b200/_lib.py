@@ -63,6 +63,7 @@ def _load():
         "lh_layer_fwd": ([SP, P, P, P, P, P, P, P], I),
         "lh_layer_bwd": ([SP, P, P, P, P, P, P, P], I),
         "lh_attn_bwd_static": ([SP, P, P, P, P, P, P, P, P, P, P], I),
+        "lh_check_static": ([P, ctypes.POINTER(ctypes.c_uint32)], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -226,3 +227,10 @@ def lh_attn_bwd_static(shape, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, d
     _check(_lib.lh_attn_bwd_static(ctypes.byref(shape.c()), _ptr(q_sub), _ptr(k_sub),
                                    _ptr(v_sub), _ptr(o_sub), _ptr(lse), _ptr(do_sub),
                                    _ptr(dq_sub), _ptr(dk_sub), _ptr(dv_sub), _stream(stream)))
+
+
+def lh_check_static(stream=None):
+    """(status, fault flags) of lh_attn_bwd_static's static status word; clears it."""
+    flags = ctypes.c_uint32(0)
+    rc = _lib.lh_check_static(_stream(stream), ctypes.byref(flags))
+    return rc, flags.value

@@ -6,18 +6,15 @@
 #include "common.cuh"
 
 namespace lh {
-namespace {
 
+namespace {
 thread_local char g_last_error[256] = "";
+}  // namespace
 
 int fail_cuda(cudaError_t e) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s", cudaGetErrorString(e));
   return LH_ERR_CUDA;
 }
-
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Fills g from a shape; returns LH_OK or the reason the GPU path cannot take it.
 int make_geo(const lh_shape* s, Geo& g) {
@@ -66,6 +63,12 @@ int make_geo(const lh_shape* s, Geo& g) {
     return LH_ERR_UNSUPPORTED;
   return LH_OK;
 }
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Workspace layout: [status 256 B | forward region or backward region (they never overlap in
 // time)]. Forward: pq, pk, pv, score, pooling scratch. Backward: do_sub, delta, dq_sub,

@@ -1,6 +1,6 @@
 // Causal attention on the gathered subsequence with fp32 FMA on the CUDA cores.
 //
-// This is the fp32 path (SPEC section 9: no TF32) and the bf16 fallback for shapes the
+// This is the fp32 path (fp32 products and sums throughout, no TF32) and the bf16 fallback for shapes the
 // tensor-core kernels do not take ("Long Context Pre-Training with Lighthouse Attention",
 // technical summary 2.C: plain dense causal attention on the S rows; row j visible to row i
 // iff j <= i).

@@ -1,6 +1,8 @@
 // Causal attention backward on the gathered subsequence with tcgen05 tensor cores ("Long Context
 // Pre-Training with Lighthouse Attention", technical summary 2.B: gradients flow through the
-// attention to Q, K and V; SPEC section 7 gives the formulas).
+// attention to Q, K and V). With D_i = dO_i . O_i and P_ij = exp(s Q_i . K_j - lse_i) for j <= i:
+// dV_j = sum_i P_ij dO_i, dS_ij = P_ij (dO_i . V_j - D_i), dQ_i = s sum_j dS_ij K_j and
+// dK_j = s sum_i dS_ij Q_i, with s = 1/sqrt(d).
 //
 // Two deterministic kernels; neither uses atomics:
 //   dkdv: one CTA per 128-key block steps through the 64-row query blocks that can see the keys:

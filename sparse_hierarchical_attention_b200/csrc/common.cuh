@@ -12,7 +12,9 @@ namespace lh {
 constexpr uint32_t kFaultIndex = 1u;    // a row id outside [0, N+R)
 constexpr uint32_t kFaultTimeout = 2u;  // a bounded wait ran out
 
-// Sizes derived from one layer shape (SPEC section 0), computed on the host.
+// Sizes derived from one layer shape (N_l = N/p^l cells per level, R pooled rows, C chunks of
+// T = p^(L-1) tokens, m = S/C rows and k = m-1 picks per chunk, M candidates per chunk),
+// computed on the host.
 struct Geo {
   int B, H, N, d, p, L, S, dtype;
   int64_t BH, R, C, T, m, k, M;
@@ -81,6 +83,11 @@ __device__ inline void stg16_stream(void* p, uint4 v) {
 __device__ inline void raise_fault(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
+
+// Fills g from a shape: LH_OK, or the lh_status that says why the GPU path cannot take it.
+int make_geo(const lh_shape* s, Geo& g);
+// Records the CUDA error's text for lh_status_string and returns LH_ERR_CUDA.
+int fail_cuda(cudaError_t e);
 
 // ---- internal launchers (one per kernel family); all return cudaError_t of the launch ----
 cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,

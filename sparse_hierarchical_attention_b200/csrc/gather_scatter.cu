@@ -6,7 +6,7 @@
 // spread: one CTA per (b,h, chunk). The chunk's m row ids become a shared-memory map
 //   (level, cell in chunk) -> subsequence row. Each token then adds the rows that cover it,
 //   one per level at most, from the coarsest level down, sharing the partial sums of the
-//   coarse levels among the tokens below them (SPEC sections 6, 7). fp32 accumulation, one
+//   coarse levels among the tokens below them. fp32 accumulation, one
 //   rounding, no atomics.
 #include "common.cuh"
 
@@ -70,7 +70,7 @@ __device__ inline void load_row(const SRC* src, int r, int col, float* x) {
 // One CTA per (b,h, chunk). Covering cells are nested, so each token's sum is formed top-down:
 // a stream of LPR lanes takes a group of p^A tokens (A = 2 when L >= 3), adds the rows of levels
 // L-1..A that cover the whole group once, then the level-1 row once per p tokens, then the
-// token's own level-0 row (SPEC sections 6 and 7: coarsest covering row first).
+// token's own level-0 row (the coarsest covering row first).
 template <typename E, typename SRC, int D>
 __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
   constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, STREAMS = kThreads / LPR;

@@ -14,8 +14,11 @@
 //                  CTA then go through a shared-memory tree up to level A2. If A2 < L-1 the
 //                  level-A2 fp32 sums (and score maxima) go to a small scratch buffer.
 //   coarse kernel - one CTA per chunk finishes levels A2+1..L-1 from that scratch.
-// Sums are fp32 in ascending child order, never re-read from rounded storage (SPEC section 1);
-// norms follow the fixed fp32 order of SPEC section 2 (16-byte groups, halving tree).
+// Sums are fp32 in ascending child order, never re-read from rounded storage; a stored cell is
+// fl32(sum * fl32(1/p^l)) rounded once. Norms take one fixed fp32 order so that the selection is
+// reproducible bit for bit: each 16-byte group of a row is summed in ascending coordinate order
+// (every square rounded on its own, no FMA), the group sums are folded by a halving tree, and
+// the root is a correctly rounded square root.
 #include <algorithm>
 
 #include "common.cuh"
@@ -51,7 +54,7 @@ struct PoolArgs {
   int do_pyr, do_score;
 };
 
-// fp32 l2 norm in the SPEC section 2 order. Each lane of a row sums the squares of its 16-byte
+// fp32 l2 norm in that fixed order. Each lane of a row sums the squares of its 16-byte
 // group in ascending order (products rounded on their own) and leaves that partial in shared
 // memory; one lane then folds the LPR partials of the row with the halving tree (partial i
 // pairs with i + s for s = LPR/2 .. 1, the pairs a lane butterfly would form) and takes the root.
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
         V::unpack(raw[u], x0);
         V::unpack(raw[u + 1], x1);
         if (norm_of) {
-          float a0 = 0.f, a1 = 0.f;  // each row's group in ascending order (SPEC section 2)
+          float a0 = 0.f, a1 = 0.f;  // each row's group in ascending order
 #pragma unroll
           for (int e = 0; e < VEC; ++e) add2(a0, a1, __fmul_rn(x0[e], x0[e]), __fmul_rn(x1[e], x1[e]));
           part[((xi * STREAMS + s) * 16 + row) * PSTR + col] = a0;

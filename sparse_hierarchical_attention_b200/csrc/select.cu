@@ -3,7 +3,7 @@
 // selection is stratified and always keeps the coarsest level).
 //
 // One CTA per (b,h, chunk). The chunk's M candidate scores become 64-bit keys that encode the
-// total ranking order of SPEC section 3: high word = the fp32 score bits (scores are >= +0, so
+// total ranking order (score descending, then level descending, then position ascending): high word = the fp32 score bits (scores are >= +0, so
 // the bit pattern orders like the value), then the level (higher wins), then the position
 // (lower wins). A most-significant-digit radix select (8-bit digits, shared-memory histograms,
 // one warp scanning the 256 bins) finds the k-th largest key; it stops as soon as the bucket

@@ -1,4 +1,4 @@
-"""Helpers shared by the GPU parity tests: conversions and the acceptance rule of SPEC 9."""
+"""Helpers shared by the GPU parity tests: conversions and the acceptance rule."""
 import numpy as np
 import torch
 
@@ -14,7 +14,7 @@ def store_of(dtype):
 
 
 def assert_close(got, want, dtype, what="", mode="scaled"):
-    """The acceptance rule (SPEC section 9).
+    """The acceptance rule.
 
     mode "literal": absolute error, for O on unit-variance workloads.
     mode "scaled": each error divided by max(|oracle element|, RMS of the oracle tensor), for
@@ -57,5 +57,5 @@ def assert_pyramid(got, x, geo, dtype, what="pyramid"):
 
 
 def g_of(dtype):
-    """Score group size of SPEC section 2: 16 bytes of the storage dtype."""
+    """Score group size: the coordinates in 16 bytes of the storage dtype."""
     return 8 if dtype == torch.bfloat16 else 4

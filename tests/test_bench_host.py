@@ -72,7 +72,19 @@ def test_peaks_come_from_the_measured_file():
 def test_measured_traffic_names_real_workloads_and_stages():
     bench = _bench()
     stages = set(bench.stage_work(bench.WORKLOADS["128k"], {"R": _levels_rows(bench.WORKLOADS["128k"])}))
-    for (workload, stage), nbytes in bench.MEASURED_TRAFFIC.items():
+    assert set(bench.STAGE_SOURCES) == stages
+    for (workload, stage), (nbytes, digest, how) in bench.MEASURED_TRAFFIC.items():
         assert workload in bench.WORKLOADS
         assert stage in stages
-        assert isinstance(nbytes, int) and nbytes > 0
+        assert isinstance(nbytes, int) and nbytes > 0 and len(digest) == 16 and how
+
+
+def test_traffic_goes_stale_when_the_kernel_sources_change():
+    bench = _bench()
+    digest = bench.source_digest("attn_bwd")
+    bench.MEASURED_TRAFFIC[("128k", "attn_bwd")] = (123, digest, "test")
+    assert bench.traffic_of("128k", "attn_bwd") == (123, False, "test")
+    bench.MEASURED_TRAFFIC[("128k", "attn_bwd")] = (123, "0" * 16, "test")
+    nbytes, stale, _ = bench.traffic_of("128k", "attn_bwd")
+    assert nbytes is None and stale
+    assert bench.traffic_of("1m", "select")[0] is None

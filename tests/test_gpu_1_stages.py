@@ -62,7 +62,7 @@ def test_pyramid_and_score(B, H, N, d, p, L, S, dt):
     assert bad.size == 0, f"{len(bad)} score mismatches, first {bad[:3]}"
     for x, px in ((q, pq), (k, pk), (v, pv)):
         got = np64(px)[:, :, :R]
-        # the stored cells follow SPEC's fp32 order and one rounding: bit-exact
+        # the stored cells follow the fixed fp32 order and one rounding: bit-exact
         want = O.pool_stored(np64(x), geo, store_of(dtype))
         bad = np.argwhere(got != want)
         assert bad.size == 0, f"{len(bad)} pooled values differ, first {bad[:3]}"

@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 if torch.cuda.is_available():
     import sparse_hierarchical_attention_b200 as lh
     from sparse_hierarchical_attention_b200 import LighthouseAttention, LighthouseLayer, Shape, saved_views
-    from sparse_hierarchical_attention_b200.workloads import WORKLOADS, make_inputs
+    from workloads import WORKLOADS, make_inputs
 
 from gpu_util import assert_close, g_of, np64, store_of
 

@@ -328,7 +328,7 @@ def test_gradients_finite_differences(N, p, L, S):
         np.testing.assert_allclose(gr, num, rtol=1e-6, atol=1e-7)
 
 
-# ---------------------------------------------------------------- storage rounding (SPEC 9)
+# ---------------------------------------------------------------- storage rounding
 def test_bf16_rounding_matches_library_conversion():
     """Round-to-nearest-even to bf16 equals torch's fp32 -> bf16 conversion on fp32 values."""
     x = np.concatenate([rand(100000, scale=10.0), np.float32([1 + 2 ** -8, 1 + 3 * 2 ** -8,

@@ -12,10 +12,8 @@ if torch.cuda.is_available():
     import sparse_hierarchical_attention_b200 as lh
     from sparse_hierarchical_attention_b200 import Shape, _lib
 
-from gpu_util import assert_close, np64
 
-
-def _run(shape, seed, static):
+def _inputs(shape, seed):
     B, H, S, d = shape.B, shape.H, shape.S, shape.d
     g = torch.Generator(device="cuda").manual_seed(seed)
     qs, ks, vs, dos = (torch.randn(B, H, S, d, generator=g, device="cuda").to(shape.dtype)
@@ -24,24 +22,45 @@ def _run(shape, seed, static):
     lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
     ws = torch.zeros(lh.lh_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
     lh.lh_attn_fwd(shape, qs, ks, vs, os_, lse, ws)
-    grads = [torch.empty(B, H, S, d, dtype=torch.float32, device="cuda") for _ in range(3)]
-    if static:
-        _lib.lh_attn_bwd_static(shape, qs, ks, vs, os_, lse, dos, *grads)
-    else:
-        lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, *grads, ws)
+    return qs, ks, vs, os_, lse, dos, ws
+
+
+def _grads(shape):
+    return [torch.empty(shape.B, shape.H, shape.S, shape.d, dtype=torch.float32, device="cuda")
+            for _ in range(3)]
+
+
+def _both(shape, seed):
+    """(static grads, workspace grads) of the same inputs, each from its own output buffers."""
+    qs, ks, vs, os_, lse, dos, ws = _inputs(shape, seed)
+    got, want = _grads(shape), _grads(shape)
+    _lib.lh_attn_bwd_static(shape, qs, ks, vs, os_, lse, dos, *got)
+    lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, *want, ws)
     torch.cuda.synchronize()
-    return grads
+    assert lh.lh_check(ws) == (0, 0)
+    return got, want
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_static_scratch_matches_workspace_version_twice(dtype):
-    """Two calls in a row (the second on other inputs and sizes) match lh_attn_bwd."""
+    """Two calls in a row (the second on other inputs and sizes) give lh_attn_bwd's gradients
+    bit for bit: the same kernels run on the same inputs; only D's address differs."""
     for seed, (H, S, d) in enumerate([(4, 1024, 128), (2, 333, 64)]):
         shape = Shape(1, H, S, d, 4, 1, S, dtype)
-        got = _run(shape, seed, static=True)
-        want = _run(shape, seed, static=False)
+        got, want = _both(shape, seed)
         for a, b, n in zip(got, want, ("dq", "dk", "dv")):
-            assert_close(np64(a), np64(b), dtype, f"static {n}", mode="scaled")
+            assert torch.equal(a, b), f"static {n} differs (call {seed})"
+    assert _lib.lh_check_static() == (0, 0)  # no fault latched in the static status word
+
+
+def test_static_scratch_at_its_row_limit():
+    """B*H*S equal to LH_STATIC_SCRATCH_ROWS is accepted and fills D to its last row."""
+    shape = Shape(1, 256, 4096, 64, 4, 1, 4096)
+    assert shape.B * shape.H * shape.S == _lib.LH_STATIC_SCRATCH_ROWS
+    got, want = _both(shape, 7)
+    for a, b, n in zip(got, want, ("dq", "dk", "dv")):
+        assert torch.equal(a, b), f"static {n} differs at the row limit"
+    assert _lib.lh_check_static() == (0, 0)
 
 
 def test_static_scratch_rejects_oversized_shapes():
