@@ -82,9 +82,16 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", default="1m",
+                    help="comma-separated workloads also device-timed in the same run ('' for none)")
     ap.add_argument("--no-sdpa", action="store_true",
                     help="skip the dense causal SDPA context timing (run when N <= 128K)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    args.also = [x for x in args.also.split(",") if x]
+    for x in args.also:
+        if x not in WORKLOADS:
+            ap.error(f"--also: unknown workload {x}")
+    return args
 
 
 # ----------------------------------------------------------------------------- process group
@@ -129,14 +136,72 @@ def throughput(total_ms_local, steps, tokens_per_rank, world):
 
 # ----------------------------------------------------------------------------- clocks
 class Clocks:
-    """nvidia-smi samples during the timed region."""
+    """SM clock, power and clock-event reasons sampled during the timed region.
+
+    NVML is polled every 5 ms from a background thread (read-only queries), so that even a
+    timed region of a few tens of milliseconds yields samples. The NVML device is found by the
+    CUDA device's PCI bus id. Without NVML, nvidia-smi samples every 200 ms instead."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index, period_s=0.005):
+        import threading
+        self.samples, self.max_mhz, self.err = [], None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            p = torch.cuda.get_device_properties(device_index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.bits = {name: getattr(nv, attr) for name, attr in self.REASONS}
+        except Exception as e:  # noqa: BLE001  (no NVML: the nvidia-smi path below)
+            self.nv, self.err = None, repr(e)
+        if self.nv is None:
+            self.smi = _SmiClocks(device_index)
+            return
+        self.thread = threading.Thread(target=self._poll, args=(period_s,), daemon=True)
+        self.thread.start()
+
+    def _poll(self, period_s):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                watts = nv.nvmlDeviceGetPowerUsage(self.h) / 1e3
+                self.samples.append((mhz, mask, watts))
+            except Exception as e:  # noqa: BLE001
+                self.err = repr(e)
+            self._stop.wait(period_s)
+
+    def stop(self):
+        if self.nv is None:
+            return self.smi.stop()
+        self._stop.set()
+        self.thread.join(timeout=5)
+        sm = [m for m, _, _ in self.samples]
+        reasons = sorted({name for _, mask, _ in self.samples for name, bit in self.bits.items()
+                          if mask & bit})
+        load = [x for x in sm if x > 0.5 * self.max_mhz] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "nvml, 5 ms",
+                "power_w_max": round(max((w for _, _, w in self.samples), default=0.0), 1)}
+
+
+class _SmiClocks:
+    """nvidia-smi samples (200 ms) during the timed region, when NVML is not importable."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
-        self.dev = device_index
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
@@ -167,7 +232,7 @@ class Clocks:
                     reasons.add(nm)
         load = [s for s in sm if mx and s > 0.5 * mx] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 def peaks():
@@ -198,17 +263,14 @@ def stage_work(w, geo):
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, world, rank, local):
-    import sparse_hierarchical_attention_b200 as lh
+def make_stages(lh, w, dev, seed):
+    """Device buffers of one workload and the eight stage calls of one step, in order."""
     from sparse_hierarchical_attention_b200 import Shape
-
-    w = WORKLOADS[args.workload]
-    dev = torch.device("cuda", local)
     shape = Shape(w.B, w.H, w.N, w.d, w.p, w.L, w.S, w.dtype)
     geo = lh.lh_validate(shape)
     B, H, N, d, S, dt = w.B, w.H, w.N, w.d, w.S, w.dtype
     R = geo["R"]
-    q, k, v, d_o = make_inputs(w, dev, seed=1000 * rank)
+    q, k, v, d_o = make_inputs(w, dev, seed=seed)
     E = lambda *s, t=dt: torch.empty(*s, dtype=t, device=dev)  # noqa: E731
     pq, pk, pv = E(B, H, max(R, 1), d), E(B, H, max(R, 1), d), E(B, H, max(R, 1), d)
     score = E(B, H, N + R, t=torch.float32)
@@ -221,7 +283,6 @@ def run_ours(args, world, rank, local):
     dqs, dks, dvs = (E(B, H, S, d, t=torch.float32) for _ in range(3))
     dq, dk, dv = (E(B, H, N, d) for _ in range(3))
     ws = torch.zeros(lh.lh_workspace_bytes(shape), dtype=torch.uint8, device=dev)
-
     stages = [
         ("pyramid_score", lambda: lh.lh_build_pyramid(shape, q, k, v, pq, pk, pv, score, ws)),
         ("select", lambda: lh.lh_select_topk(shape, score, idx)),
@@ -232,7 +293,12 @@ def run_ours(args, world, rank, local):
         ("attn_bwd", lambda: lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, dqs, dks, dvs, ws)),
         ("gather_bwd", lambda: lh.lh_gather_bwd(shape, idx, dqs, dks, dvs, dq, dk, dv)),
     ]
-    K, W = args.steps, args.warmup
+    return shape, geo, (q, k, v, d_o), ws, stages
+
+
+def time_stages(lh, stages, ws, K, W, world, local):
+    """W warm-up steps, then exactly K timed steps between a barrier and a synchronize on both
+    sides. Returns (per-stage mean ms, per-step ms, device ms of the K steps, clocks, wall s)."""
     for _ in range(W):
         for _, fn in stages:
             fn()
@@ -240,13 +306,11 @@ def run_ours(args, world, rank, local):
     rc, flags = lh.lh_check(ws)
     if rc:
         raise RuntimeError(f"device fault flags {flags:#x} during warm-up")
-
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     clocks = Clocks(local)
-    time.sleep(0.3)
     t_wall = time.perf_counter()
     for s in range(K):
         ev[s][0].record(stream)
@@ -257,12 +321,18 @@ def run_ours(args, world, rank, local):
     wall = time.perf_counter() - t_wall
     barrier(world)
     clk = clocks.stop()
+    rc, flags = lh.lh_check(ws)
+    if rc:
+        raise RuntimeError(f"device fault flags {flags:#x} in the timed steps")
     step_ms = [ev[s][0].elapsed_time(ev[s][-1]) for s in range(K)]
-    total_ms = sum(step_ms)
     per_stage = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)) / K
                  for i, (name, _) in enumerate(stages)}
-    value, ms_step = throughput(total_ms, K, B * N, world)
+    return per_stage, step_ms, sum(step_ms), clk, wall
 
+
+def report_stages(w, geo, per_stage):
+    """Each stage's achieved rate and fraction of the measured peak, and the dominant stage's
+    roofline object."""
     pk_, src = peaks()
     work = stage_work(w, geo)
     stage_report = {}
@@ -279,30 +349,44 @@ def run_ours(args, world, rank, local):
     dom = max(per_stage, key=per_stage.get)
     kind, amount = work[dom]
     rf = stage_report[dom]
+    traffic, stale, note = traffic_of(w.name, dom)
     roofline = {"kernel": dom, "bound": "hbm" if kind == "hbm" else "tensor",
                 "achieved": rf["achieved"], "peak": pk_["hbm_gbs"] if kind == "hbm" else pk_["bf16_tflops"],
-                "unit": rf["unit"], "frac": rf["frac"],
-                "traffic": traffic_of(args.workload, dom)[0],
-                "traffic_stale": traffic_of(args.workload, dom)[1],
-                "traffic_note": traffic_of(args.workload, dom)[2],
+                "unit": rf["unit"], "frac": rf["frac"], "traffic": traffic, "traffic_stale": stale,
+                "traffic_note": note,
                 "traffic_scope": "bytes of one stage call (all its launches), like achieved",
                 "peak_source": f"{src} ({'hbm_gbs' if kind == 'hbm' else 'bf16_tflops'})",
                 "units_per_launch": amount}
+    return stage_report, roofline
+
+
+def run_ours(args, world, rank, local):
+    import sparse_hierarchical_attention_b200 as lh
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    K, W = args.steps, args.warmup
+    shape, geo, (q, k, v, d_o), ws, stages = make_stages(lh, w, dev, 1000 * rank)
+    per_stage, step_ms, total_ms, clk, wall = time_stages(lh, stages, ws, K, W, world, local)
+    value, ms_step = throughput(total_ms, K, w.B * w.N, world)
+    stage_report, roofline = report_stages(w, geo, per_stage)
     nf, nb = lh.lh_launches(shape)
+    del stages, ws
+    torch.cuda.empty_cache()
 
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(lh, shape, w, dev, q, k, v, d_o, K, W, world)
     context = None
-    if world == 1 and not args.no_sdpa and N <= 131072 and dt == torch.bfloat16:
+    if world == 1 and not args.no_sdpa and w.N <= 131072 and w.dtype == torch.bfloat16:
         context = dense_sdpa_context(q, k, v, d_o, ms_step)
-    for t in (pq, pk, pv, score, qs, ks, vs, os_, dos, dqs, dks, dvs, dq, dk, dv, o):
-        del t
+    del q, k, v, d_o
+    torch.cuda.empty_cache()
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(ms_step, 4),
         "ms_per_step_median_rank0": round(statistics.median(step_ms), 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic (seeded N(0,1) Q/K/V with the workload's row-scale recipe; dO N(0,1))",
         "config": workload_config(w, world),
         "stages": stage_report, "roofline": roofline, "gpu_launches": (nf + nb) * K,
@@ -312,6 +396,25 @@ def run_ours(args, world, rank, local):
         out["e2e"] = e2e
     if context:
         out["context"] = context
+    # further workloads in the same run, device-timed the same way (no e2e, no context)
+    extra = {}
+    for name in args.also:
+        if name == w.name:
+            continue
+        wx = WORKLOADS[name]
+        shape_x, geo_x, ins, ws_x, stages_x = make_stages(lh, wx, dev, 1000 * rank)
+        per_x, steps_x, total_x, clk_x, _ = time_stages(lh, stages_x, ws_x, K, W, world, local)
+        value_x, ms_x = throughput(total_x, K, wx.B * wx.N, world)
+        rep_x, roof_x = report_stages(wx, geo_x, per_x)
+        nfx, nbx = lh.lh_launches(shape_x)
+        extra[name] = {"value": round(value_x, 1), "unit": "tokens/s", "ms_per_step": round(ms_x, 4),
+                       "steps": K, "warmup": W, "config": workload_config(wx, world),
+                       "stages": rep_x, "roofline": roof_x, "gpu_launches": (nfx + nbx) * K,
+                       "clocks": clk_x}
+        del ins, ws_x, stages_x
+        torch.cuda.empty_cache()
+    if extra:
+        out["also"] = extra
     return out
 
 

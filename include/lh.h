@@ -56,12 +56,21 @@ typedef enum {
 
 typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
 
+/* lh_shape.flags */
+#define LH_DETERMINISTIC 1 /* attention backward without atomics: bit-identical results run to run */
+
 /* One layer call. Names follow the pages: N tokens, H heads, d = d_head, pooling factor p,
  * L levels, S = subsequence length (the top-K budget plus the kept coarsest cells).
- * The softmax scale is fixed to 1/sqrt(d). */
+ * The softmax scale is fixed to 1/sqrt(d).
+ * flags: 0 or LH_DETERMINISTIC. At d = 128 the default attention backward computes dK, dV and
+ * dQ in one pass over the key blocks and adds the per-block dQ terms into dq_sub with fp32
+ * atomic adds, whose order varies from run to run (so do the last bits of dQ). With
+ * LH_DETERMINISTIC it runs a second pass for dQ instead (no atomics; slower). Everything else
+ * is deterministic either way. */
 typedef struct {
   int B, H, N, d, p, L, S;
   int dtype; /* lh_dtype */
+  int flags;
 } lh_shape;
 
 /* Sizes derived from a shape (the pages' notation: p, L, N per level, budget S). */
@@ -95,8 +104,17 @@ size_t lh_saved_bytes(const lh_shape* shape);
 int lh_workspace_init(void* ws, void* stream);
 /* Synchronises `stream`, reads and clears the status word of `ws`.
  * Returns LH_OK or LH_ERR_DEVICE (then *flags, if non-NULL, holds the fault bits:
- * 1 = row id out of range, 2 = bounded wait ran out). */
+ * 1 = row id out of range, 2 = bounded wait ran out, 4 = after that, a wait for the kernel's own
+ * copies or MMAs in flight ran out too). After flag 2 the affected outputs are unspecified;
+ * the device context stays usable. */
 int lh_check(void* ws, void* stream, uint32_t* flags);
+
+/* Sets the bound of every wait inside the tensor-core kernels (a pipeline stage that never
+ * arrives, for instance): after `ns` nanoseconds the kernel sets status flag 2, drains its own
+ * operations in flight and returns. 0 restores the default of 2 s. Applies to launches made
+ * after the call, from any thread. Returns the previous bound. Not part of the method: a
+ * failure-detection control. */
+uint64_t lh_set_wait_limit_ns(uint64_t ns);
 
 /* Step 1+2 (pyramid, section 2.A; scores, section 2.B). Reads q, k, v [B,H,N,d]; writes the
  * pooled levels pq, pk, pv [B,H,R,d]. If `score` is non-NULL it also writes the rank score

@@ -26,8 +26,11 @@ class LighthouseError(RuntimeError):
     pass
 
 
+LH_DETERMINISTIC = 1
+
+
 class lh_shape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "N", "d", "p", "L", "S", "dtype")]
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "N", "d", "p", "L", "S", "dtype", "flags")]
 
 
 class lh_sizes(ctypes.Structure):
@@ -51,6 +54,7 @@ def _load():
         "lh_launches": ([SP, ctypes.POINTER(I), ctypes.POINTER(I)], I),
         "lh_workspace_init": ([P, P], I),
         "lh_check": ([P, P, ctypes.POINTER(ctypes.c_uint32)], I),
+        "lh_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_uint64),
         "lh_build_pyramid": ([SP, P, P, P, P, P, P, P, P, P], I),
         "lh_score": ([SP, P, P, P, P, P], I),
         "lh_select_topk": ([SP, P, P, P], I),
@@ -82,7 +86,10 @@ def header_functions():
 
 @dataclass(frozen=True)
 class Shape:
-    """One layer call: N tokens, H heads, d = d_head, pooling p, L levels, S rows kept."""
+    """One layer call: N tokens, H heads, d = d_head, pooling p, L levels, S rows kept.
+
+    deterministic: run the attention backward without atomics (LH_DETERMINISTIC), so that
+    dQ is bit-identical from run to run; slower at d = 128."""
 
     B: int
     H: int
@@ -92,9 +99,11 @@ class Shape:
     L: int
     S: int
     dtype: torch.dtype = torch.bfloat16
+    deterministic: bool = False
 
     def c(self):
-        return lh_shape(self.B, self.H, self.N, self.d, self.p, self.L, self.S, _DTYPES[self.dtype])
+        return lh_shape(self.B, self.H, self.N, self.d, self.p, self.L, self.S, _DTYPES[self.dtype],
+                        LH_DETERMINISTIC if self.deterministic else 0)
 
 
 def _ptr(t):
@@ -149,6 +158,12 @@ def lh_launches(shape: Shape):
     f, b = ctypes.c_int(0), ctypes.c_int(0)
     _check(_lib.lh_launches(ctypes.byref(shape.c()), ctypes.byref(f), ctypes.byref(b)))
     return f.value, b.value
+
+
+def lh_set_wait_limit_ns(ns: int) -> int:
+    """Bound of every wait inside the tensor-core kernels (0 = the default 2 s); returns the
+    previous bound."""
+    return int(_lib.lh_set_wait_limit_ns(ctypes.c_uint64(ns)))
 
 
 def lh_workspace_init(ws, stream=None):

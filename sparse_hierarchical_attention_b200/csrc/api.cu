@@ -1,5 +1,6 @@
 // C ABI of the Lighthouse selection layer: validation, workspace layout, dispatch and the
 // layer-level orchestration of the five steps (declared in include/lh.h).
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 
@@ -9,6 +10,8 @@ namespace lh {
 
 namespace {
 thread_local char g_last_error[256] = "";
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
 }  // namespace
 
 int fail_cuda(cudaError_t e) {
@@ -22,6 +25,9 @@ int make_geo(const lh_shape* s, Geo& g) {
   std::memset(&g, 0, sizeof(g));
   g.B = s->B; g.H = s->H; g.N = s->N; g.d = s->d; g.p = s->p; g.L = s->L; g.S = s->S;
   g.dtype = s->dtype;
+  g.flags = s->flags;
+  g.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  if (s->flags & ~LH_DETERMINISTIC) return LH_ERR_INVALID_ARG;
   if (g.B < 1 || g.H < 1 || g.N < 1 || g.d < 1 || g.p < 2 || g.L < 1 || g.S < 1)
     return LH_ERR_INVALID_ARG;
   if (g.dtype != LH_F32 && g.dtype != LH_BF16) return LH_ERR_INVALID_ARG;
@@ -223,6 +229,10 @@ int lh_saved_offsets(const lh_shape* shape, size_t offsets[6]) {
   offsets[0] = s.idx; offsets[1] = s.qs; offsets[2] = s.ks;
   offsets[3] = s.vs; offsets[4] = s.os; offsets[5] = s.lse;
   return LH_OK;
+}
+
+uint64_t lh_set_wait_limit_ns(uint64_t ns) {
+  return g_wait_ns.exchange(ns ? ns : kDefaultWaitNs);
 }
 
 int lh_workspace_init(void* ws, void* stream) {

@@ -385,7 +385,7 @@ cudaError_t bwd(const Geo& g, const void* qs, const void* ks, const void* vs, co
 }  // namespace
 
 int attn_fwd_launches(const Geo&) { return 1; }
-int attn_bwd_launches(const Geo&) { return 3; }  // delta + two passes, on either path
+int attn_bwd_launches(const Geo& g) { return attn_bwd_fused(g) ? 2 : 3; }  // delta + one or two passes
 
 cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
                                  float* os, float* lse, cudaStream_t st) {

@@ -57,14 +57,14 @@ struct Layout {
 };
 
 // bars: 0 Q | 1-3 K loaded | 4-6 V loaded | 7-9 K free | 10-12 V free | 13-14 S ready
-//       | 15-16 S buffer read | 17 P written | 18 PV done
-constexpr int kBars = 19;
+//       | 15-16 S buffer read | 17 P written | 18 PV done | 19-20 drain of the two MMA issuers
+constexpr int kBars = 21;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, float* __restrict__ O, float* __restrict__ lse,
-            int S, int BH, float scale_log2, uint32_t* status) {
+            int S, int BH, float scale_log2, uint32_t* status, uint64_t wait_ns) {
   using Ly = Layout<D>;
   constexpr int KB = Ly::KB;
   constexpr int kStV = v_stages<D>();
@@ -122,12 +122,20 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       };
       mbar_expect_tx(bar_q, KB * TILE);
       for (int c = 0; c < KB; ++c) tma_load_2d(sm + Ly::Q + c * TILE, &tq, c * 64, grow0 + qb * BM, bar_q);
+      int nk = 0, nv = 0;  // loads issued into each ring
       for (int j = 0; j < nkb; ++j) {  // block j reuses the K stage of block j - 3, the V stage of j - kStV
-        if (j >= kStages && !mbar_wait(bar_kfree + j % kStages, ((j - kStages) / kStages) & 1, abort_flag, status)) break;
+        if (j >= kStages && !mbar_wait(bar_kfree + j % kStages, ((j - kStages) / kStages) & 1, abort_flag, status, wait_ns)) break;
         load_k(j);
-        if (j >= kStV && !mbar_wait(bar_vfree + j % kStV, ((j - kStV) / kStV) & 1, abort_flag, status)) break;
+        ++nk;
+        if (j >= kStV && !mbar_wait(bar_vfree + j % kStV, ((j - kStV) / kStV) & 1, abort_flag, status, wait_ns)) break;
         load_v(j);
+        ++nv;
       }
+      // every load issued has landed before this thread leaves (on the normal path they were
+      // all consumed already, so these return at once)
+      mbar_drain(bar_q, 0, status);
+      drain_ring(bar_k, kStages, nk, status);
+      drain_ring(bar_v, kStV, nv, status);
     }
   } else if (warp == kSoftmax / 32 + 1 || warp == kSoftmax / 32 + 2) {
     // ------------------------------------------------------------------ MMA warps
@@ -161,22 +169,24 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         mma_commit(bar_vfree + j % kStV);
       };
       if (s_issuer) {
-        bool ok = mbar_wait(bar_q, 0, abort_flag, status);
+        bool ok = mbar_wait(bar_q, 0, abort_flag, status, wait_ns);
         for (int n = 0; n < nkb && ok; ++n) {  // S_n into buffer n & 1 once the softmax has read S_{n-2}
-          ok = mbar_wait(bar_k + n % kStages, (n / kStages) & 1, abort_flag, status);
-          if (ok && n >= 2) ok = mbar_wait(bar_sfree + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status);
+          ok = mbar_wait(bar_k + n % kStages, (n / kStages) & 1, abort_flag, status, wait_ns);
+          if (ok && n >= 2) ok = mbar_wait(bar_sfree + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status, wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
+        mma_drain(bar + 19, status);
       } else {
         for (int j = 0; j < nkb; ++j) {
-          const bool ok = mbar_wait(bar_p, j & 1, abort_flag, status) &&
-                          mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status);
+          const bool ok = mbar_wait(bar_p, j & 1, abort_flag, status, wait_ns) &&
+                          mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status, wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_pv(j);
         }
+        mma_drain(bar + 20, status);
       }
     }
   } else {
@@ -191,7 +201,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
     // all lanes of a warp wait together, so that the warp stays converged for tcgen05.ld/st
     auto wait_all = [&](uint64_t* b, uint32_t parity) {
-      bool ok = mbar_wait(b, parity, abort_flag, status);
+      bool ok = mbar_wait(b, parity, abort_flag, status, wait_ns);
       return __all_sync(0xffffffffu, ok);
     };
     float m_used = -INFINITY, l = 0.f;
@@ -311,13 +321,10 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       if (half == 0) lse[grow0 + qb * BM + row] = (m_used + log2f(lt)) * 0.69314718055994531f;
     }
   }
+  // every role has drained its own loads and MMAs, so nothing still writes shared or tensor
+  // memory once all threads are here
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag) {  // let operations already in flight finish before the memory is released
-    const uint64_t t0 = globaltimer();
-    while (globaltimer() - t0 < 1000000ull) {
-    }
-  }
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
@@ -380,13 +387,15 @@ cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, con
     const int smem = Layout<128>::BYTES + 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status);
+      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status,
+                                                      g.wait_ns);
   } else {
     // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
     const int smem = Layout<64>::BYTES + 1024 > 120 * 1024 ? Layout<64>::BYTES + 1024 : 120 * 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status);
+      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status,
+                                                     g.wait_ns);
   }
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -11,12 +11,15 @@ namespace lh {
 
 constexpr uint32_t kFaultIndex = 1u;    // a row id outside [0, N+R)
 constexpr uint32_t kFaultTimeout = 2u;  // a bounded wait ran out
+constexpr uint32_t kFaultDrain = 4u;    // an abort-path wait for the CTA's own operations ran out
 
 // Sizes derived from one layer shape (N_l = N/p^l cells per level, R pooled rows, C chunks of
 // T = p^(L-1) tokens, m = S/C rows and k = m-1 picks per chunk, M candidates per chunk),
 // computed on the host.
 struct Geo {
   int B, H, N, d, p, L, S, dtype;
+  int flags;          // lh_shape.flags (LH_DETERMINISTIC)
+  uint64_t wait_ns;   // bound of every wait inside a kernel (lh_set_wait_limit_ns)
   int64_t BH, R, C, T, m, k, M;
   int64_t nlev[16];  // N_l = N / p^l
   int64_t off[16];   // row id of the first cell of level l (off[0] = 0, off[1] = N, ...)
@@ -106,6 +109,8 @@ cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, v
 size_t span_sum_tmp_bytes(const Geo& g);
 int span_sum_launches(const Geo& g);  // 1 or 2, as pool_launches
 bool attn_tc_eligible(const Geo& g);  // bf16, d in {64,128}, S % 128 == 0
+// The one-pass dK/dV/dQ backward runs (d = 128 on the tensor-core path, LH_DETERMINISTIC unset).
+bool attn_bwd_fused(const Geo& g);
 cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
                                float* os, float* lse, uint32_t* status, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,

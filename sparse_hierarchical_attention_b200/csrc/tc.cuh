@@ -8,9 +8,13 @@
 //  - instruction descriptor (32 bit) for kind::f16: D format (1 = f32) in [4,6), A format
 //    (1 = bf16) in [7,10), B format in [10,13), A major (0 = K, 1 = MN) bit 15, B major bit 16,
 //    N >> 3 in [17,23), M >> 4 in [24,29).
-// Every wait is bounded: after kWaitNs of wall time it records kFaultTimeout in the status word,
-// raises a CTA-wide abort flag and returns false, so that a kernel can drain and exit instead of
-// hanging the GPU.
+// Every wait is bounded: after a limit of wall time (a kernel argument, 2 s unless the caller
+// set another through lh_set_wait_limit_ns) it records kFaultTimeout in the status word, raises
+// a CTA-wide abort flag and returns false. Each role then drains: a thread that issued TMA loads
+// waits for the last phase it armed on each of its barriers, and a thread that issued MMAs
+// commits them to a barrier of its own and waits for it, both under a fixed limit (kDrainNs).
+// So no copy into shared memory and no MMA on tensor memory is still in flight when the CTA
+// frees its tensor memory and exits.
 #pragma once
 
 #include <cuda.h>
@@ -21,7 +25,7 @@
 namespace lh {
 namespace tc {
 
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kDrainNs = 2000000000ull;  // bound of the waits on the abort path (2 s)
 
 // Attention grids: blockIdx.x = head within a group of kHeadGroup heads, blockIdx.y = row block
 // (heaviest first), blockIdx.z = head group. CTAs are dispatched x fastest, so the CTAs in flight
@@ -64,21 +68,46 @@ __device__ inline bool mbar_try(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete. Returns false (and sets the abort flag
-// and the status bit) if that takes longer than kWaitNs, or if another thread aborted.
+// and the status bit) if that takes longer than limit_ns, or if another thread aborted. Limits
+// under a millisecond are checked on every poll, longer ones every 256 polls.
 __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                 uint32_t* status) {
+                                 uint32_t* status, uint64_t limit_ns) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint32_t every = limit_ns < 1000000ull ? 0u : 255u;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & every) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         raise_fault(status, kFaultTimeout);
         return false;
       }
     }
+  }
+}
+
+// Abort path: waits, at most kDrainNs, for the phase with the given parity of a barrier whose
+// completion this thread armed (its own TMA loads, or its own MMA commit). Running out of that
+// bound sets kFaultDrain: the hardware did not finish an operation it had accepted.
+__device__ inline void mbar_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > kDrainNs) {
+      raise_fault(status, kFaultDrain);
+      return;
+    }
+  }
+}
+
+// A TMA thread's loads into a ring of `stages` barriers: after `issued` loads (load i into
+// stage i % stages, one phase per load) the last phase armed on stage s has parity
+// (n_s - 1) & 1, with n_s the loads stage s received. Waits for each of them.
+__device__ inline void drain_ring(uint64_t* bars, int stages, int issued, uint32_t* status) {
+  for (int s = 0; s < stages && s < issued; ++s) {
+    const int n = (issued - s + stages - 1) / stages;
+    mbar_drain(bars + s, (uint32_t)(n - 1) & 1u, status);
   }
 }
 
@@ -233,6 +262,13 @@ __device__ inline void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+// End of an MMA-issuing role (normal or aborted): commits every MMA this thread issued to its
+// own barrier `bar` (arrival count 1, used for nothing else) and waits for it, so that none is
+// still running when the CTA frees tensor memory.
+__device__ inline void mma_drain(uint64_t* bar, uint32_t* status) {
+  mma_commit(bar);
+  mbar_drain(bar, 0, status);
 }
 
 // 2^x with the hardware approximation (flush-to-zero; relative error ~2^-22), for softmax

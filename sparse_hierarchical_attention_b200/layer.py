@@ -75,16 +75,18 @@ class _Fn(torch.autograd.Function):
 
 
 class LighthouseAttention(torch.nn.Module):
-    """Drop-in replacement of causal SDPA on [B, H, N, d] tensors during pre-training."""
+    """Drop-in replacement of causal SDPA on [B, H, N, d] tensors during pre-training.
 
-    def __init__(self, p: int, L: int, S: int):
+    deterministic=True makes the backward bit-reproducible (no atomics; slower at d = 128)."""
+
+    def __init__(self, p: int, L: int, S: int, deterministic: bool = False):
         super().__init__()
-        self.p, self.L, self.S = p, L, S
+        self.p, self.L, self.S, self.deterministic = p, L, S, deterministic
         self._layers = {}
 
     def forward(self, q, k, v):
         B, H, N, d = q.shape
-        shape = Shape(B, H, N, d, self.p, self.L, self.S, q.dtype)
+        shape = Shape(B, H, N, d, self.p, self.L, self.S, q.dtype, self.deterministic)
         key = (shape, q.device)
         if key not in self._layers:
             self._layers[key] = LighthouseLayer(shape, q.device)

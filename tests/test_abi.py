@@ -92,3 +92,17 @@ def test_binding_refuses_host_tensors():
     x = torch.zeros(1, 1, 256 + 80, dtype=torch.float32)
     with pytest.raises(lh.LighthouseError):
         lh.lh_select_topk(s, x, torch.zeros(1, 1, 64, dtype=torch.int32))
+
+
+def test_wait_limit_setter_returns_the_previous_bound_and_restores_the_default():
+    prev = lh.lh_set_wait_limit_ns(12345)
+    assert lh.lh_set_wait_limit_ns(0) == 12345
+    assert lh.lh_set_wait_limit_ns(prev) == 2_000_000_000
+
+
+def test_flags_other_than_deterministic_are_rejected():
+    s = Shape(1, 2, 4096, 128, 4, 3, 256)
+    c = s.c()
+    c.flags = 2
+    assert _lib._lib.lh_validate(ctypes.byref(c), None) == 1  # LH_ERR_INVALID_ARG
+    assert lh.lh_validate(Shape(1, 2, 4096, 128, 4, 3, 256, deterministic=True))["C"] == 256

@@ -97,14 +97,17 @@ def rand_sub(B, H, S, d, dtype, seed):
     return [torch.randn(B, H, S, d, generator=g, device="cuda").to(dtype) for _ in range(4)]
 
 
+@pytest.mark.parametrize("det", [False, True])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 @pytest.mark.parametrize("B,H,S,d", [(1, 2, 64, 64), (2, 2, 333, 128), (1, 3, 1000, 64),
                                      (1, 1, 1, 128), (1, 2, 4096, 128), (1, 1, 128, 128),
-                                     (2, 3, 256, 64), (1, 2, 1024, 128), (1, 1, 2048, 64)])
-def test_attention_fwd_bwd(B, H, S, d, dt):
+                                     (2, 3, 256, 64), (1, 2, 1024, 128), (1, 1, 2048, 64),
+                                     (3, 5, 384, 128)])
+def test_attention_fwd_bwd(B, H, S, d, dt, det):
+    """Both backward modes (one pass with atomic dQ adds; deterministic two passes)."""
     dtype = DT[dt]
     N = S  # an L = 1 shape carries (S, d) to the attention entry points
-    shape = Shape(B, H, N, d, 4, 1, S, dtype)
+    shape = Shape(B, H, N, d, 4, 1, S, dtype, det)
     qs, ks, vs, dos = rand_sub(B, H, S, d, dtype, seed=S)
     os_ = torch.empty(B, H, S, d, dtype=torch.float32, device="cuda")
     lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
@@ -187,3 +190,28 @@ def test_out_of_range_ids_are_flagged_not_faulted():
     assert rc != 0 and flags & 1
     assert (subs[0][0, 0, 5] == 0).all() and (subs[0][0, 0, 9] == 0).all()
     assert lh.lh_check(ws) == (0, 0)  # cleared by the read
+
+
+@pytest.mark.parametrize("B,H,S", [(1, 2, 4096), (1, 9, 1024), (2, 3, 384)])
+def test_fused_backward_matches_the_deterministic_one(B, H, S):
+    """The one-pass backward computes dK and dV exactly as the two-pass one (the same MMAs
+    accumulate in the same order), so they agree bit for bit. Its dQ adds fp32 partial sums per
+    128-key block in a varying order: it agrees to fp32 rounding of those sums."""
+    d, dtype = 128, torch.bfloat16
+    qs, ks, vs, dos = rand_sub(B, H, S, d, dtype, seed=S + 1)
+    out = {}
+    for det in (False, True):
+        shape = Shape(B, H, S, d, 4, 1, S, dtype, det)
+        ws = ws_for(shape)
+        os_ = torch.empty(B, H, S, d, dtype=torch.float32, device="cuda")
+        lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
+        lh.lh_attn_fwd(shape, qs, ks, vs, os_, lse, ws)
+        g = [torch.empty(B, H, S, d, dtype=torch.float32, device="cuda") for _ in range(3)]
+        lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, *g, ws)
+        assert lh.lh_check(ws) == (0, 0)
+        out[det] = g
+    (fq, fk, fv), (dq, dk, dv) = out[False], out[True]
+    assert torch.equal(fk, dk) and torch.equal(fv, dv)
+    rms = dq.pow(2).mean().sqrt()
+    err = (fq - dq).abs() / torch.maximum(dq.abs(), rms)
+    assert err.max().item() <= 1e-5, err.max().item()

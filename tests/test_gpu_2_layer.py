@@ -118,22 +118,30 @@ def test_dense_recovery_matches_torch_sdpa(dtype):
         assert_close(np64(got), np64(t.grad), dtype, n)
 
 
-def test_deterministic_bits():
+@pytest.mark.parametrize("det", [True, False])
+def test_deterministic_bits(det):
+    """With LH_DETERMINISTIC every output is bit-identical run to run. Without it only dQ may
+    differ, by the rounding of its atomic fp32 sums: at most one bf16 unit in the last place."""
     w = WORKLOADS["128k"]
-    shape = Shape(1, 2, 8192, w.d, w.p, w.L, 512, w.dtype)
+    shape = Shape(1, 2, 8192, w.d, w.p, w.L, 512, w.dtype, det)
     q, k, v, d_o = make_inputs(w, "cuda", B=1, H=2, N=8192)
     a = run_layer(shape, q, k, v, d_o)
     b = run_layer(shape, q, k, v, d_o)
     assert torch.equal(a[0], b[0])
-    for x, y in zip(a[2], b[2]):
-        assert torch.equal(x, y)
+    assert torch.equal(a[2][1], b[2][1]) and torch.equal(a[2][2], b[2][2])
+    if det:
+        assert torch.equal(a[2][0], b[2][0])
+    else:
+        x, y = a[2][0].float(), b[2][0].float()
+        assert ((x - y).abs() <= 2.0 ** -7 * torch.maximum(x.abs(), y.abs())).all()
 
 
 def test_layer_replays_as_one_cuda_graph():
     """The layer allocates nothing and never synchronises, so a whole forward + backward step
-    captures into one CUDA graph; replays with new inputs give the eager results bit for bit."""
+    captures into one CUDA graph; replays with new inputs give the eager results bit for bit
+    (in deterministic mode, so that bit equality is defined)."""
     w = WORKLOADS["128k"]
-    shape = Shape(1, 2, 8192, w.d, w.p, w.L, 512, w.dtype)
+    shape = Shape(1, 2, 8192, w.d, w.p, w.L, 512, w.dtype, deterministic=True)
     layer = LighthouseLayer(shape)
     saved = layer.new_saved()
     ins = [torch.empty(1, 2, 8192, w.d, dtype=w.dtype, device="cuda") for _ in range(4)]
@@ -208,13 +216,13 @@ def test_full_size_sampled_heads(name, unit):
 def test_autograd_module_matches_layer_calls(dtype):
     """LighthouseAttention (nn.Module over a torch.autograd.Function) returns the O, dQ, dK and dV
     of explicit LighthouseLayer forward/backward calls on the same inputs, bit for bit: the same
-    kernels run, and the layer is deterministic."""
+    kernels run, and in deterministic mode the layer is bit-reproducible."""
     name, B, H, N, S = SMALL[1] if dtype == torch.bfloat16 else SMALL[0]
     w = WORKLOADS[name]
-    shape = Shape(B, H, N, w.d, w.p, w.L, S, dtype)
+    shape = Shape(B, H, N, w.d, w.p, w.L, S, dtype, deterministic=True)
     q, k, v, d_o = (t.to(dtype) for t in make_inputs(w, "cuda", seed=3, B=B, H=H, N=N))
     o_ref, _, (dq_ref, dk_ref, dv_ref) = run_layer(shape, q, k, v, d_o)
-    attn = LighthouseAttention(w.p, w.L, S)
+    attn = LighthouseAttention(w.p, w.L, S, deterministic=True)
     qq, kk, vv = (x.clone().requires_grad_() for x in (q, k, v))
     o = attn(qq, kk, vv)
     o.backward(d_o)

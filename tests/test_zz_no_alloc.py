@@ -44,18 +44,31 @@ def _both(shape, seed):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_static_scratch_matches_workspace_version_twice(dtype):
     """Two calls in a row (the second on other inputs and sizes) give lh_attn_bwd's gradients
-    bit for bit: the same kernels run on the same inputs; only D's address differs."""
+    bit for bit: the same deterministic kernels run on the same inputs; only D's address
+    differs."""
     for seed, (H, S, d) in enumerate([(4, 1024, 128), (2, 333, 64)]):
-        shape = Shape(1, H, S, d, 4, 1, S, dtype)
+        shape = Shape(1, H, S, d, 4, 1, S, dtype, deterministic=True)
         got, want = _both(shape, seed)
         for a, b, n in zip(got, want, ("dq", "dk", "dv")):
             assert torch.equal(a, b), f"static {n} differs (call {seed})"
     assert _lib.lh_check_static() == (0, 0)  # no fault latched in the static status word
 
 
+def test_static_scratch_on_the_one_pass_backward():
+    """Without LH_DETERMINISTIC both entry points run the one-pass backward: dK and dV agree bit
+    for bit, dQ (atomic fp32 adds in a varying order) to fp32 rounding."""
+    shape = Shape(1, 4, 1024, 128, 4, 1, 1024, torch.bfloat16)
+    for seed in (11, 12):
+        (gq, gk, gv), (wq, wk, wv) = _both(shape, seed)
+        assert torch.equal(gk, wk) and torch.equal(gv, wv)
+        rms = wq.pow(2).mean().sqrt()
+        assert ((gq - wq).abs() / torch.maximum(wq.abs(), rms)).max().item() <= 1e-5
+    assert _lib.lh_check_static() == (0, 0)
+
+
 def test_static_scratch_at_its_row_limit():
     """B*H*S equal to LH_STATIC_SCRATCH_ROWS is accepted and fills D to its last row."""
-    shape = Shape(1, 256, 4096, 64, 4, 1, 4096)
+    shape = Shape(1, 256, 4096, 64, 4, 1, 4096, deterministic=True)
     assert shape.B * shape.H * shape.S == _lib.LH_STATIC_SCRATCH_ROWS
     got, want = _both(shape, 7)
     for a, b, n in zip(got, want, ("dq", "dk", "dv")):
