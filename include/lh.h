@@ -73,14 +73,19 @@ typedef struct {
   int flags;
 } lh_shape;
 
-/* Sizes derived from a shape (the pages' notation: p, L, N per level, budget S). */
+/* Sizes derived from a shape (the pages' notation: p, L, N per level, budget S).
+ * The selection is stratified: a stratum is a run of G consecutive chunks, the fewest over
+ * which the budget S divides evenly (G = C / gcd(S, C); G = 1, one chunk, whenever S is a
+ * multiple of C). Each stratum keeps its G coarsest cells and picks k more among its G*M
+ * candidates. */
 typedef struct {
   int64_t R;  /* pooled rows per (b,h): sum_{l=1}^{L-1} N/p^l */
   int64_t C;  /* chunks = coarsest cells = N/p^(L-1) */
   int64_t T;  /* tokens per chunk = p^(L-1) */
-  int64_t m;  /* subsequence rows per chunk = S/C */
-  int64_t k;  /* selected entries per chunk besides the coarsest cell = m-1 */
+  int64_t m;  /* subsequence rows per stratum = S*G/C */
+  int64_t k;  /* selected entries per stratum besides its G coarsest cells = m-G */
   int64_t M;  /* candidates per chunk = sum_{l=0}^{L-2} p^(L-1-l) */
+  int64_t G;  /* chunks per stratum = C/gcd(S, C) */
 } lh_sizes;
 
 const char* lh_status_string(int status);
@@ -88,10 +93,12 @@ const char* lh_version(void);
 
 /* Validates a shape for the GPU path and fills `out` (may be NULL).
  * Method constraints (LH_ERR_INVALID_ARG): B, H, N, d, S >= 1, p >= 2, L >= 1, dtype f32 or
- *   bf16, N % p^(L-1) == 0, S % C == 0, 1 <= S/C <= M+1.
+ *   bf16, flags 0 or LH_DETERMINISTIC, N % p^(L-1) == 0, C <= S <= C*(M+1) (every coarsest
+ *   cell kept, at most every cell).
  * GPU constraints (LH_ERR_UNSUPPORTED): d in {64, 128}; p <= 16; L <= 12; p^(L-1) <= 2^20;
- *   B*H <= 65535; N + R < 2^31; (M + k) * 8 <= 200 KiB, because a chunk's candidate keys are
- *   ranked in shared memory (at p = 4 this allows L <= 8). */
+ *   B*H <= 65535; N + R < 2^31; (G*M + k) * 8 + G * 4 <= 200 KiB, because a stratum's
+ *   candidate keys are ranked in shared memory (at p = 4 and G = 1 this allows L <= 8);
+ *   G * p^(L-1) < 2^24. */
 int lh_validate(const lh_shape* shape, lh_sizes* out);
 
 /* Bytes of the workspace `ws` that the entry points below take. The first 256 bytes hold the
@@ -128,8 +135,10 @@ int lh_score(const lh_shape* shape, const void* q, const void* k, float* score, 
              void* stream);
 
 /* Step 3 (stratified top-K, section 2.B and the article's four-stage paragraph). Per (b,h) and
- * chunk: keep the coarsest cell and the k best candidates by (r desc, level desc, position asc);
- * write their row ids in causal order (end asc, then level asc) to idx int32 [B,H,S]. */
+ * stratum (G chunks, see lh_sizes): keep the G coarsest cells and the k best candidates by
+ * (r desc, level desc, position asc); write their row ids in causal order (end asc, then level
+ * asc) to idx int32 [B,H,S], stratum after stratum (m rows each). The rows of one chunk are then
+ * contiguous and end with its coarsest cell. */
 int lh_select_topk(const lh_shape* shape, const float* score, int32_t* idx, void* stream);
 
 /* Step 4 (gather, section 2.C). x_sub[b,h,i] = row idx[b,h,i] of [x | px]. Any idx whose ids
@@ -151,8 +160,8 @@ int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, con
                 float* dk_sub, float* dv_sub, void* ws, void* stream);
 
 /* Step 6 (deterministic scatter-back, section 2.C). o[t] = sum of o_sub[i] over the rows i of
- * t's chunk whose span covers t, added in ascending i, no atomics. idx must be a valid
- * selection (causal order, coarsest cell last in each chunk). o_sub is float [B,H,S,d]. */
+ * t's stratum whose span covers t, coarsest first, no atomics. idx must be a valid selection
+ * (rows of stratum s at s*m .. s*m+m-1, each cell at most once). o_sub is float [B,H,S,d]. */
 int lh_scatter(const lh_shape* shape, const int32_t* idx, const float* o_sub, void* o,
                void* stream);
 

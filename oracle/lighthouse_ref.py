@@ -25,6 +25,7 @@ printed values.
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass
 
 import numpy as np
@@ -35,8 +36,12 @@ import numpy as np
 # ---------------------------------------------------------------------------------------
 @dataclass(frozen=True)
 class Geometry:
-    """Derived sizes of one layer call: R pooled rows, C chunks of T = p^(L-1) tokens,
-    m = S / C rows and k = m - 1 picks per chunk, M candidates per chunk."""
+    """Derived sizes of one layer call: R pooled rows, C chunks of T = p^(L-1) tokens, M
+    candidates per chunk; strata of G chunks, m = S G / C rows and k = m - G picks per stratum.
+
+    The strata are the fewest consecutive chunks over which the budget S divides evenly:
+    G = C / gcd(S, C). When S is a multiple of C (every configuration but the pages' p = 2,
+    L = 3, k = 1536 ablation), G = 1 and a stratum is one chunk."""
 
     N: int
     p: int
@@ -68,12 +73,16 @@ class Geometry:
         return self.p ** (self.L - 1)
 
     @property
+    def G(self):
+        return self.C // math.gcd(self.S, self.C)
+
+    @property
     def m(self):
-        return self.S // self.C
+        return self.S * self.G // self.C
 
     @property
     def k(self):
-        return self.m - 1
+        return self.m - self.G
 
     @property
     def M(self):
@@ -84,8 +93,8 @@ class Geometry:
             raise ValueError("need p >= 2, L >= 1, N >= 1")
         if self.N % self.T:
             raise ValueError("N must be a multiple of p^(L-1)")
-        if self.S % self.C or not (1 <= self.m <= self.M + 1):
-            raise ValueError("S must be m*C with 1 <= m <= M+1")
+        if not (self.C <= self.S <= self.C * (self.M + 1)):
+            raise ValueError("S must lie between C (the coarsest cells) and C (M + 1) (every cell)")
         return self
 
     def decode(self, rid):
@@ -160,38 +169,42 @@ def score(q, k, geo: Geometry, g):
 #    sections 2.B-2.C; the article keeps the coarsest level always).
 # ---------------------------------------------------------------------------------------
 def select_topk(r, geo: Geometry):
-    """r: float32 [B,H,N+R] -> idx int32 [B,H,S] (row ids, in subsequence order)."""
+    """r: float32 [B,H,N+R] -> idx int32 [B,H,S] (row ids, in subsequence order).
+
+    Per stratum (G consecutive chunks): keep the G coarsest cells, pick the k best of the
+    stratum's G M candidates (every cell of levels 0..L-2 inside it) by the total key (r
+    descending, level descending, position ascending), and order the m rows by (end, level)."""
     B, H, _ = r.shape
-    C, L, p, k = geo.C, geo.L, geo.p, geo.k
-    # candidates of every chunk: all cells of levels 0..L-2 inside it
+    C, L, p, G, k = geo.C, geo.L, geo.p, geo.G, geo.k
+    ns = C // G  # strata
     cand_r, cand_l, cand_j = [], [], []
     for l in range(L - 1):
-        per = p ** (L - 1 - l)  # cells of level l per chunk
-        lev = r[:, :, geo.offsets[l]:geo.offsets[l] + geo.n_level[l]].reshape(B, H, C, per)
+        per = G * p ** (L - 1 - l)  # cells of level l per stratum
+        lev = r[:, :, geo.offsets[l]:geo.offsets[l] + geo.n_level[l]].reshape(B, H, ns, per)
         cand_r.append(lev)
         cand_l.append(np.full(per, l))
-        cand_j.append(np.arange(per))  # cell index within the chunk
+        cand_j.append(np.arange(per))  # cell index within the stratum
     if L > 1:
-        cr = np.concatenate(cand_r, axis=3)  # [B,H,C,M]
+        cr = np.concatenate(cand_r, axis=3)  # [B,H,ns,G*M]
         cl = np.concatenate(cand_l)
         cj = np.concatenate(cand_j)
         # total ranking key: r descending, level descending, position ascending
         order = np.lexsort((np.broadcast_to(cj, cr.shape),
                             np.broadcast_to(-cl, cr.shape),
                             -cr), axis=-1)
-        top = order[..., :k]  # [B,H,C,k] candidate numbers
+        top = order[..., :k]  # [B,H,ns,k] candidate numbers
         sel_l = cl[top]
-        chunk = np.arange(C).reshape(1, 1, C, 1)
-        sel_j = cj[top] + chunk * (p ** (L - 1 - sel_l))  # global cell index at its level
+        stratum = np.arange(ns).reshape(1, 1, ns, 1)
+        sel_j = cj[top] + stratum * G * (p ** (L - 1 - sel_l))  # global cell index at its level
     else:
-        sel_l = np.zeros((B, H, C, 0), dtype=np.int64)
-        sel_j = np.zeros((B, H, C, 0), dtype=np.int64)
-    # append the coarsest cell of every chunk
-    coarse_l = np.full((B, H, C, 1), L - 1)
-    coarse_j = np.broadcast_to(np.arange(C).reshape(1, 1, C, 1), (B, H, C, 1))
+        sel_l = np.zeros((B, H, ns, 0), dtype=np.int64)
+        sel_j = np.zeros((B, H, ns, 0), dtype=np.int64)
+    # the G coarsest cells of every stratum
+    coarse_l = np.full((B, H, ns, G), L - 1)
+    coarse_j = np.broadcast_to(np.arange(C).reshape(1, 1, ns, G), (B, H, ns, G))
     all_l = np.concatenate([sel_l, coarse_l], axis=3)
     all_j = np.concatenate([sel_j, coarse_j], axis=3)
-    # causal order inside the chunk: ascending (end, level)
+    # causal order inside the stratum: ascending (end, level)
     end = (all_j + 1) * (p ** all_l)
     order = np.lexsort((all_l, end), axis=-1)
     all_l = np.take_along_axis(all_l, order, axis=-1)

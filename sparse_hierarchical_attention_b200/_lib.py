@@ -34,7 +34,7 @@ class lh_shape(ctypes.Structure):
 
 
 class lh_sizes(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int64) for n in ("R", "C", "T", "m", "k", "M")]
+    _fields_ = [(n, ctypes.c_int64) for n in ("R", "C", "T", "m", "k", "M", "G")]
 
 
 def _load():

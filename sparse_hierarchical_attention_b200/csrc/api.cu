@@ -40,9 +40,14 @@ int make_geo(const lh_shape* s, Geo& g) {
   if (g.N % T) return LH_ERR_INVALID_ARG;
   g.T = T;
   g.C = g.N / T;
-  if (g.S % g.C) return LH_ERR_INVALID_ARG;
-  g.m = g.S / g.C;
-  g.k = g.m - 1;
+  // Strata: the fewest consecutive chunks over which the budget S divides evenly.
+  {
+    int64_t a = g.S, b = g.C;
+    while (b) { const int64_t t = a % b; a = b; b = t; }
+    g.G = g.C / a;  // C / gcd(S, C): 1 whenever S is a multiple of C
+  }
+  g.m = g.S * g.G / g.C;  // rows per stratum
+  g.k = g.m - g.G;        // picks per stratum besides its G coarsest cells
   g.M = 0;
   for (int l = 0; l + 1 < g.L; ++l) {
     g.cand_off[l] = g.M;
@@ -50,7 +55,7 @@ int make_geo(const lh_shape* s, Geo& g) {
     for (int q = l; q + 1 < g.L; ++q) per *= g.p;
     g.M += per;
   }
-  if (g.m < 1 || g.m > g.M + 1) return LH_ERR_INVALID_ARG;
+  if (g.S < g.C || g.S > g.C * (g.M + 1)) return LH_ERR_INVALID_ARG;
   g.BH = (int64_t)g.B * g.H;
   g.R = 0;
   int64_t nl = g.N;
@@ -65,8 +70,11 @@ int make_geo(const lh_shape* s, Geo& g) {
   g.esize = g.dtype == LH_BF16 ? 2 : 4;
   if (g.BH > 65535 || g.C > 0x7fffffff) return LH_ERR_UNSUPPORTED;
   // shared-memory limits of the selection and spread kernels
-  if ((size_t)(g.M + g.k) * 8 > 200 * 1024 || (size_t)(g.M + 1) * 4 > 200 * 1024)
+  // shared-memory limits of the selection (a stratum's candidate keys, its winners and per-chunk
+  // counts) and spread kernels; the key packs a cell's stratum-local index into 24 bits
+  if ((size_t)(g.G * g.M + g.k) * 8 + (size_t)g.G * 4 > 200 * 1024 || (size_t)(g.M + 1) * 4 > 200 * 1024)
     return LH_ERR_UNSUPPORTED;
+  if (g.G * g.T >= ((int64_t)1 << 24)) return LH_ERR_UNSUPPORTED;
   return LH_OK;
 }
 
@@ -197,6 +205,7 @@ int lh_validate(const lh_shape* shape, lh_sizes* out) {
   LH_CHECK_GEO(shape, g);
   if (out) {
     out->R = g.R; out->C = g.C; out->T = g.T; out->m = g.m; out->k = g.k; out->M = g.M;
+    out->G = g.G;
   }
   return LH_OK;
 }

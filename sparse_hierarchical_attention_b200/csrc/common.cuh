@@ -14,13 +14,14 @@ constexpr uint32_t kFaultTimeout = 2u;  // a bounded wait ran out
 constexpr uint32_t kFaultDrain = 4u;    // an abort-path wait for the CTA's own operations ran out
 
 // Sizes derived from one layer shape (N_l = N/p^l cells per level, R pooled rows, C chunks of
-// T = p^(L-1) tokens, m = S/C rows and k = m-1 picks per chunk, M candidates per chunk),
-// computed on the host.
+// T = p^(L-1) tokens, M candidates per chunk; strata of G chunks with m = S G / C rows and
+// k = m - G picks each), computed on the host.
 struct Geo {
   int B, H, N, d, p, L, S, dtype;
   int flags;          // lh_shape.flags (LH_DETERMINISTIC)
   uint64_t wait_ns;   // bound of every wait inside a kernel (lh_set_wait_limit_ns)
   int64_t BH, R, C, T, m, k, M;
+  int64_t G;          // chunks per stratum (C / gcd(S, C))
   int64_t nlev[16];  // N_l = N / p^l
   int64_t off[16];   // row id of the first cell of level l (off[0] = 0, off[1] = N, ...)
   int64_t cand_off[16];  // offset of level l inside a chunk's candidate list (levels 0..L-2)

@@ -50,7 +50,7 @@ struct SpreadArgs {
   void* dst[3];
   const int32_t* idx;
   uint32_t* status;
-  int64_t N, R, S, T, m;
+  int64_t N, R, S, T, m, G;  // m rows per stratum of G chunks
   int64_t off[16];
   float inv[16];  // per-level weight: 1 (scatter) or fl32(1/p^l) (gather backward)
   int p, L, ntensor;
@@ -67,7 +67,9 @@ __device__ inline void load_row(const SRC* src, int r, int col, float* x) {
   }
 }
 
-// One CTA per (b,h, chunk). Covering cells are nested, so each token's sum is formed top-down:
+// One CTA per (b,h, chunk). It maps the rows of its stratum (the m rows s*m .. s*m+m-1 of the
+// chunk's stratum s) whose cells lie in this chunk; a row outside the stratum's cells raises the
+// index fault. Covering cells are nested, so each token's sum is formed top-down:
 // a stream of LPR lanes takes a group of p^A tokens (A = 2 when L >= 3), adds the rows of levels
 // L-1..A that cover the whole group once, then the level-1 row once per p tokens, then the
 // token's own level-0 row (the coarsest covering row first).
@@ -88,14 +90,17 @@ __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
   }
   for (int i = tid; i < tot; i += kThreads) cmap[i] = -1;
   __syncthreads();
-  for (int64_t i = c * a.m + tid; i < (c + 1) * a.m; i += kThreads) {
+  const int64_t st = c / a.G;  // this chunk's stratum
+  for (int64_t i = st * a.m + tid; i < (st + 1) * a.m; i += kThreads) {
     const int64_t rid = a.idx[bh * a.S + i];
     int lvl = 0;
     if (rid < 0 || rid >= a.N + a.R) { raise_fault(a.status, kFaultIndex); continue; }
     for (int l = 1; l < L; ++l)
       if (rid >= a.off[l]) lvl = l;
+    const int64_t in_stratum = rid - a.off[lvl] - st * a.G * per[lvl];
+    if (in_stratum < 0 || in_stratum >= a.G * per[lvl]) { raise_fault(a.status, kFaultIndex); continue; }
     const int64_t local = rid - a.off[lvl] - c * per[lvl];
-    if (local < 0 || local >= per[lvl]) { raise_fault(a.status, kFaultIndex); continue; }
+    if (local < 0 || local >= per[lvl]) continue;  // a cell of another chunk of the stratum
     cmap[base[lvl] + (int)local] = (int)i;
   }
   __syncthreads();
@@ -205,7 +210,7 @@ cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool sr
   SpreadArgs a{};
   for (int i = 0; i < ntensor; ++i) { a.src[i] = src[i]; a.dst[i] = dst[i]; }
   a.idx = idx; a.status = status;
-  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.G = g.G;
   a.p = g.p; a.L = g.L; a.ntensor = ntensor;
   for (int l = 0; l < 16; ++l) {
     a.off[l] = l < g.L ? g.off[l] : 0;

@@ -46,7 +46,7 @@ struct PoolArgs {
   float* tmp;        // level-A2 fp32 sums [BH, N/p^A2, ntensor, D] then maxima [BH, N/p^A2, 2]
   const int32_t* idx;  // span sums: the selection [BH, S]
   uint32_t* status;
-  int64_t N, R, S, T, m, C;
+  int64_t N, R, S, T, m, C, G;  // m rows per stratum of G chunks
   int64_t off[16];    // row id offsets of levels
   float inv[16];      // fl32(1 / p^l)
   int wdiv[8];        // W / p^l for l = 1..A: level-l cells per stream
@@ -136,9 +136,10 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
     }
     for (int i = tid; i < acc; i += kThreads) smap[i] = -1;
     __syncthreads();
+    // the rows of the strata that hold this tile's chunks; cells outside the tile are skipped
     const int64_t c0 = t_tile / a.T;
     const int64_t c1 = std::min<int64_t>((t_tile + tile - 1) / a.T, a.C - 1);
-    const int64_t r0 = c0 * a.m, r1 = (c1 + 1) * a.m;
+    const int64_t r0 = (c0 / a.G) * a.m, r1 = (c1 / a.G + 1) * a.m;
     for (int64_t i = r0 + tid; i < r1; i += kThreads) {
       const int64_t rid = a.idx[bh * a.S + i];
       if (rid < 0 || rid >= NR) { raise_fault(a.status, kFaultIndex); continue; }
@@ -415,7 +416,8 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
     }
     for (int i = tid; i < tot; i += blockDim.x) cmap[i] = -1;
     __syncthreads();
-    for (int64_t i = chunk * a.m + tid; i < (chunk + 1) * a.m; i += blockDim.x) {
+    const int64_t st = chunk / a.G;  // the rows of this chunk's stratum; other chunks' cells skipped
+    for (int64_t i = st * a.m + tid; i < (st + 1) * a.m; i += blockDim.x) {
       const int64_t rid = a.idx[bh * a.S + i];
       if (rid < 0 || rid >= a.N + a.R) { raise_fault(a.status, kFaultIndex); continue; }
       int lvl; int64_t cell;
@@ -531,7 +533,7 @@ cudaError_t launch_tile(const Plan& pl, const PoolArgs& a, int64_t BH, cudaStrea
 template <int MODE>
 cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
   const Plan pl = make_plan(g, MODE == MODE_SPANSUM ? kWMaxSpan : kWMaxPyr);
-  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C; a.G = g.G;
   a.p = g.p; a.L = g.L; a.W = pl.W; a.A2 = pl.A2; a.U = pl.U;
   for (int l = 0, w = pl.W; l < 8; ++l) {  // level-(l+1) cells per stream
     w = l < pl.A ? w / g.p : 0;

@@ -2,13 +2,15 @@
 // 2.B: joint top-K over all levels; the Nous Research article's four-stage paragraph: the
 // selection is stratified and always keeps the coarsest level).
 //
-// One CTA per (b,h, chunk). The chunk's M candidate scores become 64-bit keys that encode the
-// total ranking order (score descending, then level descending, then position ascending): high word = the fp32 score bits (scores are >= +0, so
-// the bit pattern orders like the value), then the level (higher wins), then the position
-// (lower wins). A most-significant-digit radix select (8-bit digits, shared-memory histograms,
-// one warp scanning the 256 bins) finds the k-th largest key; it stops as soon as the bucket
-// that holds the k-th key is taken whole. The k winners are then placed in causal order
-// (end, level) by counting, and the chunk's coarsest cell goes last.
+// One CTA per (b,h, stratum of G chunks; G = 1 whenever S is a multiple of the chunk count).
+// The stratum's G*M candidate scores become 64-bit keys that encode the total ranking order
+// (score descending, then level descending, then position ascending): high word = the fp32 score
+// bits (scores are >= +0, so the bit pattern orders like the value), then the level (higher
+// wins), then the stratum-local position (lower wins). A most-significant-digit radix select
+// (8-bit digits, shared-memory histograms, one warp scanning the 256 bins) finds the k-th
+// largest key; it stops as soon as the bucket that holds the k-th key is taken whole. The k
+// winners are then placed in causal order (end, level) by counting, each chunk's coarsest cell
+// right after the winners of that chunk.
 #include "common.cuh"
 
 namespace lh {
@@ -17,37 +19,43 @@ namespace {
 struct SelArgs {
   const float* score;
   int32_t* idx;
-  int64_t N, R, S, m, k, M;
+  int64_t N, R, S, m, k, M, G, T;
   int64_t off[16];
-  int64_t cand_off[16];
   int p, L;
 };
 
 template <int kSelThreads>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
-  extern __shared__ unsigned long long keys[];  // [M] candidate keys, then [k] winners
+  // [G*M] candidate keys, then [k] winners, then [G] winners per chunk of the stratum
+  extern __shared__ unsigned long long keys[];
   __shared__ unsigned hist[256];
   __shared__ int s_digit, s_need, s_cnt, s_nsel;
 
   const int tid = threadIdx.x;
-  const int64_t bh = blockIdx.y, c = blockIdx.x;
+  const int64_t bh = blockIdx.y, st = blockIdx.x;  // stratum st: chunks st*G .. st*G + G-1
   const float* sc = a.score + bh * (a.N + a.R);
-  int32_t* out = a.idx + bh * a.S + c * a.m;
-  const int L = a.L, p = a.p;
-  const int M = (int)a.M, k = (int)a.k;
+  int32_t* out = a.idx + bh * a.S + st * a.m;
+  const int L = a.L, p = a.p, G = (int)a.G;
+  const int M = (int)(a.G * a.M), k = (int)a.k;  // candidates and picks of the stratum
+  int* per_chunk = reinterpret_cast<int*>(keys + M + k);
 
-  // 1. candidate keys: level l holds p^(L-1-l) cells per chunk
-  for (int l = 0; l < L - 1; ++l) {
-    int per = 1;
-    for (int q = l; q < L - 1; ++q) per *= p;
-    const int base = (int)a.cand_off[l];
-    for (int jl = tid; jl < per; jl += kSelThreads) {
-      const float r = sc[a.off[l] + c * per + jl];
-      const unsigned long long key = ((unsigned long long)__float_as_uint(r) << 32) |
-                                     ((unsigned long long)l << 24) | (unsigned)(0xFFFFFF - jl);
-      keys[base + jl] = key;
+  // 1. candidate keys: level l holds G p^(L-1-l) cells per stratum. The key orders by score,
+  //    then level (higher first), then stratum-local position (lower first).
+  {
+    int base = 0;
+    for (int l = 0; l < L - 1; ++l) {
+      int per = G;
+      for (int q = l; q < L - 1; ++q) per *= p;
+      for (int jl = tid; jl < per; jl += kSelThreads) {
+        const float r = sc[a.off[l] + st * per + jl];
+        const unsigned long long key = ((unsigned long long)__float_as_uint(r) << 32) |
+                                       ((unsigned long long)l << 24) | (unsigned)(0xFFFFFF - jl);
+        keys[base + jl] = key;
+      }
+      base += per;
     }
   }
+  for (int i = tid; i < G; i += kSelThreads) per_chunk[i] = 0;
   if (tid == 0) s_nsel = 0;
   __syncthreads();
 
@@ -111,8 +119,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
       }
     }
     __syncthreads();
-    // 4. causal order: rank by (end, level) among the winners
     const int nsel = s_nsel < k ? s_nsel : k;
+    for (int w = tid; w < nsel; w += kSelThreads) {  // winners per chunk of the stratum
+      const int l = (int)((win[w] >> 24) & 0xFF);
+      const int jl = 0xFFFFFF - (int)(win[w] & 0xFFFFFF);
+      int64_t pw = 1;
+      for (int q = 0; q < l; ++q) pw *= p;
+      atomicAdd(&per_chunk[(int)((int64_t)jl * pw / a.T)], 1);
+    }
+    __syncthreads();
+    // 4. causal order: a winner's row is its rank by (end, level) among the winners plus the
+    //    coarsest cells of the chunks before its own (they end before it starts)
     for (int w = tid; w < nsel; w += kSelThreads) {
       const unsigned long long key = win[w];
       const int l = (int)((key >> 24) & 0xFF);
@@ -129,12 +146,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
         for (int q = 0; q < l2; ++q) pw2 *= p;
         rank += ((((int64_t)j2 + 1) * pw2) * 16 + l2) < ord;
       }
-      int per = 1;
+      int per = G;
       for (int q = l; q < L - 1; ++q) per *= p;
-      if (rank < a.m - 1) out[rank] = (int32_t)(a.off[l] + c * per + jl);
+      const int row = rank + (int)((int64_t)jl * pw / a.T);
+      if (row < a.m) out[row] = (int32_t)(a.off[l] + st * per + jl);
     }
   }
-  if (tid == 0) out[a.m - 1] = (int32_t)(a.off[L - 1] + c);
+  // the coarsest cell of chunk cl comes after the winners of chunks 0..cl and the cl coarsest
+  // cells before it
+  for (int cl = tid; cl < G; cl += kSelThreads) {
+    int before = cl;
+    for (int u = 0; u <= cl; ++u) before += per_chunk[u];
+    if (before < a.m) out[before] = (int32_t)(a.off[L - 1] + st * G + cl);
+  }
 }
 
 }  // namespace
@@ -142,16 +166,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a) {
 cudaError_t launch_select(const Geo& g, const float* score, int32_t* idx, cudaStream_t st) {
   SelArgs a{};
   a.score = score; a.idx = idx;
-  a.N = g.N; a.R = g.R; a.S = g.S; a.m = g.m; a.k = g.k; a.M = g.M;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.m = g.m; a.k = g.k; a.M = g.M; a.G = g.G; a.T = g.T;
   a.p = g.p; a.L = g.L;
-  for (int l = 0; l < 16; ++l) {
-    a.off[l] = l < g.L ? g.off[l] : 0;
-    a.cand_off[l] = l < g.L ? g.cand_off[l] : 0;
-  }
-  const size_t smem = (size_t)(g.M + g.k) * sizeof(unsigned long long);
-  dim3 grid((unsigned)g.C, (unsigned)g.BH);
+  for (int l = 0; l < 16; ++l) a.off[l] = l < g.L ? g.off[l] : 0;
+  const size_t smem = (size_t)(g.G * g.M + g.k) * sizeof(unsigned long long) + (size_t)g.G * sizeof(int);
+  dim3 grid((unsigned)(g.C / g.G), (unsigned)g.BH);
   // The kernel is bound by latency (shared-memory passes, synchronisations), so what counts is
-  // how many chunks an SM holds at once. Up to 16 KB of keys, 128-thread CTAs fit 16 per SM
+  // how many strata an SM holds at once. Up to 16 KB of keys, 128-thread CTAs fit 16 per SM
   // (2048 threads); with more keys shared memory caps the CTAs per SM, and 256 threads each keep
   // the passes short (measured: 1364 keys 70 -> 59 us with 128 threads, 5460 keys 78 -> 91 us).
   cudaError_t e;

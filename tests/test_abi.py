@@ -21,11 +21,14 @@ def test_version():
 
 
 @pytest.mark.parametrize("N,p,L,S,want", [
-    (131072, 4, 6, 8192, dict(R=43648, C=128, T=1024, m=64, k=63, M=1364)),
-    (1048576, 4, 7, 16384, dict(R=349440, C=256, T=4096, m=64, k=63, M=5460)),
-    (98304, 4, 6, 6144, dict(R=32736, C=96, T=1024, m=64, k=63, M=1364)),
-    (2048, 4, 3, 512, dict(R=640, C=128, T=16, m=4, k=3, M=20)),
-    (640, 4, 1, 640, dict(R=0, C=640, T=1, m=1, k=0, M=0)),
+    (131072, 4, 6, 8192, dict(R=43648, C=128, T=1024, m=64, k=63, M=1364, G=1)),
+    (1048576, 4, 7, 16384, dict(R=349440, C=256, T=4096, m=64, k=63, M=5460, G=1)),
+    (98304, 4, 6, 6144, dict(R=32736, C=96, T=1024, m=64, k=63, M=1364, G=1)),
+    (2048, 4, 3, 512, dict(R=640, C=128, T=16, m=4, k=3, M=20, G=1)),
+    (640, 4, 1, 640, dict(R=0, C=640, T=1, m=1, k=0, M=0, G=1)),
+    # the pages' ablation p = 2, L = 3, k = 1536 at 98K: S = C + k, strata of 16 chunks
+    (98304, 2, 3, 24576 + 1536, dict(R=73728, C=24576, T=4, m=17, k=1, M=6, G=16)),
+    (4096, 4, 3, 256 + 96, dict(R=1280, C=256, T=16, m=11, k=3, M=20, G=8)),
 ])
 def test_sizes(N, p, L, S, want):
     assert lh.lh_validate(Shape(1, 2, N, 128, p, L, S)) == want
@@ -33,7 +36,7 @@ def test_sizes(N, p, L, S, want):
 
 @pytest.mark.parametrize("bad", [
     Shape(1, 2, 1000, 128, 4, 6, 64),      # N not a multiple of p^(L-1)
-    Shape(1, 2, 4096, 128, 4, 6, 102),     # S not a multiple of C = 4
+    Shape(1, 2, 4096, 128, 4, 6, 3),       # S < C = 4: not every coarsest cell fits
     Shape(1, 2, 4096, 128, 4, 3, 256 * 22),  # m = 22 > M + 1 = 21
     Shape(0, 2, 4096, 128, 4, 3, 256),     # empty batch
     Shape(1, 2, 4096, 128, 1, 3, 256),     # p < 2
@@ -54,6 +57,7 @@ def test_unsupported_head_dim():
     (Shape(1, 1, 2 * 2 ** 12, 64, 2, 13, 2), 2),     # L = 13
     (Shape(1, 1, 2 * 16 ** 2, 64, 16, 3, 2 * 17), 0),  # p = 16, L = 3
     (Shape(1, 1, 2 * 2 ** 11, 64, 2, 12, 2 * 64), 0),  # p = 2, L = 12
+    (Shape(1, 1, 98304, 64, 2, 3, 24576 + 1), 2),    # one stratum of all 24576 chunks: too many keys
 ])
 def test_gpu_path_limits(shape, status):
     assert _lib.lh_validate_status(shape) == status

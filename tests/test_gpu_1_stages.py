@@ -72,7 +72,10 @@ def test_pyramid_and_score(B, H, N, d, p, L, S, dt):
 SEL_SHAPES = [(1, 2, 4096, 128, 4, 5, 1024), (2, 3, 2048, 64, 4, 3, 512),
               (1, 2, 8192, 128, 4, 6, 8 * 64), (1, 2, 1024, 128, 2, 6, 32 * 32),
               (1, 2, 2187, 64, 3, 4, 27 * 3), (1, 1, 1024, 64, 4, 4, 16 * 85),
-              (1, 3, 640, 128, 4, 1, 640), (1, 2, 4096, 64, 4, 6, 4 * 1)]
+              (1, 3, 640, 128, 4, 1, 640), (1, 2, 4096, 64, 4, 6, 4 * 1),
+              # strata of G > 1 chunks (S no multiple of C): G = 16, 8, 2, and one stratum
+              (1, 2, 4096, 64, 2, 3, 1024 + 64), (1, 2, 4096, 128, 4, 3, 256 + 96),
+              (2, 2, 2048, 64, 4, 4, 32 * 5 + 16), (1, 1, 729, 64, 3, 4, 27 + 1)]
 
 
 @pytest.mark.parametrize("quantised", [False, True])
@@ -133,7 +136,8 @@ def valid_idx(B, H, N, p, L, S, seed):
 
 SPREAD_SHAPES = [(1, 2, 4096, 128, 4, 5, 1024), (2, 3, 2048, 64, 4, 3, 512),
                  (1, 2, 1024, 128, 2, 6, 32 * 32), (1, 2, 2187, 64, 3, 4, 81),
-                 (1, 3, 640, 128, 4, 1, 640), (1, 1, 16384, 128, 4, 7, 64)]
+                 (1, 3, 640, 128, 4, 1, 640), (1, 1, 16384, 128, 4, 7, 64),
+                 (1, 2, 4096, 64, 2, 3, 1024 + 64), (2, 2, 2048, 128, 4, 4, 32 * 5 + 16)]
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
@@ -214,4 +218,4 @@ def test_fused_backward_matches_the_deterministic_one(B, H, S):
     assert torch.equal(fk, dk) and torch.equal(fv, dv)
     rms = dq.pow(2).mean().sqrt()
     err = (fq - dq).abs() / torch.maximum(dq.abs(), rms)
-    assert err.max().item() <= 1e-5, err.max().item()
+    assert err.max().item() <= 1e-4, err.max().item()

@@ -87,6 +87,9 @@ def test_unit_variance_literal_thresholds(name, B, H, N, S, dtype):
     (1, 1, 2048, 64, 16, 3, 8 * 17),    # p = 16, the largest pooling factor
     (1, 1, 4096, 64, 2, 12, 2 * 64),    # L = 12, the most levels: five tree levels and a coarse pass
     (1, 1, 32768, 128, 4, 8, 2 * 64),   # M = 21844 candidates per chunk, near the shared-memory limit
+    (1, 2, 4096, 64, 2, 3, 1024 + 64),  # strata of G = 16 chunks (p = 2, L = 3, one pick per stratum)
+    (1, 2, 4096, 128, 4, 3, 256 + 96),  # G = 8, S = 352 (ragged attention tiles)
+    (1, 1, 729, 64, 3, 4, 28),          # one stratum over the whole sequence
 ])
 def test_layer_edge_cases(B, H, N, d, p, L, S, dtype):
     shape = Shape(B, H, N, d, p, L, S, dtype)
@@ -231,3 +234,27 @@ def test_autograd_module_matches_layer_calls(dtype):
     assert torch.equal(qq.grad, dq_ref)
     assert torch.equal(kk.grad, dk_ref)
     assert torch.equal(vv.grad, dv_ref)
+
+
+@pytest.mark.parametrize("det", [False, True])
+def test_pages_ablation_p2_L3_k1536(det):
+    """The pages' best ablation (Lighthouse summary, technical summary 4, hyper-parameter bullet):
+    p = 2, L = 3 and a top-K budget of k = 1536, at the 98K context of the 530M model (d = 64).
+    The 24576 coarsest cells are all kept, so S = 24576 + 1536 = 26112 rows; the budget divides
+    evenly over strata of 16 chunks (64 tokens), one pick each. One head is checked whole."""
+    w = WORKLOADS["llama530m-98k"]
+    N, p, L = 98304, 2, 3
+    C = N // p ** (L - 1)
+    S = C + 1536
+    shape = Shape(1, 2, N, w.d, p, L, S, w.dtype, det)
+    sz = lh.lh_validate(shape)
+    assert (sz["C"], sz["G"], sz["m"], sz["k"]) == (24576, 16, 17, 1)
+    q, k, v, d_o = make_inputs(w, "cuda", seed=0, B=1, H=2, N=N)
+    o, saved, grads = run_layer(shape, q, k, v, d_o)
+    geo = O.Geometry(N, p, L, S).check()
+    sl = (slice(0, 1), slice(1, 2))
+    wo, sv, wgrads = oracle_layer(q[sl], k[sl], v[sl], d_o[sl], geo, w.dtype)
+    assert np.array_equal(saved_views(shape, saved)["idx"][sl].cpu().numpy(), sv["idx"])
+    assert_close(np64(o[sl]), wo, w.dtype, "O")
+    for got, want, n in zip(grads, wgrads, ("dQ", "dK", "dV")):
+        assert_close(np64(got[sl]), want, w.dtype, n)

@@ -28,6 +28,15 @@ SMALL = [  # (N, p, L, S)
     (16, 2, 3, 8), (16, 2, 3, 16), (32, 4, 2, 16), (64, 4, 3, 16), (27, 3, 3, 9),
     (64, 2, 4, 40), (8, 2, 1, 8), (48, 4, 3, 12),
 ]
+# budgets that are no multiple of the chunk count C: strata of G = C / gcd(S, C) chunks
+STRATA = [  # (N, p, L, S): G
+    (16, 2, 3, 6),     # C = 4: G = 2, 3 rows per stratum
+    (64, 4, 3, 18),    # C = 4: G = 2, 9 rows
+    (64, 2, 4, 12),    # C = 8: G = 2, 3 rows
+    (27, 3, 3, 4),     # C = 3: G = 3, one stratum over the whole sequence
+    (96, 2, 3, 26),    # C = 24: G = 12, 13 rows
+    (128, 2, 3, 34),   # C = 32: G = 16, 17 rows (the structure of p = 2, L = 3, k = 1536 at 98K)
+]
 
 
 # ---------------------------------------------------------------- pyramid (section 2.A)
@@ -98,22 +107,26 @@ def test_coarse_score_is_max_over_span(N, p, L, S):
 
 # ---------------------------------------------------------------- selection (2.B, 2.C)
 def brute_select(r, geo):
-    """Every chunk: full sort of all its candidates by the total key, then causal order."""
+    """Every stratum of G chunks: full sort of all its candidates by the total key, the k best
+    plus the G coarsest cells, then causal order."""
     out = []
-    for c in range(geo.C):
+    G = geo.C // math.gcd(geo.S, geo.C)  # restated here from the reading, not taken from geo
+    k = geo.S * G // geo.C - G
+    assert (G, k) == (geo.G, geo.k)
+    for s in range(geo.C // G):
         cands = []
         for l in range(geo.L - 1):
-            per = geo.p ** (geo.L - 1 - l)
-            for j in range(c * per, (c + 1) * per):
+            per = geo.p ** (geo.L - 1 - l)  # cells of level l in one chunk
+            for j in range(s * G * per, (s + 1) * G * per):
                 cands.append((float(r[geo.offsets[l] + j]), l, j))
-        best = sorted(cands, key=lambda e: (-e[0], -e[1], e[2]))[:geo.k]
-        rows = [(l, j) for _, l, j in best] + [(geo.L - 1, c)]
+        best = sorted(cands, key=lambda e: (-e[0], -e[1], e[2]))[:k]
+        rows = [(l, j) for _, l, j in best] + [(geo.L - 1, c) for c in range(s * G, (s + 1) * G)]
         rows.sort(key=lambda e: ((e[1] + 1) * geo.p ** e[0], e[0]))
         out += [geo.offsets[l] + j for l, j in rows]
     return out
 
 
-@pytest.mark.parametrize("N,p,L,S", SMALL)
+@pytest.mark.parametrize("N,p,L,S", SMALL + STRATA)
 def test_topk_equals_full_sort(N, p, L, S):
     geo = O.Geometry(N, p, L, S).check()
     # quantised scores so that exact ties (and the tie-break) occur often
@@ -123,6 +136,33 @@ def test_topk_equals_full_sort(N, p, L, S):
     idx = O.select_topk(r, geo)
     for b, h in itertools.product(range(2), range(2)):
         assert idx[b, h].tolist() == brute_select(r[b, h], geo)
+
+
+@pytest.mark.parametrize("N,p,L,S", STRATA)
+def test_topk_strata_invariants(N, p, L, S):
+    """Every stratum keeps its G coarsest cells and k picks from inside it, in causal order;
+    the rows of one chunk are contiguous and end with its coarsest cell."""
+    geo = O.Geometry(N, p, L, S).check()
+    assert geo.G > 1 and geo.C % geo.G == 0 and geo.m * (geo.C // geo.G) == S
+    r = O.score(rand(1, 2, N, 8), rand(1, 2, N, 8), geo, 8)
+    idx = O.select_topk(r, geo)
+    level, cell = geo.decode(idx)
+    end = (cell + 1) * geo.p ** level
+    start = end - geo.p ** level
+    span = geo.G * geo.T
+    for h in range(2):
+        assert len(set(idx[0, h].tolist())) == S
+        for s in range(geo.C // geo.G):
+            rows = slice(s * geo.m, (s + 1) * geo.m)
+            lv, ce, st, en = level[0, h, rows], cell[0, h, rows], start[0, h, rows], end[0, h, rows]
+            assert (st >= s * span).all() and (en <= (s + 1) * span).all()
+            assert sorted(ce[lv == L - 1].tolist()) == list(range(s * geo.G, (s + 1) * geo.G))
+            key = list(zip(en.tolist(), lv.tolist()))
+            assert key == sorted(key) and len(set(key)) == len(key)
+            chunk = st // geo.T
+            assert (np.diff(chunk) >= 0).all()  # chunk segments are contiguous
+            last = np.r_[chunk[1:] != chunk[:-1], True]
+            assert (lv[last] == L - 1).all()  # each segment ends with its chunk's coarsest cell
 
 
 @pytest.mark.parametrize("N,p,L,S", SMALL)
@@ -152,7 +192,7 @@ def test_topk_worked_example(golden_dir):
     k = np.zeros_like(q)
     q[0, 0, :, 0] = ex["q_norms"]
     k[0, 0, :, 1] = ex["k_norms"]
-    for S, want in ex["idx"].items():
+    for S, want in list(ex["idx"].items()) + list(ex["idx_strata"].items()):
         geo = O.Geometry(sh["N"], sh["p"], sh["L"], int(S)).check()
         r = O.score(q, k, geo, 4)
         assert r[0, 0].tolist() == ex["score"]
@@ -235,7 +275,8 @@ def by_definition_layer(q, k, v, geo, g):
 
 
 @pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (32, 4, 3, 8), (27, 3, 3, 9),
-                                     (32, 2, 3, 8 * 7), (8, 2, 1, 8)])
+                                     (32, 2, 3, 8 * 7), (8, 2, 1, 8), (16, 2, 3, 6), (27, 3, 3, 4),
+                                     (96, 2, 3, 26)])
 def test_layer_equals_by_definition(N, p, L, S):
     geo = O.Geometry(N, p, L, S).check()
     q, k, v = (rand(1, 2, N, 8) for _ in range(3))
@@ -259,7 +300,7 @@ def test_recovery_identity_dense_sdpa():
 
 
 # ---------------------------------------------------------------- scatter and adjoints (2.C)
-@pytest.mark.parametrize("N,p,L,S", SMALL)
+@pytest.mark.parametrize("N,p,L,S", SMALL + STRATA)
 def test_scatter_adjoints(N, p, L, S):
     """scatter_bwd is the adjoint of scatter; gather_bwd is the adjoint of pool-then-gather."""
     geo = O.Geometry(N, p, L, S).check()
@@ -286,14 +327,17 @@ def test_every_token_covered_between_1_and_L_times():
 
 
 # ---------------------------------------------------------------- causality (2.C, 5)
-@pytest.mark.parametrize("N,p,L,S", [(64, 4, 3, 16), (64, 2, 4, 40), (16, 2, 1, 16)])
+@pytest.mark.parametrize("N,p,L,S", [(64, 4, 3, 16), (64, 2, 4, 40), (16, 2, 1, 16),
+                                     (64, 2, 4, 12), (96, 2, 3, 26)])
 def test_future_chunks_do_not_change_the_past(N, p, L, S):
+    """Perturbing the tokens of stratum s and later (a stratum is G chunks; G = 1 when S is a
+    multiple of C) changes no output of the strata before s."""
     geo = O.Geometry(N, p, L, S).check()
     q, k, v = (rand(1, 2, N, 8) for _ in range(3))
     o, _ = O.layer_fwd(q, k, v, geo, 4)
-    for c in range(1, geo.C):
+    for c in range(1, geo.C // geo.G):
         q2, k2, v2 = q.copy(), k.copy(), v.copy()
-        t0 = c * geo.T
+        t0 = c * geo.G * geo.T
         for x in (q2, k2, v2):
             x[:, :, t0:] = rand(1, 2, N - t0, 8, scale=3.0)
         o2, _ = O.layer_fwd(q2, k2, v2, geo, 4)
@@ -302,7 +346,8 @@ def test_future_chunks_do_not_change_the_past(N, p, L, S):
 
 
 # ---------------------------------------------------------------- gradients (2.B)
-@pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (32, 4, 2, 16), (27, 3, 3, 9), (8, 2, 1, 8)])
+@pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (32, 4, 2, 16), (27, 3, 3, 9), (8, 2, 1, 8),
+                                     (16, 2, 3, 6)])
 def test_gradients_finite_differences(N, p, L, S):
     """Central differences in fp64 with the selection held fixed (it is piecewise constant)."""
     geo = O.Geometry(N, p, L, S).check()
