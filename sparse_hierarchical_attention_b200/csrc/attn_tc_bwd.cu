@@ -12,12 +12,11 @@
 //       dV += P^T dO and dK += dS^T Q (accumulated in tensor memory over the whole block), and
 //       dQ^T = K^T dS^T for this query block (fresh every step), which the warps add into the
 //       fp32 dq_sub rows with atomic adds (red.global.add.f32). dq_sub is zeroed first.
-//     P^T and dS^T go to 128-byte-swizzled shared-memory tiles [128 keys][64 queries]: P^T is
-//     the K-major A operand of dV, dS^T at once the K-major A operand of dK and the MN-major B
-//     operand of dQ^T, whose A operand K^T the warps place in tensor memory once per CTA. So
-//     each step's S and dP are computed once for all three gradients. dV and dK are
-//     deterministic; the order in which the key blocks' dQ terms reach a dq_sub row varies from
-//     run to run.
+//     P^T goes to tensor memory (A operand of dV). dS^T goes to one 128-byte-swizzled
+//     shared-memory tile [128 keys][64 queries] that is at once the K-major A operand of dK and
+//     the MN-major B operand of dQ^T; K^T is the CTA's K tile read MN-major. So each step's S and
+//     dP are computed once for all three gradients. dV and dK are deterministic; the order in
+//     which the key blocks' dQ terms reach a dq_sub row varies from run to run.
 //   deterministic (LH_DETERMINISTIC, and every d = 64 call): two kernels without atomics:
 //     dkdv: the fused kernel's dV/dK part, with dS^T in tensor memory;
 //     dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
@@ -353,20 +352,15 @@ struct LayFused {
   static constexpr int Q = V + KB * T128;          // kStF stages of [64][D]
   static constexpr int DO = Q + kStF * KB * T64;   // kStF stages of [64][D]
   static constexpr int DS = DO + kStF * KB * T64;  // dS^T hi, then lo: [128 keys][64 queries] each
-  static constexpr int PT = DS + 2 * T128;         // P^T hi, then lo: [128 keys][64 queries] each
-  static constexpr int VEC = PT + 2 * T128;        // kStF stages of lse[64], delta[64]
+  static constexpr int VEC = DS + 2 * T128;        // kStF stages of lse[64], delta[64]
   static constexpr int BAR = VEC + kStF * 512;
-  static constexpr int BYTES = BAR + 256;          // 231168 at D = 128: 227 KB with the alignment
+  static constexpr int BYTES = BAR + 256;
 };
 
 // bars: 0 K+V | 1-3 Q/dO stages loaded | 4 S ready | 5 S read | 6 P written | 7 acc done
 //       | 8-10 Q/dO stages free | 11-12 drain of the two MMA issuers
-// TMEM columns: S^T 0-63, dP^T 64-127, dV 128-255, dK 256-383, K^T 384-447 (lanes = the D
-// columns, 128 keys as bf16 pairs: the A operand of dQ^T, written once), dQ^T 448-511 (lanes =
-// the D columns of dQ, columns = the step's 64 queries). P^T and dS^T live in shared memory:
-// with both in one 128-byte-swizzled [keys][queries] layout, dV and dK are SS MMAs at N = 128
-// (bound by the math rate), and the N = 64 dQ^T MMAs read only their B operand (2 KB) from
-// shared memory instead of 6 KB, which at 128 B per clock bounded them below the math rate.
+// TMEM columns: S^T 0-63, dP^T 64-127, dV 128-255, dK 256-383, P^T hi 384, lo 416 (64 queries
+// as bf16 pairs), dQ^T 448-511 (lanes = the D columns of dQ, columns = the step's 64 queries)
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -412,13 +406,13 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t t_st = tbase, t_dpt = tbase + 64, t_dv = tbase + 128, t_dk = tbase + 256;
-  const uint32_t t_kt = tbase + 384, t_dqt = tbase + 448;
+  const uint32_t t_pt = tbase + 384, t_dqt = tbase + 448;
   const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
   const uint32_t s_q = smem_u32(sm + Ly::Q), s_do = smem_u32(sm + Ly::DO);
-  const uint32_t s_ds = smem_u32(sm + Ly::DS), s_pt = smem_u32(sm + Ly::PT);
+  const uint32_t s_ds = smem_u32(sm + Ly::DS);
   constexpr uint32_t IDESC_S = idesc_bf16(128, 64, false, false);
   constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
-  constexpr uint32_t IDESC_DQ = idesc_bf16(128, 64, false, true);  // A = K^T (TMEM), B = dS^T MN-major
+  constexpr uint32_t IDESC_DQ = idesc_bf16(128, 64, true, true);  // A = K^T, B = dS^T: both MN-major
 
   if (warp == kCompute / 32) {
     // ------------------------------------------------------------------ TMA warp
@@ -460,7 +454,7 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       const uint64_t dQm = desc_base(T64, 1024) + (s_q >> 4), dOm = desc_base(T64, 1024) + (s_do >> 4);
       const uint64_t dSk = desc_base(16, 1024) + (s_ds >> 4);     // dS^T as A of dK, K-major
       const uint64_t dSm = desc_base(T128, 1024) + (s_ds >> 4);   // dS^T as B of dQ^T (N = 64)
-      const uint64_t dPk = desc_base(16, 1024) + (s_pt >> 4);     // P^T as A of dV, K-major
+      const uint64_t dKm = desc_base(T128, 1024) + (s_k >> 4);    // K^T as A of dQ^T (M = 128)
       auto issue_s = [&](int it) {  // S^T = K Q^T, dP^T = V dO^T
         const uint32_t sg = (uint32_t)((it % kStF) * KB * T64) >> 4;
 #pragma unroll
@@ -478,17 +472,17 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t bq = dQm + sg + ks * 128, bo = dOm + sg + ks * 128;  // + ks * 2048 bytes
           const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
-          mma_ss(t_dv, dPk + ks * 2, bo, IDESC_ACC, acc);                     // + ks * 32 bytes
-          mma_ss(t_dv, dPk + (T128 >> 4) + ks * 2, bo, IDESC_ACC, 1u);
-          mma_ss(t_dk, dSk + ks * 2, bq, IDESC_ACC, acc);
+          mma_ts(t_dv, t_pt + ks * 8, bo, IDESC_ACC, acc);
+          mma_ts(t_dv, t_pt + 32 + ks * 8, bo, IDESC_ACC, 1u);
+          mma_ss(t_dk, dSk + ks * 2, bq, IDESC_ACC, acc);                     // + ks * 32 bytes
           mma_ss(t_dk, dSk + (T128 >> 4) + ks * 2, bq, IDESC_ACC, 1u);
         }
         // dQ^T = K^T (dS^T_hi + dS^T_lo), 16 keys per MMA, fresh for this query block
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t b = dSm + kk * 128;  // + kk * 2048 bytes
-          mma_ts(t_dqt, t_kt + kk * 8, b, IDESC_DQ, kk > 0 ? 1u : 0u);
-          mma_ts(t_dqt, t_kt + kk * 8, b + (T128 >> 4), IDESC_DQ, 1u);
+          const uint64_t a = dKm + kk * 128, b = dSm + kk * 128;  // + kk * 2048 bytes
+          mma_ss(t_dqt, a, b, IDESC_DQ, kk > 0 ? 1u : 0u);
+          mma_ss(t_dqt, a, b + (T128 >> 4), IDESC_DQ, 1u);
         }
         mma_commit(bar_acc);
         mma_commit(bar_stfree + it % kStF);  // the stage of step it is free once this completes
@@ -518,9 +512,8 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
     const int row = (warp % 4) * 32 + (tid % 32);  // key row of S^T, and the dQ^T column d
     const int qtr = warp / 4;                       // this thread's 16 of the step's 64 columns
     const int kj = k0 + row;
-    // this thread's two 16-byte chunks of the swizzled dS^T and P^T rows (queries qtr*16 .. +15)
+    // this thread's two 16-byte chunks of the swizzled dS^T row (queries qtr*16 .. +15)
     uint8_t* const ds_row = sm + Ly::DS + (row >> 3) * 1024 + (row & 7) * 128;
-    uint8_t* const pt_row = sm + Ly::PT + (row >> 3) * 1024 + (row & 7) * 128;
     const int ch0 = ((2 * qtr) ^ (row & 7)) * 16, ch1 = ((2 * qtr + 1) ^ (row & 7)) * 16;
     auto wait_all = [&](uint64_t* b, uint32_t parity) {
       bool ok = mbar_wait(b, parity, abort_flag, status, wait_ns);
@@ -533,28 +526,6 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       for (int j = 0; j < 16; ++j) red_add(p + (size_t)j * D, __uint_as_float(r[j]) * sigma);
     };
     uint32_t dqr[16];
-    // K^T into tensor memory, once: this thread's lane is column `row` of K, its 16 columns are
-    // keys 32 qtr .. 32 qtr + 31 as bf16 pairs (read from the 128-byte-swizzled K tile). The
-    // first accumulation reads it only after every warp's arrival on bar_p.
-    if (wait_all(bar_kv, 0)) {
-      const uint8_t* kc = sm + Ly::K + (row >> 6) * T128;  // the 64-column sub-tile of column row
-      const int cin = row & 63;
-      uint32_t kt[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        uint32_t pair = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int key = qtr * 32 + 2 * e + h;
-          const uint16_t x = *reinterpret_cast<const uint16_t*>(
-              kc + (key >> 3) * 1024 + (key & 7) * 128 + (((cin >> 3) ^ (key & 7)) << 4) + (cin & 7) * 2);
-          pair |= (uint32_t)x << (16 * h);
-        }
-        kt[e] = pair;
-      }
-      tmem_st16(t_kt + lane_off + qtr * 16, kt);
-      tmem_wait_st();
-    }
     for (int it = 0; it < nit; ++it) {
       if (!wait_all(bar_s, it & 1)) break;
       if (!wait_all(bar_st + it % kStF, (it / kStF) & 1)) break;  // lse, D of this step (visibility)
@@ -592,15 +563,14 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         tmem_ld16(t_dqt + lane_off + qtr * 16, dqr);  // dQ^T of step it-1, before step it's MMAs
         tmem_wait_ld();
       }
-      *reinterpret_cast<uint4*>(pt_row + ch0) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
-      *reinterpret_cast<uint4*>(pt_row + ch1) = make_uint4(wp[4], wp[5], wp[6], wp[7]);
-      *reinterpret_cast<uint4*>(pt_row + T128 + ch0) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
-      *reinterpret_cast<uint4*>(pt_row + T128 + ch1) = make_uint4(wq[4], wq[5], wq[6], wq[7]);
+      tmem_st8(t_pt + lane_off + qtr * 8, wp);
+      tmem_st8(t_pt + lane_off + 32 + qtr * 8, wq);
       *reinterpret_cast<uint4*>(ds_row + ch0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
       *reinterpret_cast<uint4*>(ds_row + ch1) = make_uint4(wh[4], wh[5], wh[6], wh[7]);
       *reinterpret_cast<uint4*>(ds_row + T128 + ch0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
       *reinterpret_cast<uint4*>(ds_row + T128 + ch1) = make_uint4(wl[4], wl[5], wl[6], wl[7]);
-      fence_async_smem();  // the P^T and dS^T stores, visible to the MMAs that read them
+      tmem_wait_st();
+      fence_async_smem();  // the dS^T stores, visible to the MMAs that read them
       tc_fence_before();
       __syncwarp();
       if ((tid % 32) == 0) mbar_arrive(bar_p);  // P^T, dS^T of step it are written
@@ -893,7 +863,6 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
                   (unsigned)((g.BH + kHeadGroup - 1) / kHeadGroup));
   if constexpr (D == 128) {
     if (fused) {
-      static_assert(LayFused<D>::BYTES + 1024 <= 232448, "the fused layout exceeds 227 KB per CTA");
       const int smem = padded_smem(LayFused<D>::BYTES);
       e = cudaFuncSetAttribute(attn_bwd_fused_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
