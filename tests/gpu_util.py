@@ -1,4 +1,7 @@
 """Helpers shared by the GPU parity tests: conversions and the acceptance rule."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -11,6 +14,20 @@ def np64(t):
 
 def store_of(dtype):
     return "bf16" if dtype == torch.bfloat16 else "f32"
+
+
+def bf16_ulps_above_rms(got, want):
+    """Largest distance, in bf16 units in the last place, between a bf16 result and the oracle
+    value rounded to bf16, over the elements whose oracle value exceeds the tensor's RMS (0 if
+    there are none). 0 means the correctly rounded result; 1, the neighbour of it. One bf16 ulp
+    at x is 2^(e - 7) with 2^e <= |x| < 2^(e + 1), the spacing of the 8-bit significand."""
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    big = np.abs(want) > rms
+    if not big.any():
+        return 0.0
+    w = torch.from_numpy(want[big]).to(torch.bfloat16).double().numpy()
+    ulp = np.ldexp(1.0, np.frexp(np.abs(w))[1] - 8)  # frexp: |w| = m 2^e with m in [0.5, 1)
+    return float((np.abs(got[big] - w) / ulp).max())
 
 
 def assert_close(got, want, dtype, what="", mode="scaled"):
@@ -33,6 +50,12 @@ def assert_close(got, want, dtype, what="", mode="scaled"):
         err = err / np.maximum(np.abs(want), rms)
     mx, mean = float(err.max()), float(err.mean())
     msg = f"{what} ({mode}): max {mx:.3g} mean {mean:.3g}"
+    log = os.environ.get("LH_ACCEPT_LOG")
+    if log:  # measurement of the margins, for choosing bounds; no effect on the verdict
+        with open(log, "a") as f:
+            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", ""), "what": what,
+                                "mode": mode, "dtype": str(dtype), "max": mx, "mean": mean,
+                                "ulps_above_rms": bf16_ulps_above_rms(got, want)}) + "\n")
     if dtype == torch.bfloat16:
         assert mx <= 2e-2 and mean <= 2e-3, msg
     else:
