@@ -58,9 +58,25 @@ def assert_close(got, want, dtype, what="", mode="scaled"):
                                 "ulps_above_rms": bf16_ulps_above_rms(got, want)}) + "\n")
     if dtype == torch.bfloat16:
         assert mx <= 2e-2 and mean <= 2e-3, msg
+        if is_bf16_valued(got):  # a result stored in bf16 (not an fp32 intermediate)
+            bound = ulp_bound(what)
+            ulps = bf16_ulps_above_rms(got, want)
+            assert ulps <= bound, f"{what}: {ulps:.2f} bf16 ulps from the rounded oracle (bound {bound})"
     else:
         assert mx <= 1e-4, msg
     return mx, mean
+
+
+def is_bf16_valued(x):
+    x = np.asarray(x, np.float64)
+    return bool(np.array_equal(torch.from_numpy(x).to(torch.bfloat16).double().numpy(), x))
+
+
+def ulp_bound(what):
+    """Largest distance in bf16 ulps, for elements above the RMS, between a bf16 layer output and
+    the correctly rounded oracle value: 1 (the rounded value or its neighbour) for O, dK and dV;
+    2 for dQ, whose fp32 sums arrive by atomic adds in an order that varies from run to run."""
+    return 2 if what.lower().startswith("dq") else 1
 
 
 def assert_pyramid(got, x, geo, dtype, what="pyramid"):
