@@ -159,6 +159,26 @@ int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, con
                 const float* o_sub, const float* lse, const void* do_sub, float* dq_sub,
                 float* dk_sub, float* dv_sub, void* ws, void* stream);
 
+/* Context parallelism: one rank's share of steps 5 and its backward, when a sequence is split
+ * over ranks by tokens ("Long Context Pre-Training with Lighthouse Attention", technical summary
+ * section 4: 1M tokens on 32 GPUs with context parallelism). `shape` is the rank's problem (its
+ * tokens and its shape->S subsequence rows). Its query rows are the global rows
+ * row0 .. row0 + S - 1 of the whole subsequence; k_seen and v_seen hold the global rows
+ * 0 .. row0 + S - 1 (row0 + S rows per (b,h), gathered from the ranks). The causal rule is on
+ * global rows.
+ *  - lh_attn_fwd_cp writes o_sub and lse for the rank's rows ([B,H,S,d], [B,H,S]).
+ *  - lh_attn_bwd_cp writes dq_sub for the rank's rows and dk_seen, dv_seen with row0 + S rows
+ *    per (b,h): the rank's part of dK_sub and dV_sub, which the caller sums over the ranks.
+ *    Like lh_attn_bwd without LH_DETERMINISTIC, dq_sub's fp32 sums arrive in varying order.
+ *  - bf16 and d = 128 only, row0 and S multiples of 128: otherwise LH_ERR_UNSUPPORTED.
+ *    row0 = 0 computes what lh_attn_fwd / lh_attn_bwd compute.
+ * Other arguments, layouts and errors as lh_attn_fwd / lh_attn_bwd. */
+int lh_attn_fwd_cp(const lh_shape* shape, int64_t row0, const void* q_sub, const void* k_seen,
+                   const void* v_seen, float* o_sub, float* lse, void* ws, void* stream);
+int lh_attn_bwd_cp(const lh_shape* shape, int64_t row0, const void* q_sub, const void* k_seen,
+                   const void* v_seen, const float* o_sub, const float* lse, const void* do_sub,
+                   float* dq_sub, float* dk_seen, float* dv_seen, void* ws, void* stream);
+
 /* Step 6 (deterministic scatter-back, section 2.C). o[t] = sum of o_sub[i] over the rows i of
  * t's stratum whose span covers t, coarsest first, no atomics. idx must be a valid selection
  * (rows of stratum s at s*m .. s*m+m-1, each cell at most once). o_sub is float [B,H,S,d]. */

@@ -61,6 +61,8 @@ def _load():
         "lh_gather": ([SP, P, P, P, P, P, P, P, P, P, P, P, P], I),
         "lh_attn_fwd": ([SP, P, P, P, P, P, P, P], I),
         "lh_attn_bwd": ([SP, P, P, P, P, P, P, P, P, P, P, P], I),
+        "lh_attn_fwd_cp": ([SP, ctypes.c_int64, P, P, P, P, P, P, P], I),
+        "lh_attn_bwd_cp": ([SP, ctypes.c_int64, P, P, P, P, P, P, P, P, P, P, P], I),
         "lh_scatter": ([SP, P, P, P, P], I),
         "lh_scatter_bwd": ([SP, P, P, P, P, P], I),
         "lh_gather_bwd": ([SP, P, P, P, P, P, P, P, P], I),
@@ -206,6 +208,18 @@ def lh_attn_bwd(shape, q_sub, k_sub, v_sub, o_sub, lse, do_sub, dq_sub, dk_sub, 
     _check(_lib.lh_attn_bwd(ctypes.byref(shape.c()), _ptr(q_sub), _ptr(k_sub), _ptr(v_sub),
                             _ptr(o_sub), _ptr(lse), _ptr(do_sub), _ptr(dq_sub), _ptr(dk_sub),
                             _ptr(dv_sub), _ptr(ws), _stream(stream)))
+
+
+def lh_attn_fwd_cp(shape, row0, q_sub, k_seen, v_seen, o_sub, lse, ws, stream=None):
+    _check(_lib.lh_attn_fwd_cp(ctypes.byref(shape.c()), row0, _ptr(q_sub), _ptr(k_seen), _ptr(v_seen),
+                               _ptr(o_sub), _ptr(lse), _ptr(ws), _stream(stream)))
+
+
+def lh_attn_bwd_cp(shape, row0, q_sub, k_seen, v_seen, o_sub, lse, do_sub, dq_sub, dk_seen, dv_seen,
+                   ws, stream=None):
+    _check(_lib.lh_attn_bwd_cp(ctypes.byref(shape.c()), row0, _ptr(q_sub), _ptr(k_seen), _ptr(v_seen),
+                               _ptr(o_sub), _ptr(lse), _ptr(do_sub), _ptr(dq_sub), _ptr(dk_seen),
+                               _ptr(dv_seen), _ptr(ws), _stream(stream)))
 
 
 def lh_scatter(shape, idx, o_sub, o, stream=None):

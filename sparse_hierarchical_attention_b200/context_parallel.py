@@ -140,3 +140,77 @@ class ContextParallelLayer:
         else:
             dk_sub, dv_sub = dk_seen, dv_seen
         return self.ops.gather_bwd(state, dq_sub, dk_sub, dv_sub)
+
+
+class GpuOps:
+    """One rank's stages on its GPU, every step a liblh kernel: the shard's pyramid, scores,
+    top-K, gather, scatter-back and their backward through the single-GPU entry points on the
+    shard's shape (N/W tokens, budget S/W), and the attention through lh_attn_fwd_cp /
+    lh_attn_bwd_cp, which take the rank's query rows at a global offset. bf16, d = 128."""
+
+    def __init__(self, shape, device="cuda"):
+        from . import _lib
+        self.lib, self.shape = _lib, shape
+        self.dev = torch.device(device)
+        sz = _lib.lh_validate(shape)
+        self.R = sz["R"]
+        self.ws = torch.zeros(_lib.lh_workspace_bytes(shape), dtype=torch.uint8, device=self.dev)
+
+    @staticmethod
+    def _dense(*ts):
+        for t in ts:  # the kernels read [B, H, rows, d] through raw pointers
+            if not t.is_contiguous():
+                raise ValueError("context-parallel operands must be contiguous [B, H, rows, d]")
+
+    def _e(self, rows, dtype=None):
+        s = self.shape
+        return torch.empty(s.B, s.H, rows, s.d, dtype=dtype or s.dtype, device=self.dev)
+
+    def local_fwd(self, q, k, v):
+        s, L = self.shape, self.lib
+        R = max(self.R, 1)
+        pq, pk, pv = self._e(R), self._e(R), self._e(R)
+        score = torch.empty(s.B, s.H, s.N + self.R, dtype=torch.float32, device=self.dev)
+        idx = torch.empty(s.B, s.H, s.S, dtype=torch.int32, device=self.dev)
+        L.lh_build_pyramid(s, q, k, v, pq, pk, pv, score, self.ws)
+        L.lh_select_topk(s, score, idx)
+        subs = [self._e(s.S) for _ in range(3)]
+        L.lh_gather(s, q, k, v, pq, pk, pv, idx, *subs, self.ws)
+        return (idx, *subs, idx)
+
+    def attn_fwd(self, q_sub, k_seen, v_seen, row0):
+        s = self.shape
+        self._dense(q_sub, k_seen, v_seen)
+        o_sub = self._e(s.S, torch.float32)
+        lse = torch.empty(s.B, s.H, s.S, dtype=torch.float32, device=self.dev)
+        self.lib.lh_attn_fwd_cp(s, row0, q_sub, k_seen, v_seen, o_sub, lse, self.ws)
+        return o_sub, lse
+
+    def scatter(self, idx, o_sub):
+        o = self._e(self.shape.N)
+        self.lib.lh_scatter(self.shape, idx, o_sub, o)
+        return o
+
+    def span_sums(self, idx, d_o):
+        do_sub = self._e(self.shape.S)
+        self.lib.lh_scatter_bwd(self.shape, idx, d_o, do_sub, self.ws)
+        return do_sub
+
+    def attn_bwd(self, q_sub, k_seen, v_seen, o_sub, lse, do_sub, row0):
+        s = self.shape
+        self._dense(q_sub, k_seen, v_seen, o_sub, lse, do_sub)
+        dq_sub = self._e(s.S, torch.float32)
+        dk_seen, dv_seen = (self._e(k_seen.shape[2], torch.float32) for _ in range(2))
+        self.lib.lh_attn_bwd_cp(s, row0, q_sub, k_seen, v_seen, o_sub, lse, do_sub, dq_sub, dk_seen,
+                                dv_seen, self.ws)
+        return dq_sub, dk_seen, dv_seen
+
+    def gather_bwd(self, idx, dq_sub, dk_sub, dv_sub):
+        out = [self._e(self.shape.N) for _ in range(3)]
+        self.lib.lh_gather_bwd(self.shape, idx, dq_sub, dk_sub.contiguous(), dv_sub.contiguous(), *out)
+        return tuple(out)
+
+    def check(self):
+        rc, flags = self.lib.lh_check(self.ws)
+        if rc:
+            raise self.lib.LighthouseError(f"device fault flags {flags:#x}")

@@ -322,6 +322,48 @@ int lh_attn_bwd(const lh_shape* shape, const void* q_sub, const void* k_sub, con
   return LH_OK;
 }
 
+namespace {
+// Shapes the context-parallel attention takes; fills the key rows per (b,h).
+int cp_check(const Geo& g, int64_t row0, int* kb0, int* Sk) {
+  if (row0 < 0) return LH_ERR_INVALID_ARG;
+  if (g.dtype != LH_BF16 || g.d != 128 || g.S % 128 || row0 % 128) return LH_ERR_UNSUPPORTED;
+  if (g.BH * (row0 + g.S) >= ((int64_t)1 << 31)) return LH_ERR_UNSUPPORTED;
+  *kb0 = (int)(row0 / 128);
+  *Sk = (int)(row0 + g.S);
+  return LH_OK;
+}
+}  // namespace
+
+int lh_attn_fwd_cp(const lh_shape* shape, int64_t row0, const void* q_sub, const void* k_seen,
+                   const void* v_seen, float* o_sub, float* lse, void* ws, void* stream) {
+  LH_CHECK_GEO(shape, g);
+  int kb0 = 0, Sk = 0;
+  const int rc = cp_check(g, row0, &kb0, &Sk);
+  if (rc != LH_OK) return rc;
+  LH_REQUIRE_PTR(q_sub); LH_REQUIRE_PTR(k_seen); LH_REQUIRE_PTR(v_seen);
+  LH_REQUIRE_PTR(o_sub); LH_REQUIRE_PTR(lse); LH_REQUIRE_PTR(ws);
+  LH_CUDA(launch_attn_fwd_tc_rows(g, kb0, Sk, q_sub, k_seen, v_seen, o_sub, lse, at<uint32_t>(ws, 0),
+                                  static_cast<cudaStream_t>(stream)));
+  return LH_OK;
+}
+
+int lh_attn_bwd_cp(const lh_shape* shape, int64_t row0, const void* q_sub, const void* k_seen,
+                   const void* v_seen, const float* o_sub, const float* lse, const void* do_sub,
+                   float* dq_sub, float* dk_seen, float* dv_seen, void* ws, void* stream) {
+  LH_CHECK_GEO(shape, g);
+  int kb0 = 0, Sk = 0;
+  const int rc = cp_check(g, row0, &kb0, &Sk);
+  if (rc != LH_OK) return rc;
+  LH_REQUIRE_PTR(q_sub); LH_REQUIRE_PTR(k_seen); LH_REQUIRE_PTR(v_seen); LH_REQUIRE_PTR(o_sub);
+  LH_REQUIRE_PTR(lse); LH_REQUIRE_PTR(do_sub); LH_REQUIRE_PTR(dq_sub); LH_REQUIRE_PTR(dk_seen);
+  LH_REQUIRE_PTR(dv_seen); LH_REQUIRE_PTR(ws);
+  const WsLayout w = ws_layout(g);
+  LH_CUDA(launch_attn_bwd_tc_rows(g, kb0, Sk, q_sub, k_seen, v_seen, o_sub, lse, do_sub, dq_sub, dk_seen,
+                                  dv_seen, at<float>(ws, w.delta), at<uint32_t>(ws, 0),
+                                  static_cast<cudaStream_t>(stream)));
+  return LH_OK;
+}
+
 int lh_scatter(const lh_shape* shape, const int32_t* idx, const float* o_sub, void* o,
                void* stream) {
   LH_CHECK_GEO(shape, g);

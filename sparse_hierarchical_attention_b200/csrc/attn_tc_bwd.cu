@@ -367,7 +367,8 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
                   const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                   const float* __restrict__ lse, const float* __restrict__ delta,
                   float* __restrict__ dQ, float* __restrict__ dK, float* __restrict__ dV, int S,
-                  int BH, float sigma, float scale_log2, uint32_t* status, uint64_t wait_ns) {
+                  int BH, int kb0, int Sk, float sigma, float scale_log2, uint32_t* status,
+                  uint64_t wait_ns) {
   static_assert(D == 128, "dQ^T = K^T dS^T takes M = D = 128 tensor-memory lanes");
   using Ly = LayFused<D>;
   constexpr int KB = Ly::KB;
@@ -390,9 +391,14 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   const int kb = blockIdx.y;  // low key blocks see the most queries: heaviest first in a group
   const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
   if (bh >= BH) return;  // the last group may be partial
-  const int g0 = bh * S;
-  const int k0 = kb * 128;
-  const int nit = (S - k0) / 64;  // 64-row query blocks starting at k0
+  // S query rows and Sk key rows per (b,h); the queries are the global rows 128 kb0 .. Sk - 1 of
+  // the keys' sequence (kb0 = 0, Sk = S on one GPU; a context-parallel rank owns a later slice)
+  const int g0 = bh * S;                   // first query row of this (b,h)
+  const int gk0 = bh * Sk;                 // first key row of this (b,h)
+  const int k0 = kb * 128;                 // first key of the block (global row)
+  const int qs = k0 > kb0 * 128 ? k0 : kb0 * 128;  // first query that sees the block (global)
+  const int ql0 = qs - kb0 * 128;          // ... as a row of this CTA's query rows
+  const int nit = (Sk - qs) / 64;          // 64-row query blocks from qs
 
   if (tid == 0) {
     for (int i = 0; i < kBars; ++i)
@@ -423,16 +429,16 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         uint64_t* b = bar_st + sg;
         mbar_expect_tx(b, 2 * KB * T64 + 512);
         for (int c = 0; c < KB; ++c) {
-          tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + k0 + it * 64, b);
-          tma_load_2d(sm + Ly::DO + sg * KB * T64 + c * T64, &tdo, c * 64, g0 + k0 + it * 64, b);
+          tma_load_2d(sm + Ly::Q + sg * KB * T64 + c * T64, &tq, c * 64, g0 + ql0 + it * 64, b);
+          tma_load_2d(sm + Ly::DO + sg * KB * T64 + c * T64, &tdo, c * 64, g0 + ql0 + it * 64, b);
         }
-        bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + k0 + it * 64, 256, b);
-        bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + k0 + it * 64, 256, b);
+        bulk_load(sm + Ly::VEC + sg * 512, lse + g0 + ql0 + it * 64, 256, b);
+        bulk_load(sm + Ly::VEC + sg * 512 + 256, delta + g0 + ql0 + it * 64, 256, b);
       };
       mbar_expect_tx(bar_kv, 2 * KB * T128);
       for (int c = 0; c < KB; ++c) {
-        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, g0 + k0, bar_kv);
-        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, g0 + k0, bar_kv);
+        tma_load_2d(sm + Ly::K + c * T128, &tk, c * 64, gk0 + k0, bar_kv);
+        tma_load_2d(sm + Ly::V + c * T128, &tv, c * 64, gk0 + k0, bar_kv);
       }
       int issued = 0;
       for (int it = 0; it < nit; ++it) {  // step it reuses the stage of step it - kStF
@@ -521,7 +527,7 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
     };
     // adds sigma * dQ^T[row][qtr*16 + j] of step `it` to dq_sub (query rows, column row)
     auto add_dq = [&](int it, const uint32_t (&r)[16]) {
-      float* p = dQ + (size_t)(g0 + k0 + it * 64 + qtr * 16) * D + row;
+      float* p = dQ + (size_t)(g0 + ql0 + it * 64 + qtr * 16) * D + row;
 #pragma unroll
       for (int j = 0; j < 16; ++j) red_add(p + (size_t)j * D, __uint_as_float(r[j]) * sigma);
     };
@@ -547,7 +553,7 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       if ((tid % 32) == 0) mbar_arrive(bar_sfree);  // S^T / dP^T may be overwritten
       const float4* lv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStF) * 512) + qtr * 4;
       const float4* dv4 = reinterpret_cast<const float4*>(sm + Ly::VEC + (it % kStF) * 512 + 256) + qtr * 4;
-      const int q0 = k0 + it * 64 + qtr * 16;
+      const int q0 = qs + it * 64 + qtr * 16;  // global query row of this thread's first column
       uint64_t p2[8], ds2[8];
       kv_step_elements(st, dpt, lv4, dv4, scale_log2, kj, q0, q0 < k0 + 128, p2, ds2);
       uint32_t wp[8], wq[8], wh[8], wl[8];
@@ -583,7 +589,7 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       tmem_ld16(t_dqt + lane_off + qtr * 16, dqr);
       tmem_wait_ld();
       add_dq(nit - 1, dqr);
-      store_dkdv<D>(dV + (size_t)(g0 + kj) * D, dK + (size_t)(g0 + kj) * D, t_dv, t_dk, lane_off, qtr, sigma);
+      store_dkdv<D>(dV + (size_t)(gk0 + kj) * D, dK + (size_t)(gk0 + kj) * D, t_dv, t_dk, lane_off, qtr, sigma);
     }
   }
   // every role has drained its own loads and MMAs: nothing still writes shared or tensor memory
@@ -867,7 +873,8 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
       e = cudaFuncSetAttribute(attn_bwd_fused_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       attn_bwd_fused_tc<D><<<grid, kThreads, smem, st>>>(k128, v128, q64, do64, lse, delta, dq, dk, dv,
-                                                          g.S, (int)g.BH, sigma, scale_log2, status, g.wait_ns);
+                                                          g.S, (int)g.BH, 0, g.S, sigma, scale_log2, status,
+                                                          g.wait_ns);
       return cudaGetLastError();
     }
   }
@@ -890,6 +897,33 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
 }
 
 }  // namespace
+
+cudaError_t launch_attn_bwd_tc_rows(const Geo& g, int kb0, int Sk, const void* qs, const void* ks,
+                                    const void* vs, const float* os, const float* lse,
+                                    const void* dos, float* dq, float* dk, float* dv, float* delta,
+                                    uint32_t* status, cudaStream_t st) {
+  if (g.d != 128) return cudaErrorNotSupported;  // the one-pass kernel takes d = 128
+  constexpr int D = 128;
+  const int64_t rows = g.BH * g.S, krows = g.BH * (int64_t)Sk;
+  CUtensorMap q64, do64, k128, v128;
+  if (!make_tmap_rows_box(&q64, qs, rows, D, 64) || !make_tmap_rows_box(&do64, dos, rows, D, 64) ||
+      !make_tmap_rows_box(&k128, ks, krows, D, 128) || !make_tmap_rows_box(&v128, vs, krows, D, 128))
+    return cudaErrorInvalidValue;
+  delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(os, (const __nv_bfloat16*)dos, delta, dq, rows, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const float sigma = 1.0f / sqrtf((float)D);
+  const float scale_log2 = sigma * kLog2e;
+  const dim3 grid((unsigned)(g.BH < kHeadGroup ? g.BH : kHeadGroup), (unsigned)(Sk / 128),
+                  (unsigned)((g.BH + kHeadGroup - 1) / kHeadGroup));
+  const int smem = padded_smem(LayFused<D>::BYTES);
+  e = cudaFuncSetAttribute(attn_bwd_fused_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_bwd_fused_tc<D><<<grid, kThreads, smem, st>>>(k128, v128, q64, do64, lse, delta, dq, dk, dv, g.S,
+                                                      (int)g.BH, kb0, Sk, sigma, scale_log2, status,
+                                                      g.wait_ns);
+  return cudaGetLastError();
+}
 
 bool attn_bwd_fused(const Geo& g) {
   return attn_tc_eligible(g) && g.d == 128 && !(g.flags & LH_DETERMINISTIC);

@@ -64,7 +64,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, float* __restrict__ O, float* __restrict__ lse,
-            int S, int BH, float scale_log2, uint32_t* status, uint64_t wait_ns) {
+            int S, int BH, int kb0, int Sk, float scale_log2, uint32_t* status, uint64_t wait_ns) {
   using Ly = Layout<D>;
   constexpr int KB = Ly::KB;
   constexpr int kStV = v_stages<D>();
@@ -84,12 +84,15 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   uint64_t* const bar_pv = bar + 18;
 
   const int tid = threadIdx.x, warp = tid / 32;
+  // S query rows and Sk key rows per (b,h); the queries are the global rows 128 kb0 .. of the
+  // keys' sequence (kb0 = 0, Sk = S on one GPU; a context-parallel rank owns a later slice)
   const int nqb = S / BM;
   const int qb = nqb - 1 - (int)blockIdx.y;  // heaviest tiles first within a head group
   const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
   if (bh >= BH) return;  // the last group may be partial
-  const int grow0 = bh * S;                  // first row of this (b,h) in the [BH*S, D] view
-  const int nkb = qb + 1;
+  const int grow0 = bh * S;                  // first query row of this (b,h) in the [BH*S, D] view
+  const int krow0 = bh * Sk;                 // first key row of this (b,h)
+  const int nkb = kb0 + qb + 1;              // key blocks up to the diagonal
 
   if (tid == 0) {
     for (int i = 0; i < kBars; ++i)
@@ -112,13 +115,13 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         uint64_t* b = bar_k + j % kStages;
         mbar_expect_tx(b, KB * TILE);
         for (int c = 0; c < KB; ++c)
-          tma_load_2d(sm + Ly::K + (j % kStages) * KB * TILE + c * TILE, &tk, c * 64, grow0 + j * BN, b);
+          tma_load_2d(sm + Ly::K + (j % kStages) * KB * TILE + c * TILE, &tk, c * 64, krow0 + j * BN, b);
       };
       auto load_v = [&](int j) {
         uint64_t* b = bar_v + j % kStV;
         mbar_expect_tx(b, KB * TILE);
         for (int c = 0; c < KB; ++c)
-          tma_load_2d(sm + Ly::V + (j % kStV) * KB * TILE + c * TILE, &tv, c * 64, grow0 + j * BN, b);
+          tma_load_2d(sm + Ly::V + (j % kStV) * KB * TILE + c * TILE, &tv, c * 64, krow0 + j * BN, b);
       };
       mbar_expect_tx(bar_q, KB * TILE);
       for (int c = 0; c < KB; ++c) tma_load_2d(sm + Ly::Q + c * TILE, &tq, c * 64, grow0 + qb * BM, bar_q);
@@ -228,7 +231,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       tc_fence_before();
       __syncwarp();
       if (ok && (tid % 32) == 0) mbar_arrive(bar_sfree + (j & 1));
-      if (j == qb) {  // diagonal block: key column > query row is invisible
+      if (j == kb0 + qb) {  // diagonal block: key column > query row is invisible
 #pragma unroll
         for (int e = 0; e < 64; ++e)
           if (half * 64 + e > row) s[e] = -INFINITY;
@@ -372,12 +375,12 @@ bool attn_tc_eligible(const Geo& g) {
          g.BH * (int64_t)g.S < (int64_t)1 << 31;
 }
 
-cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
-                               float* os, float* lse, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_attn_fwd_tc_rows(const Geo& g, int kb0, int Sk, const void* qs, const void* ks,
+                                    const void* vs, float* os, float* lse, uint32_t* status,
+                                    cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  const int64_t rows = g.BH * g.S;
-  if (!make_tmap_rows(&mq, qs, rows, g.d) || !make_tmap_rows(&mk, ks, rows, g.d) ||
-      !make_tmap_rows(&mv, vs, rows, g.d))
+  if (!make_tmap_rows(&mq, qs, g.BH * g.S, g.d) || !make_tmap_rows(&mk, ks, g.BH * Sk, g.d) ||
+      !make_tmap_rows(&mv, vs, g.BH * Sk, g.d))
     return cudaErrorInvalidValue;
   const float scale_log2 = (1.0f / sqrtf((float)g.d)) * 1.4426950408889634f;
   const unsigned gx = g.BH < kHeadGroup ? (unsigned)g.BH : (unsigned)kHeadGroup;
@@ -387,17 +390,22 @@ cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, con
     const int smem = Layout<128>::BYTES + 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status,
-                                                      g.wait_ns);
+      attn_fwd_tc<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, kb0, Sk, scale_log2,
+                                                      status, g.wait_ns);
   } else {
     // padded so that two CTAs never share an SM (each holds all 512 TMEM columns)
     const int smem = Layout<64>::BYTES + 1024 > 120 * 1024 ? Layout<64>::BYTES + 1024 : 120 * 1024;
     e = cudaFuncSetAttribute(attn_fwd_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, scale_log2, status,
-                                                     g.wait_ns);
+      attn_fwd_tc<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, g.S, (int)g.BH, kb0, Sk, scale_log2,
+                                                     status, g.wait_ns);
   }
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,
+                               float* os, float* lse, uint32_t* status, cudaStream_t st) {
+  return launch_attn_fwd_tc_rows(g, 0, g.S, qs, ks, vs, os, lse, status, st);
 }
 
 }  // namespace lh

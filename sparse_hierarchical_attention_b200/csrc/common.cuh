@@ -121,6 +121,15 @@ cudaError_t launch_attn_bwd_tc(const Geo& g, const void* qs, const void* ks, con
 cudaError_t attn_bwd_dispatch(const Geo& g, const void* qs, const void* ks, const void* vs,
                               const float* os, const float* lse, const void* dos, float* dq,
                               float* dk, float* dv, float* delta, uint32_t* status, cudaStream_t st);
+// Context-parallel forms: g.S query rows per (b,h) at global rows 128 kb0 .. of a key sequence of
+// Sk rows per (b,h) (Sk = 128 kb0 + g.S); bf16, S % 128 == 0. The backward's dk, dv have Sk rows.
+cudaError_t launch_attn_fwd_tc_rows(const Geo& g, int kb0, int Sk, const void* qs, const void* ks,
+                                    const void* vs, float* os, float* lse, uint32_t* status,
+                                    cudaStream_t st);
+cudaError_t launch_attn_bwd_tc_rows(const Geo& g, int kb0, int Sk, const void* qs, const void* ks,
+                                    const void* vs, const float* os, const float* lse,
+                                    const void* dos, float* dq, float* dk, float* dv, float* delta,
+                                    uint32_t* status, cudaStream_t st);
 int attn_fwd_launches(const Geo& g);
 int attn_bwd_launches(const Geo& g);
 cudaError_t launch_attn_fwd_simt(const Geo& g, const void* qs, const void* ks, const void* vs,
