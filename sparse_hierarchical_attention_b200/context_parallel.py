@@ -168,6 +168,7 @@ class GpuOps:
 
     def local_fwd(self, q, k, v):
         s, L = self.shape, self.lib
+        self._dense(q, k, v)
         R = max(self.R, 1)
         pq, pk, pv = self._e(R), self._e(R), self._e(R)
         score = torch.empty(s.B, s.H, s.N + self.R, dtype=torch.float32, device=self.dev)
@@ -192,6 +193,7 @@ class GpuOps:
         return o
 
     def span_sums(self, idx, d_o):
+        self._dense(d_o)
         do_sub = self._e(self.shape.S)
         self.lib.lh_scatter_bwd(self.shape, idx, d_o, do_sub, self.ws)
         return do_sub

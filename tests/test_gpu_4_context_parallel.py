@@ -34,7 +34,8 @@ def test_two_ranks_equal_the_whole_sequence(N, p, L, S):
     plans = [plan(N, p, L, S, W, r) for r in range(W)]
     ops = [GpuOps(Shape(B, H, N // W, d, p, L, S // W)) for _ in range(W)]
     tok = [slice(pl.tok0, pl.tok0 + pl.n_local) for pl in plans]
-    local = [ops[r].local_fwd(q[:, :, tok[r]], k[:, :, tok[r]], v[:, :, tok[r]]) for r in range(W)]
+    shard = lambda x, r: x[:, :, tok[r]].contiguous()  # what rank r holds  # noqa: E731
+    local = [ops[r].local_fwd(shard(q, r), shard(k, r), shard(v, r)) for r in range(W)]
     k_all = torch.cat([x[2] for x in local], dim=2)  # the all-gather
     v_all = torch.cat([x[3] for x in local], dim=2)
     outs, ctx = [], []
@@ -50,7 +51,7 @@ def test_two_ranks_equal_the_whole_sequence(N, p, L, S):
     dq_subs = []
     for r, pl in enumerate(plans):
         ks, vs, o_sub, lse = ctx[r]
-        do_sub = ops[r].span_sums(local[r][4], d_o[:, :, tok[r]])
+        do_sub = ops[r].span_sums(local[r][4], shard(d_o, r))
         dq_sub, dk_seen, dv_seen = ops[r].attn_bwd(local[r][1], ks, vs, o_sub, lse, do_sub, pl.row0)
         dq_subs.append(dq_sub)
         dk_sum[:, :, :pl.rows_seen] += dk_seen
