@@ -41,7 +41,13 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # capture, with the digest of the kernel sources the capture ran. `roofline.traffic` reports them
 # only while those sources are unchanged; after any change it is null and `traffic_stale` true.
 # (workload, stage) -> (bytes per call, source digest, how the bytes were obtained)
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("128k", "attn_bwd"): (
+        994826240, "9bd396dd863674f1",
+        "ncu dram__bytes_read.sum + dram__bytes_write.sum of the D and one-pass kernels at 16 of the "
+        "32 heads (two of four head groups), x2; reads grow in proportion to head groups (8 -> 16 "
+        "heads: 156 -> 312 MB), writes faster (51 -> 186 MB), so the write part is a lower bound"),
+}
 # the sources whose kernels run in each stage
 STAGE_SOURCES = {
     "pyramid_score": ["pool.cu"], "select": ["select.cu"], "gather": ["gather_scatter.cu"],
