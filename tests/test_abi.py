@@ -110,3 +110,16 @@ def test_flags_other_than_deterministic_are_rejected():
     c.flags = 2
     assert _lib._lib.lh_validate(ctypes.byref(c), None) == 1  # LH_ERR_INVALID_ARG
     assert lh.lh_validate(Shape(1, 2, 4096, 128, 4, 3, 256, deterministic=True))["C"] == 256
+
+
+@pytest.mark.parametrize("shape,row0,status", [
+    (Shape(1, 2, 4096, 128, 4, 3, 256 * 4, torch.float32), 0, 2),  # fp32: unsupported
+    (Shape(1, 2, 4096, 64, 4, 3, 256 * 4), 0, 2),                 # d = 64: unsupported
+    (Shape(1, 2, 4096, 128, 4, 3, 256 * 4), 64, 2),               # row0 not a multiple of 128
+    (Shape(1, 2, 4096, 128, 4, 3, 256 * 4), -128, 1),             # negative row0
+    (Shape(1, 2, 4096, 128, 4, 3, 256 * 5 + 4), 0, 2),            # S not a multiple of 128
+])
+def test_context_parallel_attention_rejects_before_any_launch(shape, row0, status):
+    c = shape.c()
+    assert _lib._lib.lh_attn_fwd_cp(ctypes.byref(c), row0, *([None] * 7)) == status
+    assert _lib._lib.lh_attn_bwd_cp(ctypes.byref(c), row0, *([None] * 11)) == status
