@@ -389,7 +389,9 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
 }
 
 // Levels A2+1..L-1 of one chunk from the level-A2 fp32 sums. Thread (xi, dd) walks the
-// chunk's level-A2 cells in order with one partial sum per coarser level.
+// chunk's level-A2 cells in order with one partial sum per coarser level; thread NX*D takes the
+// score maxima the same way. Each fetches the cells eight at a time (independent loads), since
+// the kernel is bound by load latency.
 template <typename E, int MODE>
 __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
   const int64_t bh = blockIdx.y, chunk = blockIdx.x;
@@ -432,48 +434,65 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
     __syncthreads();
   }
 
+  constexpr int kBatch = 8;
   if (tid < NX * D) {
     const int xi = tid / D, dd = tid % D;
+    const float* src = a.tmp + ((bh * n_a2 + first) * NX + xi) * D + dd;  // cell c at c NX D
     float acc[16];
     for (int u = 0; u < 16; ++u) acc[u] = 0.f;
-    for (int64_t c = 0; c < ncell; ++c) {
-      acc[0] += a.tmp[((bh * n_a2 + first + c) * NX + xi) * D + dd];
-      int64_t pw = 1;
-      for (int u = 0; u < nlev; ++u) {
-        pw *= p;
-        if ((c + 1) % pw != 0) break;
-        const int lvl = a.A2 + 1 + u;
-        const int64_t j = (first + c + 1) / pw - 1;
-        if constexpr (MODE == MODE_PYRAMID) {
-          if (a.do_pyr)
-            static_cast<E*>(a.px[xi])[(bh * a.R + (a.off[lvl] - a.N) + j) * D + dd] =
-                from_f32<E>(__fmul_rn(acc[u], a.inv[lvl]));
-        } else {
-          int64_t cells_per_chunk = ncell / pw;
-          const int r = cmap[cbase[u] + (int)(j - chunk * cells_per_chunk)];
-          if (r >= 0) static_cast<E*>(a.px[0])[(bh * a.S + r) * D + dd] = from_f32<E>(acc[u]);
+    for (int64_t c0 = 0; c0 < ncell; c0 += kBatch) {
+      float x[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) x[i] = c0 + i < ncell ? __ldg(src + (c0 + i) * NX * D) : 0.f;
+      for (int i = 0; i < kBatch && c0 + i < ncell; ++i) {
+        const int64_t c = c0 + i;
+        acc[0] += x[i];
+        int64_t pw = 1;
+        for (int u = 0; u < nlev; ++u) {
+          pw *= p;
+          if ((c + 1) % pw != 0) break;
+          const int lvl = a.A2 + 1 + u;
+          const int64_t j = (first + c + 1) / pw - 1;
+          if constexpr (MODE == MODE_PYRAMID) {
+            if (a.do_pyr)
+              static_cast<E*>(a.px[xi])[(bh * a.R + (a.off[lvl] - a.N) + j) * D + dd] =
+                  from_f32<E>(__fmul_rn(acc[u], a.inv[lvl]));
+          } else {
+            int64_t cells_per_chunk = ncell / pw;
+            const int r = cmap[cbase[u] + (int)(j - chunk * cells_per_chunk)];
+            if (r >= 0) static_cast<E*>(a.px[0])[(bh * a.S + r) * D + dd] = from_f32<E>(acc[u]);
+          }
+          if (u + 1 < nlev) acc[u + 1] += acc[u];
+          acc[u] = 0.f;
         }
-        if (u + 1 < nlev) acc[u + 1] += acc[u];
-        acc[u] = 0.f;
       }
     }
   }
-  if (MODE == MODE_PYRAMID && a.do_score && tid == 0) {
-    const float* mx = a.tmp + (int64_t)gridDim.y * n_a2 * NX * D;
+  if (MODE == MODE_PYRAMID && a.do_score && tid == NX * D) {
+    const float* mx = a.tmp + (int64_t)gridDim.y * n_a2 * NX * D + (bh * n_a2 + first) * 2;
     float q[16], k[16];
     for (int u = 0; u < 16; ++u) { q[u] = 0.f; k[u] = 0.f; }
-    for (int64_t c = 0; c < ncell; ++c) {
-      q[0] = fmaxf(q[0], mx[(bh * n_a2 + first + c) * 2 + 0]);
-      k[0] = fmaxf(k[0], mx[(bh * n_a2 + first + c) * 2 + 1]);
-      int64_t pw = 1;
-      for (int u = 0; u < nlev; ++u) {
-        pw *= p;
-        if ((c + 1) % pw != 0) break;
-        const int lvl = a.A2 + 1 + u;
-        const int64_t j = (first + c + 1) / pw - 1;
-        a.score[bh * (a.N + a.R) + a.off[lvl] + j] = __fadd_rn(q[u], k[u]);
-        if (u + 1 < nlev) { q[u + 1] = fmaxf(q[u + 1], q[u]); k[u + 1] = fmaxf(k[u + 1], k[u]); }
-        q[u] = 0.f; k[u] = 0.f;
+    for (int64_t c0 = 0; c0 < ncell; c0 += kBatch) {
+      float xq[kBatch], xk[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        xq[i] = c0 + i < ncell ? __ldg(mx + (c0 + i) * 2) : 0.f;
+        xk[i] = c0 + i < ncell ? __ldg(mx + (c0 + i) * 2 + 1) : 0.f;
+      }
+      for (int i = 0; i < kBatch && c0 + i < ncell; ++i) {
+        const int64_t c = c0 + i;
+        q[0] = fmaxf(q[0], xq[i]);
+        k[0] = fmaxf(k[0], xk[i]);
+        int64_t pw = 1;
+        for (int u = 0; u < nlev; ++u) {
+          pw *= p;
+          if ((c + 1) % pw != 0) break;
+          const int lvl = a.A2 + 1 + u;
+          const int64_t j = (first + c + 1) / pw - 1;
+          a.score[bh * (a.N + a.R) + a.off[lvl] + j] = __fadd_rn(q[u], k[u]);
+          if (u + 1 < nlev) { q[u + 1] = fmaxf(q[u + 1], q[u]); k[u + 1] = fmaxf(k[u + 1], k[u]); }
+          q[u] = 0.f; k[u] = 0.f;
+        }
       }
     }
   }
@@ -554,7 +573,7 @@ cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
   if (e != cudaSuccess || pl.A2 >= g.L - 1) return e;
   const int nx = MODE == MODE_PYRAMID ? 3 : 1;
   dim3 grid((unsigned)g.C, (unsigned)g.BH);
-  const int threads = ((nx * g.d + 31) / 32) * 32;
+  const int threads = ((nx * g.d + (MODE == MODE_PYRAMID ? 1 : 0) + 31) / 32) * 32;  // + the score thread
   // span sums: one map slot per cell of the levels above A2 inside a chunk
   size_t smem = 0;
   if (MODE == MODE_SPANSUM) {
