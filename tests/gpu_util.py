@@ -51,7 +51,7 @@ def assert_close(got, want, dtype, what="", mode="scaled"):
     mx, mean = float(err.max()), float(err.mean())
     msg = f"{what} ({mode}): max {mx:.3g} mean {mean:.3g}"
     log = os.environ.get("LH_ACCEPT_LOG")
-    if log:  # measurement of the margins, for choosing bounds; no effect on the verdict
+    if log:  # measurement of the margins, for choosing bounds; no effect on pass or fail
         with open(log, "a") as f:
             f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", ""), "what": what,
                                 "mode": mode, "dtype": str(dtype), "max": mx, "mean": mean,

@@ -28,7 +28,7 @@ def _bench():
 #              write dQ, dK, dV), plus the ids
 #   attention FLOPs: 2 B H S^2 d forward and 5 B H S^2 d backward (causal)
 # in GB (1e9 bytes) and GFLOP, rounded to the digits below. The table's forward total counts
-# O_sub in bf16; this build keeps O_sub in fp32, which adds B H S d (4 - 2) bytes to the scatter.
+# O_sub in bf16; the library keeps O_sub in fp32, which adds B H S d (4 - 2) bytes to the scatter.
 EXPECTED = {
     "32k": dict(fwd=0.79, bwd=0.65, attn_fwd=69, attn_bwd=172),
     "llama530m-98k": dict(fwd=1.11, bwd=0.89, attn_fwd=77, attn_bwd=193),
