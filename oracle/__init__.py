@@ -3,12 +3,12 @@
 Only the tests, the smoke check and the benchmark's CPU-baseline leg import this package.
 """
 from .lighthouse_ref import (Geometry, attn_bwd, attn_fwd, build_pyramid, gather, gather_bwd,
-                             layer_bwd, layer_fwd, pool_stored, round_to, row_norm_f32, scatter, scatter_bwd,
-                             score, select_topk)
+                             kv_head_of, layer_bwd, layer_fwd, pool_stored, round_to, row_norm_f32,
+                             scatter, scatter_bwd, score, select_topk)
 
 __all__ = ["Geometry", "attn_bwd", "attn_fwd", "build_pyramid", "gather", "gather_bwd",
-           "layer_bwd", "layer_fwd", "pool_stored", "round_to", "row_norm_f32", "scatter", "scatter_bwd", "score",
-           "select_topk"]
+           "kv_head_of", "layer_bwd", "layer_fwd", "pool_stored", "round_to", "row_norm_f32",
+           "scatter", "scatter_bwd", "score", "select_topk"]
 
 # The same operations under the C ABI's names (lh_<stage> -> lh_ref_<stage>), on host arrays.
 lh_ref_build_pyramid = build_pyramid

@@ -150,17 +150,29 @@ def row_norm_f32(x, g):
     return np.sqrt(acc[..., 0])
 
 
+def kv_head_of(H, Hkv):
+    """Grouped-query heads (a reading; the pages state none): with H query heads and Hkv
+    key/value heads, H = g Hkv, query head h uses key/value head h // g, so g consecutive query
+    heads share one. Hkv = H is the plain layer."""
+    if Hkv < 1 or H % Hkv:
+        raise ValueError("the query heads must split evenly over the key/value heads")
+    return np.arange(H) // (H // Hkv)
+
+
 def score(q, k, geo: Geometry, g):
-    """Rank score r for every row id: float32 [B,H,N+R]."""
+    """Rank score r for every row id: float32 [B,H,N+R]. k may have fewer heads than q
+    (grouped-query heads): query head h then scores with the norms of key head kv_head_of(h)."""
     B, H, N, _ = q.shape
+    Hk = k.shape[1]
     sq, sk = row_norm_f32(q, g), row_norm_f32(k, g)
     levels_q, levels_k = [sq], [sk]
     for _ in range(1, geo.L):
         sq = sq.reshape(B, H, -1, geo.p).max(axis=3)
-        sk = sk.reshape(B, H, -1, geo.p).max(axis=3)
+        sk = sk.reshape(B, Hk, -1, geo.p).max(axis=3)
         levels_q.append(sq)
         levels_k.append(sk)
-    r = [a + b for a, b in zip(levels_q, levels_k)]  # float32 sum per cell
+    hmap = kv_head_of(H, Hk)
+    r = [a + b[:, hmap] for a, b in zip(levels_q, levels_k)]  # float32 sum per cell
     return np.concatenate(r, axis=2).astype(np.float32)
 
 
@@ -371,6 +383,9 @@ def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
     idx may be given to force a selection (used for the dense recovery identity). store names
     the storage type of the stored intermediates: the pooled cells (and, in layer_bwd, the
     span sums dO_sub) are then the fp32 children sums of pool_stored rounded to it.
+    k and v may have fewer heads than q (kv_head_of): each tensor is pooled over its own heads,
+    every query head selects its own cells, and its subsequence takes the key and value rows
+    of its key/value head.
     Returns (O [B,H,N,d] float64, saved dict for layer_bwd).
     """
     geo.check()
@@ -382,15 +397,19 @@ def layer_fwd(q, k, v, geo: Geometry, g, idx=None, store=None):
     if idx is None:
         r = score(q, k, geo, g)
         idx = select_topk(r, geo)
-    qs, ks, vs = gather(q, pq, idx), gather(k, pk, idx), gather(v, pv, idx)
+    hmap = kv_head_of(q.shape[1], k.shape[1])
+    qs = gather(q, pq, idx)
+    ks, vs = gather(k[:, hmap], pk[:, hmap], idx), gather(v[:, hmap], pv[:, hmap], idx)
     os_, lse = attn_fwd(qs, ks, vs)  # O_sub is kept in fp32 by the layer: no storage rounding
     o = scatter(idx, os_, geo)
-    saved = dict(idx=idx, score=r, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, geo=geo, store=store)
+    saved = dict(idx=idx, score=r, qs=qs, ks=ks, vs=vs, os=os_, lse=lse, geo=geo, store=store,
+                 kv_heads=k.shape[1])
     return o, saved
 
 
 def layer_bwd(saved, d_o):
-    """Backward of the layer: returns (dQ, dK, dV) [B,H,N,d] float64."""
+    """Backward of the layer: returns (dQ [B,H,N,d], dK, dV [B,Hkv,N,d]) float64. A key/value
+    head's gradients are the sums of those reaching it from each of its query heads."""
     geo, idx, store = saved["geo"], saved["idx"], saved.get("store")
     if store is None:
         dos = scatter_bwd(idx, d_o, geo)
@@ -399,4 +418,10 @@ def layer_bwd(saved, d_o):
                                pool_stored(d_o, geo, store, mean=False)], axis=2)
         dos = np.take_along_axis(full, idx[..., None].astype(np.int64), axis=2)
     dqs, dks, dvs = attn_bwd(saved["qs"], saved["ks"], saved["vs"], saved["os"], saved["lse"], dos)
-    return gather_bwd(idx, dqs, geo), gather_bwd(idx, dks, geo), gather_bwd(idx, dvs, geo)
+    dq, dk, dv = gather_bwd(idx, dqs, geo), gather_bwd(idx, dks, geo), gather_bwd(idx, dvs, geo)
+    B, H, N, d = dq.shape
+    Hkv = saved.get("kv_heads", H)
+    kv_head_of(H, Hkv)  # the same validation as the forward
+    dk = dk.reshape(B, Hkv, H // Hkv, N, d).sum(axis=2)  # query heads j g .. j g + g - 1
+    dv = dv.reshape(B, Hkv, H // Hkv, N, d).sum(axis=2)
+    return dq, dk, dv

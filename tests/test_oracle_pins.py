@@ -105,6 +105,27 @@ def test_coarse_score_is_max_over_span(N, p, L, S):
                 assert r[0, h, geo.offsets[l] + j] == want
 
 
+@pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (64, 4, 3, 16), (27, 3, 3, 9)])
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (4, 1), (6, 3)])
+def test_grouped_heads_score_with_their_key_head(N, p, L, S, H, Hkv):
+    """Grouped-query heads: query head h ranks with its own q norms and the k norms of key head
+    h // (H / Hkv), each max-pooled over the cell's span, then summed (brute force)."""
+    geo = O.Geometry(N, p, L, S)
+    q, k = rand(1, H, N, 8, scale=2.0), rand(1, Hkv, N, 8)
+    r = O.score(q, k, geo, 4)
+    sq, sk = O.row_norm_f32(q, 4), O.row_norm_f32(k, 4)
+    for h in range(H):
+        hk = h // (H // Hkv)
+        for l in range(L):
+            w = p ** l
+            for j in range(N // w):
+                want = np.float32(sq[0, h, j * w:(j + 1) * w].max()) + \
+                    np.float32(sk[0, hk, j * w:(j + 1) * w].max())
+                assert r[0, h, geo.offsets[l] + j] == want
+    with pytest.raises(ValueError):
+        O.score(q, rand(1, 3, N, 8) if H == 4 else rand(1, 4, N, 8), geo, 4)
+
+
 # ---------------------------------------------------------------- selection (2.B, 2.C)
 def brute_select(r, geo):
     """Every stratum of G chunks: full sort of all its candidates by the total key, the k best
@@ -251,14 +272,16 @@ def by_definition_layer(q, k, v, geo, g):
     r = O.score(q, k, geo, g)
     idx = O.select_topk(r, geo)
     out = np.zeros((B, H, N, d))
-    for b, h in itertools.product(range(B), range(H)):
-        cells = [geo.decode(int(i)) for i in idx[b, h]]
+    for b, hq in itertools.product(range(B), range(H)):
+        hk = hq * k.shape[1] // H  # the key/value head of query head hq (grouped-query heads)
+        cells = [geo.decode(int(i)) for i in idx[b, hq]]
         cells = [(int(l), int(j)) for l, j in cells]
-        rng_local = np.random.default_rng(b * 31 + h)
+        rng_local = np.random.default_rng(b * 31 + hq)
         rng_local.shuffle(cells)  # the definition needs no particular order
 
         def mean_of(x, l, j):
             w = geo.p ** l
+            h = hq if x.shape[1] == H else hk
             return np.asarray(x[b, h, j * w:(j + 1) * w], np.float64).mean(axis=0)
 
         for (l, j) in cells:
@@ -270,7 +293,7 @@ def by_definition_layer(q, k, v, geo, g):
             wts = [math.exp(a - mx) for a in logits]
             z = sum(wts)
             oi = sum(w_ / z * mean_of(v, l2, j2) for w_, (l2, j2) in zip(wts, vis))
-            out[b, h, j * geo.p ** l:(j + 1) * geo.p ** l] += oi
+            out[b, hq, j * geo.p ** l:(j + 1) * geo.p ** l] += oi
     return out
 
 
@@ -280,6 +303,16 @@ def by_definition_layer(q, k, v, geo, g):
 def test_layer_equals_by_definition(N, p, L, S):
     geo = O.Geometry(N, p, L, S).check()
     q, k, v = (rand(1, 2, N, 8) for _ in range(3))
+    o, _ = O.layer_fwd(q, k, v, geo, 4)
+    np.testing.assert_allclose(o, by_definition_layer(q, k, v, geo, 4), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (27, 3, 3, 9), (16, 2, 3, 6)])
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (4, 1)])
+def test_grouped_heads_layer_equals_by_definition(N, p, L, S, H, Hkv):
+    geo = O.Geometry(N, p, L, S).check()
+    q = rand(1, H, N, 8)
+    k, v = (rand(1, Hkv, N, 8) for _ in range(2))
     o, _ = O.layer_fwd(q, k, v, geo, 4)
     np.testing.assert_allclose(o, by_definition_layer(q, k, v, geo, 4), rtol=1e-11, atol=1e-12)
 
@@ -346,13 +379,18 @@ def test_future_chunks_do_not_change_the_past(N, p, L, S):
 
 
 # ---------------------------------------------------------------- gradients (2.B)
-@pytest.mark.parametrize("N,p,L,S", [(16, 2, 3, 8), (32, 4, 2, 16), (27, 3, 3, 9), (8, 2, 1, 8),
-                                     (16, 2, 3, 6)])
-def test_gradients_finite_differences(N, p, L, S):
-    """Central differences in fp64 with the selection held fixed (it is piecewise constant)."""
+@pytest.mark.parametrize("N,p,L,S,H,Hkv", [(16, 2, 3, 8, 2, 2), (32, 4, 2, 16, 2, 2),
+                                            (27, 3, 3, 9, 2, 2), (8, 2, 1, 8, 2, 2),
+                                            (16, 2, 3, 6, 2, 2), (16, 2, 3, 8, 4, 2),
+                                            (16, 2, 3, 6, 3, 1)])
+def test_gradients_finite_differences(N, p, L, S, H, Hkv):
+    """Central differences in fp64 with the selection held fixed (it is piecewise constant).
+    With grouped-query heads (Hkv < H) a key/value element feeds every query head of its group,
+    so its difference quotient checks the sum over the group."""
     geo = O.Geometry(N, p, L, S).check()
-    B, H, d = 1, 2, 4
-    q, k, v = (rand(B, H, N, d).astype(np.float64) for _ in range(3))
+    B, d = 1, 4
+    q = rand(B, H, N, d).astype(np.float64)
+    k, v = (rand(B, Hkv, N, d).astype(np.float64) for _ in range(2))
     do = rand(B, H, N, d).astype(np.float64)
     o, saved = O.layer_fwd(q, k, v, geo, 4)
     idx = saved["idx"]
@@ -364,7 +402,7 @@ def test_gradients_finite_differences(N, p, L, S):
     eps = 1e-6
     for which, gr in enumerate(grads):
         num = np.zeros_like(gr)
-        for pos in itertools.product(range(B), range(H), range(N), range(d)):
+        for pos in itertools.product(*(range(n) for n in gr.shape)):
             args = [q.copy(), k.copy(), v.copy()]
             args[which][pos] += eps
             up = loss(*args)
