@@ -66,11 +66,19 @@ typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
  * dQ in one pass over the key blocks and adds the per-block dQ terms into dq_sub with fp32
  * atomic adds, whose order varies from run to run (so do the last bits of dQ). With
  * LH_DETERMINISTIC it runs a second pass for dQ instead (no atomics; slower). Everything else
- * is deterministic either way. */
+ * is deterministic either way.
+ * Hkv: key/value heads (grouped-query attention; the pages state no such model, this is a
+ * reading). 0 means Hkv = H. Otherwise H must be a multiple of Hkv: query head h then uses
+ * key/value head h / (H / Hkv). K, V, their pyramid levels and dK, dV have Hkv heads; Q, O,
+ * the scores, the selection, the subsequence (q_sub, k_sub, v_sub) and dQ have H: every
+ * query head selects its own cells, and its k_sub / v_sub rows come from its key/value head.
+ * A key/value head's dK and dV add the terms of its H / Hkv query heads, in ascending head
+ * order. */
 typedef struct {
   int B, H, N, d, p, L, S;
   int dtype; /* lh_dtype */
   int flags;
+  int Hkv;
 } lh_shape;
 
 /* Sizes derived from a shape (the pages' notation: p, L, N per level, budget S).
@@ -126,11 +134,13 @@ uint64_t lh_set_wait_limit_ns(uint64_t ns);
 /* Step 1+2 (pyramid, section 2.A; scores, section 2.B). Reads q, k, v [B,H,N,d]; writes the
  * pooled levels pq, pk, pv [B,H,R,d]. If `score` is non-NULL it also writes the rank score
  * r = max-pooled |q| + max-pooled |k| for every row id, float [B,H,N+R], in the same pass.
+ * With grouped heads (shape.Hkv < H) k, v, pk, pv have Hkv heads; a first pass pools them and
+ * leaves the key norms in the workspace, a second pools q and adds them to the scores.
  * pq/pk/pv may all be NULL to compute only the score (then v is not read). */
 int lh_build_pyramid(const lh_shape* shape, const void* q, const void* k, const void* v,
                      void* pq, void* pk, void* pv, float* score, void* ws, void* stream);
 
-/* Step 2 alone: the rank score float [B,H,N+R] from q, k [B,H,N,d]. */
+/* Step 2 alone: the rank score float [B,H,N+R] from q [B,H,N,d] and k [B,Hkv,N,d]. */
 int lh_score(const lh_shape* shape, const void* q, const void* k, float* score, void* ws,
              void* stream);
 
@@ -142,7 +152,8 @@ int lh_score(const lh_shape* shape, const void* q, const void* k, float* score, 
 int lh_select_topk(const lh_shape* shape, const float* score, int32_t* idx, void* stream);
 
 /* Step 4 (gather, section 2.C). x_sub[b,h,i] = row idx[b,h,i] of [x | px]. Any idx whose ids
- * are in range is accepted; out-of-range ids give zero rows and set status bit 1. */
+ * are in range is accepted; out-of-range ids give zero rows and set status bit 1. With grouped
+ * heads k_sub and v_sub rows of query head h come from key/value head h / (H / Hkv). */
 int lh_gather(const lh_shape* shape, const void* q, const void* k, const void* v,
               const void* pq, const void* pk, const void* pv, const int32_t* idx,
               void* q_sub, void* k_sub, void* v_sub, void* ws, void* stream);
@@ -190,7 +201,9 @@ int lh_scatter_bwd(const lh_shape* shape, const int32_t* idx, const void* d_o, v
                    void* ws, void* stream);
 
 /* Backward of steps 1+4: dx[t] = sum over rows i covering t of dx_sub[i] / p^level(i), for
- * x in q, k, v. dx_sub are float [B,H,S,d]; dq, dk, dv are [B,H,N,d] in shape.dtype. */
+ * x in q, k, v. dx_sub are float [B,H,S,d]; dq, dk, dv are [B,H,N,d] in shape.dtype. With
+ * grouped heads dk, dv are [B,Hkv,N,d]: each adds the terms of its query heads in ascending
+ * order, each head's from the coarsest level down, in one fp32 sum (two launches). */
 int lh_gather_bwd(const lh_shape* shape, const int32_t* idx, const float* dq_sub,
                   const float* dk_sub, const float* dv_sub, void* dq, void* dk, void* dv,
                   void* stream);
@@ -201,7 +214,7 @@ int lh_layer_fwd(const lh_shape* shape, const void* q, const void* k, const void
                  void* saved, void* ws, void* stream);
 
 /* The whole layer backward. Reads `saved` from lh_layer_fwd and d_o [B,H,N,d]; writes
- * dq, dk, dv [B,H,N,d]. */
+ * dq, dk, dv [B,H,N,d] (dk, dv [B,Hkv,N,d] with grouped heads). */
 int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void* dq, void* dk,
                  void* dv, void* ws, void* stream);
 

@@ -30,7 +30,7 @@ LH_DETERMINISTIC = 1
 
 
 class lh_shape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "N", "d", "p", "L", "S", "dtype", "flags")]
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "N", "d", "p", "L", "S", "dtype", "flags", "Hkv")]
 
 
 class lh_sizes(ctypes.Structure):
@@ -91,7 +91,9 @@ class Shape:
     """One layer call: N tokens, H heads, d = d_head, pooling p, L levels, S rows kept.
 
     deterministic: run the attention backward without atomics (LH_DETERMINISTIC), so that
-    dQ is bit-identical from run to run; slower at d = 128."""
+    dQ is bit-identical from run to run; slower at d = 128.
+    Hkv: key/value heads when they are fewer than H (grouped-query heads; 0 = H). Query head h
+    then uses key/value head h // (H // Hkv); K, V and their gradients have Hkv heads."""
 
     B: int
     H: int
@@ -102,10 +104,15 @@ class Shape:
     S: int
     dtype: torch.dtype = torch.bfloat16
     deterministic: bool = False
+    Hkv: int = 0
+
+    @property
+    def kv_heads(self):
+        return self.Hkv or self.H
 
     def c(self):
         return lh_shape(self.B, self.H, self.N, self.d, self.p, self.L, self.S, _DTYPES[self.dtype],
-                        LH_DETERMINISTIC if self.deterministic else 0)
+                        LH_DETERMINISTIC if self.deterministic else 0, self.Hkv)
 
 
 def _ptr(t):

@@ -26,11 +26,14 @@ int make_geo(const lh_shape* s, Geo& g) {
   g.B = s->B; g.H = s->H; g.N = s->N; g.d = s->d; g.p = s->p; g.L = s->L; g.S = s->S;
   g.dtype = s->dtype;
   g.flags = s->flags;
+  g.Hkv = s->Hkv ? s->Hkv : s->H;
   g.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   if (s->flags & ~LH_DETERMINISTIC) return LH_ERR_INVALID_ARG;
   if (g.B < 1 || g.H < 1 || g.N < 1 || g.d < 1 || g.p < 2 || g.L < 1 || g.S < 1)
     return LH_ERR_INVALID_ARG;
   if (g.dtype != LH_F32 && g.dtype != LH_BF16) return LH_ERR_INVALID_ARG;
+  if (g.Hkv < 1 || g.H % g.Hkv) return LH_ERR_INVALID_ARG;
+  g.grp = g.H / g.Hkv;
   if (g.L > 12 || g.p > 16) return LH_ERR_UNSUPPORTED;
   int64_t T = 1;
   for (int l = 1; l < g.L; ++l) {
@@ -57,6 +60,7 @@ int make_geo(const lh_shape* s, Geo& g) {
   }
   if (g.S < g.C || g.S > g.C * (g.M + 1)) return LH_ERR_INVALID_ARG;
   g.BH = (int64_t)g.B * g.H;
+  g.BHkv = (int64_t)g.B * g.Hkv;
   g.R = 0;
   int64_t nl = g.N;
   for (int l = 0; l < g.L; ++l) {
@@ -72,7 +76,9 @@ int make_geo(const lh_shape* s, Geo& g) {
   // shared-memory limits of the selection and spread kernels
   // shared-memory limits of the selection (a stratum's candidate keys, its winners and per-chunk
   // counts) and spread kernels; the key packs a cell's stratum-local index into 24 bits
-  if ((size_t)(g.G * g.M + g.k) * 8 + (size_t)g.G * 4 > 200 * 1024 || (size_t)(g.M + 1) * 4 > 200 * 1024)
+  // (the spread of grouped heads maps the cells of all grp query heads of a chunk at once)
+  if ((size_t)(g.G * g.M + g.k) * 8 + (size_t)g.G * 4 > 200 * 1024 ||
+      (size_t)(g.M + 1) * 4 * g.grp > 200 * 1024)
     return LH_ERR_UNSUPPORTED;
   if (g.G * g.T >= ((int64_t)1 << 24)) return LH_ERR_UNSUPPORTED;
   return LH_OK;
@@ -88,7 +94,7 @@ bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0
 // time)]. Forward: pq, pk, pv, score, pooling scratch. Backward: do_sub, delta, dq_sub,
 // dk_sub, dv_sub, span-sum scratch.
 struct WsLayout {
-  size_t status, pq, pk, pv, score, ptmp, fwd_end;
+  size_t status, pq, pk, pv, score, ptmp, kscore, fwd_end;
   size_t do_sub, delta, dq, dk, dv, stmp, bwd_end;
   size_t total;
 };
@@ -96,6 +102,7 @@ struct WsLayout {
 WsLayout ws_layout(const Geo& g) {
   WsLayout w{};
   const size_t pyr = align256((size_t)(g.BH * g.R * g.d) * g.esize);
+  const size_t pyr_kv = align256((size_t)(g.BHkv * g.R * g.d) * g.esize);
   const size_t sub = align256((size_t)(g.BH * g.S * g.d) * g.esize);
   const size_t sub32 = align256((size_t)(g.BH * g.S * g.d) * 4);
   const size_t row32 = align256((size_t)(g.BH * g.S) * 4);
@@ -103,10 +110,12 @@ WsLayout ws_layout(const Geo& g) {
   w.status = o; o += 256;
   const size_t base = o;
   w.pq = o; o += pyr;
-  w.pk = o; o += pyr;
-  w.pv = o; o += pyr;
+  w.pk = o; o += pyr_kv;
+  w.pv = o; o += pyr_kv;
   w.score = o; o += align256((size_t)(g.BH * (g.N + g.R)) * 4);
   w.ptmp = o; o += align256(pyramid_tmp_bytes(g));
+  w.kscore = o;  // grouped heads: the max-pooled key norms of every key/value head
+  if (g.grp > 1) o += align256((size_t)(g.BHkv * (g.N + g.R)) * 4);
   w.fwd_end = o;
   o = base;
   w.do_sub = o; o += sub;
@@ -163,6 +172,26 @@ cudaError_t attn_fwd(const Geo& g, const void* qs, const void* ks, const void* v
                      float* lse, uint32_t* status, cudaStream_t st) {
   if (attn_tc_eligible(g)) return launch_attn_fwd_tc(g, qs, ks, vs, os, lse, status, st);
   return launch_attn_fwd_simt(g, qs, ks, vs, os, lse, st);
+}
+
+// dQ, dK, dV from the fp32 sub-gradients: one spread of the three when every query head has its
+// own key/value head; with grouped heads dQ per query head, then dK and dV per key/value head
+// over its group's selections.
+cudaError_t spread_grads(const Geo& g, const int32_t* idx, const float* dqs, const float* dks,
+                         const float* dvs, void* dq, void* dk, void* dv, uint32_t* status,
+                         cudaStream_t st) {
+  if (g.grp == 1) {
+    const void* src[3] = {dqs, dks, dvs};
+    void* dst[3] = {dq, dk, dv};
+    return launch_spread(g, idx, 3, true, true, src, dst, status, st);
+  }
+  const void* src_q[1] = {dqs};
+  void* dst_q[1] = {dq};
+  cudaError_t e = launch_spread(g, idx, 1, true, true, src_q, dst_q, status, st);
+  if (e != cudaSuccess) return e;
+  const void* src_kv[2] = {dks, dvs};
+  void* dst_kv[2] = {dk, dv};
+  return launch_spread_group(g, idx, src_kv, dst_kv, status, st);
 }
 
 cudaError_t attn_bwd(const Geo& g, const void* qs, const void* ks, const void* vs,
@@ -224,10 +253,11 @@ size_t lh_saved_bytes(const lh_shape* shape) {
 
 int lh_launches(const lh_shape* shape, int* fwd, int* bwd) {
   LH_CHECK_GEO(shape, g);
-  // forward: pyramid (+coarse), select, gather, attention, scatter
+  // forward: pyramid (+coarse; a key/value pass first with grouped heads), select, gather,
+  // attention, scatter
   if (fwd) *fwd = pool_launches(g) + 1 + 1 + attn_fwd_launches(g) + 1;
-  // backward: span sums (+coarse), attention backward, gather backward
-  if (bwd) *bwd = span_sum_launches(g) + attn_bwd_launches(g) + 1;
+  // backward: span sums (+coarse), attention backward, gather backward (two with grouped heads)
+  if (bwd) *bwd = span_sum_launches(g) + attn_bwd_launches(g) + (g.grp > 1 ? 2 : 1);
   return LH_OK;
 }
 
@@ -271,7 +301,7 @@ int lh_build_pyramid(const lh_shape* shape, const void* q, const void* k, const 
   if (score && !aligned(score)) return LH_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(g);
   LH_CUDA(launch_pyramid(g, q, k, v, (pyr && g.R > 0) ? pq : nullptr, pk, pv, score,
-                         at<char>(ws, w.ptmp), static_cast<cudaStream_t>(stream)));
+                         at<char>(ws, w.ptmp), at<float>(ws, w.kscore), static_cast<cudaStream_t>(stream)));
   return LH_OK;
 }
 
@@ -390,9 +420,8 @@ int lh_gather_bwd(const lh_shape* shape, const int32_t* idx, const float* dq_sub
   LH_CHECK_GEO(shape, g);
   LH_REQUIRE_PTR(idx); LH_REQUIRE_PTR(dq_sub); LH_REQUIRE_PTR(dk_sub); LH_REQUIRE_PTR(dv_sub);
   LH_REQUIRE_PTR(dq); LH_REQUIRE_PTR(dk); LH_REQUIRE_PTR(dv);
-  const void* src[3] = {dq_sub, dk_sub, dv_sub};
-  void* dst[3] = {dq, dk, dv};
-  LH_CUDA(launch_spread(g, idx, 3, true, true, src, dst, nullptr, static_cast<cudaStream_t>(stream)));
+  LH_CUDA(spread_grads(g, idx, dq_sub, dk_sub, dv_sub, dq, dk, dv, nullptr,
+                       static_cast<cudaStream_t>(stream)));
   return LH_OK;
 }
 
@@ -410,7 +439,7 @@ int lh_layer_fwd(const lh_shape* shape, const void* q, const void* k, const void
   void* pv = g.R > 0 ? at<char>(ws, w.pv) : nullptr;
   float* score = at<float>(ws, w.score);
   int32_t* idx = at<int32_t>(saved, s.idx);
-  LH_CUDA(launch_pyramid(g, q, k, v, pq, pk, pv, score, at<char>(ws, w.ptmp), st));
+  LH_CUDA(launch_pyramid(g, q, k, v, pq, pk, pv, score, at<char>(ws, w.ptmp), at<float>(ws, w.kscore), st));
   LH_CUDA(launch_select(g, score, idx, st));
   LH_CUDA(launch_gather(g, q, k, v, pq, pk, pv, idx, at<char>(saved, s.qs), at<char>(saved, s.ks),
                         at<char>(saved, s.vs), status, st));
@@ -440,9 +469,7 @@ int lh_layer_bwd(const lh_shape* shape, const void* saved, const void* d_o, void
   LH_CUDA(attn_bwd(g, at<char>(saved, s.qs), at<char>(saved, s.ks), at<char>(saved, s.vs),
                    at<float>(saved, s.os), at<float>(saved, s.lse), dos, dqs, dks, dvs,
                    at<float>(ws, w.delta), status, st));
-  const void* src[3] = {dqs, dks, dvs};
-  void* dst[3] = {dq, dk, dv};
-  LH_CUDA(launch_spread(g, idx, 3, true, true, src, dst, status, st));
+  LH_CUDA(spread_grads(g, idx, dqs, dks, dvs, dq, dk, dv, status, st));
   return LH_OK;
 }
 

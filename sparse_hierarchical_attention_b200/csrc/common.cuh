@@ -19,6 +19,8 @@ constexpr uint32_t kFaultDrain = 4u;    // an abort-path wait for the CTA's own 
 struct Geo {
   int B, H, N, d, p, L, S, dtype;
   int flags;          // lh_shape.flags (LH_DETERMINISTIC)
+  int Hkv, grp;       // key/value heads and query heads per key/value head (grp = H / Hkv)
+  int64_t BHkv;       // B * Hkv
   uint64_t wait_ns;   // bound of every wait inside a kernel (lh_set_wait_limit_ns)
   int64_t BH, R, C, T, m, k, M;
   int64_t G;          // chunks per stratum (C / gcd(S, C))
@@ -94,8 +96,10 @@ int make_geo(const lh_shape* s, Geo& g);
 int fail_cuda(cudaError_t e);
 
 // ---- internal launchers (one per kernel family); all return cudaError_t of the launch ----
+// kscore: [B Hkv, N+R] scratch for the max-pooled key norms when heads are grouped (grp > 1)
 cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,
-                           void* pk, void* pv, float* score, void* tmp, cudaStream_t st);
+                           void* pk, void* pv, float* score, void* tmp, float* kscore,
+                           cudaStream_t st);
 size_t pyramid_tmp_bytes(const Geo& g);
 int pool_launches(const Geo& g);  // 1 or 2: the tile kernel, plus the coarse kernel if needed
 cudaError_t launch_select(const Geo& g, const float* score, int32_t* idx, cudaStream_t st);
@@ -105,6 +109,10 @@ cudaError_t launch_gather(const Geo& g, const void* q, const void* k, const void
 cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool from_f32,
                           bool scale_by_level, const void* const* src, void* const* dst,
                           uint32_t* status, cudaStream_t st);
+// gather backward of K and V with grouped heads: dX of key/value head j adds, per token, the
+// level-scaled fp32 rows of its query heads j grp .. j grp + grp - 1 (two tensors)
+cudaError_t launch_spread_group(const Geo& g, const int32_t* idx, const void* const* src,
+                                void* const* dst, uint32_t* status, cudaStream_t st);
 cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, void* do_sub,
                             void* tmp, uint32_t* status, cudaStream_t st);
 size_t span_sum_tmp_bytes(const Geo& g);

@@ -2,7 +2,8 @@
 // with Lighthouse Attention", technical summary 2.C), and the backward of the gather through
 // the pooling (technical summary 2.B: gradients reach Q, K, V through the gather).
 //
-// gather: one 16-byte lane per column slice, rows independent, a pure copy.
+// gather: one 16-byte lane per column slice, rows independent, a pure copy. With grouped heads
+//   the K and V rows of query head h come from its key/value head h / grp.
 // spread: one CTA per (b,h, chunk). The chunk's m row ids become a shared-memory map
 //   (level, cell in chunk) -> subsequence row. Each token then adds the rows that cover it,
 //   one per level at most, from the coarsest level down, sharing the partial sums of the
@@ -20,12 +21,13 @@ __global__ void __launch_bounds__(kThreads)
 gather_kernel(const E* __restrict__ q, const E* __restrict__ k, const E* __restrict__ v,
               const E* __restrict__ pq, const E* __restrict__ pk, const E* __restrict__ pv,
               const int32_t* __restrict__ idx, E* qs, E* ks, E* vs, int64_t BH, int64_t N,
-              int64_t R, int64_t S, uint32_t* status) {
+              int64_t R, int64_t S, int H, int grp, uint32_t* status) {
   constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, RPC = kThreads / LPR;
   const int col = threadIdx.x % LPR;
   const int64_t row = (int64_t)blockIdx.x * RPC + threadIdx.x / LPR;  // over BH*S
   if (row >= BH * S) return;
   const int64_t bh = row / S;
+  const int64_t bk = (bh / H) * (H / grp) + (bh % H) / grp;  // its key/value head
   const int64_t rid = idx[row];
   const E* src[3];
   E* dst[3] = {qs, ks, vs};
@@ -33,10 +35,10 @@ gather_kernel(const E* __restrict__ q, const E* __restrict__ k, const E* __restr
   if (!ok) {
     if (col == 0) raise_fault(status, kFaultIndex);
   } else if (rid < N) {
-    src[0] = q + (bh * N + rid) * D; src[1] = k + (bh * N + rid) * D; src[2] = v + (bh * N + rid) * D;
+    src[0] = q + (bh * N + rid) * D; src[1] = k + (bk * N + rid) * D; src[2] = v + (bk * N + rid) * D;
   } else {
-    const int64_t pr = bh * R + (rid - N);
-    src[0] = pq + pr * D; src[1] = pk + pr * D; src[2] = pv + pr * D;
+    src[0] = pq + (bh * R + (rid - N)) * D;
+    src[1] = pk + (bk * R + (rid - N)) * D; src[2] = pv + (bk * R + (rid - N)) * D;
   }
 #pragma unroll
   for (int xi = 0; xi < 3; ++xi) {
@@ -51,6 +53,7 @@ struct SpreadArgs {
   const int32_t* idx;
   uint32_t* status;
   int64_t N, R, S, T, m, G;  // m rows per stratum of G chunks
+  int H, Hkv, grp;           // heads (grouped-head spread)
   int64_t off[16];
   float inv[16];  // per-level weight: 1 (scatter) or fl32(1/p^l) (gather backward)
   int p, L, ntensor;
@@ -168,6 +171,73 @@ __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
   }
 }
 
+// Gather backward of K and V with grouped heads. One CTA per (b, key/value head, chunk). It maps
+// the chunk's rows for each of the head's grp query heads (as spread_kernel does for one), then
+// each stream takes tokens one at a time: for query head h of the group in ascending order, and
+// within it from the coarsest level down, it adds the covering row of that head, scaled by
+// 1/p^level, into one fp32 sum per element.
+template <typename E, typename SRC, int D>
+__global__ void __launch_bounds__(kThreads) spread_group_kernel(const SpreadArgs a) {
+  constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, STREAMS = kThreads / LPR;
+  extern __shared__ int cmap[];  // [grp][(level, cell in chunk)] -> subsequence row
+  const int tid = threadIdx.x, col = tid % LPR, stream = tid / LPR;
+  const int64_t bk = blockIdx.y, c = blockIdx.x;  // b Hkv + j, chunk
+  const int L = a.L, p = a.p, grp = a.grp;
+  const int64_t bh0 = (bk / a.Hkv) * (int64_t)a.H + (bk % a.Hkv) * grp;  // its first query head
+
+  int base[16], per[16];
+  int tot = 0;
+  {
+    int cells = 1;
+    for (int l = L - 1; l >= 0; --l) { per[l] = cells; cells *= p; }
+    for (int l = 0; l < L; ++l) { base[l] = tot; tot += per[l]; }
+  }
+  for (int i = tid; i < grp * tot; i += kThreads) cmap[i] = -1;
+  __syncthreads();
+  const int64_t st = c / a.G;  // this chunk's stratum
+  for (int hm = 0; hm < grp; ++hm) {
+    for (int64_t i = st * a.m + tid; i < (st + 1) * a.m; i += kThreads) {
+      const int64_t rid = a.idx[(bh0 + hm) * a.S + i];
+      int lvl = 0;
+      if (rid < 0 || rid >= a.N + a.R) { raise_fault(a.status, kFaultIndex); continue; }
+      for (int l = 1; l < L; ++l)
+        if (rid >= a.off[l]) lvl = l;
+      const int64_t in_stratum = rid - a.off[lvl] - st * a.G * per[lvl];
+      if (in_stratum < 0 || in_stratum >= a.G * per[lvl]) { raise_fault(a.status, kFaultIndex); continue; }
+      const int64_t local = rid - a.off[lvl] - c * per[lvl];
+      if (local < 0 || local >= per[lvl]) continue;  // a cell of another chunk of the stratum
+      cmap[hm * tot + base[lvl] + (int)local] = (int)i;
+    }
+  }
+  __syncthreads();
+
+  for (int xi = 0; xi < a.ntensor; ++xi) {
+    E* dst = static_cast<E*>(a.dst[xi]) + (bk * a.N + c * a.T) * D + col * VEC;
+    for (int64_t t = stream; t < a.T; t += STREAMS) {
+      float out[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) out[e] = 0.f;
+      for (int hm = 0; hm < grp; ++hm) {
+        const SRC* src = static_cast<const SRC*>(a.src[xi]) + (bh0 + hm) * a.S * D;
+        int64_t cell = t;
+        int cells_of[16];
+        for (int l = 0; l < L; ++l) { cells_of[l] = (int)cell; cell /= p; }
+        for (int l = L - 1; l >= 0; --l) {
+          const int r = cmap[hm * tot + base[l] + cells_of[l]];
+          if (r >= 0) {
+            float x[VEC];
+            load_row<E, SRC, D>(src, r, col, x);
+            const float w = a.inv[l];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(x[e], w));
+          }
+        }
+      }
+      stg16_stream(dst + t * D, Vec<E>::pack(out));
+    }
+  }
+}
+
 template <typename E, typename SRC>
 cudaError_t run_spread(const Geo& g, const SpreadArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)(g.M + 1) * sizeof(int);
@@ -194,7 +264,7 @@ cudaError_t launch_gather(const Geo& g, const void* q, const void* k, const void
 #define LH_GATHER(E, D)                                                                      \
   gather_kernel<E, D><<<grid, kThreads, 0, st>>>(                                            \
       (const E*)q, (const E*)k, (const E*)v, (const E*)pq, (const E*)pk, (const E*)pv, idx, \
-      (E*)qs, (E*)ks, (E*)vs, g.BH, g.N, g.R, g.S, status)
+      (E*)qs, (E*)ks, (E*)vs, g.BH, g.N, g.R, g.S, g.H, g.grp, status)
   if (g.dtype == LH_BF16) {
     if (g.d == 64) LH_GATHER(__nv_bfloat16, 64); else LH_GATHER(__nv_bfloat16, 128);
   } else {
@@ -221,6 +291,36 @@ cudaError_t launch_spread(const Geo& g, const int32_t* idx, int ntensor, bool sr
   if (g.dtype == LH_BF16)
     return src_f32 ? run_spread<__nv_bfloat16, float>(g, a, st) : run_spread<__nv_bfloat16, __nv_bfloat16>(g, a, st);
   return run_spread<float, float>(g, a, st);
+}
+
+cudaError_t launch_spread_group(const Geo& g, const int32_t* idx, const void* const* src,
+                                void* const* dst, uint32_t* status, cudaStream_t st) {
+  SpreadArgs a{};
+  for (int i = 0; i < 2; ++i) { a.src[i] = src[i]; a.dst[i] = dst[i]; }
+  a.idx = idx; a.status = status;
+  a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.G = g.G;
+  a.p = g.p; a.L = g.L; a.ntensor = 2;
+  a.H = g.H; a.Hkv = g.Hkv; a.grp = g.grp;
+  for (int l = 0; l < 16; ++l) {
+    a.off[l] = l < g.L ? g.off[l] : 0;
+    double pw = 1.0;
+    for (int q = 0; q < l; ++q) pw *= g.p;
+    a.inv[l] = (float)(1.0 / pw);
+  }
+  const size_t smem = (size_t)(g.M + 1) * g.grp * sizeof(int);
+  dim3 grid((unsigned)g.C, (unsigned)g.BHkv);
+  cudaError_t e;
+#define LH_SPREAD_GROUP(E, D)                                                                        \
+  e = cudaFuncSetAttribute(spread_group_kernel<E, float, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           (int)smem);                                                               \
+  if (e == cudaSuccess) spread_group_kernel<E, float, D><<<grid, kThreads, smem, st>>>(a)
+  if (g.dtype == LH_BF16) {
+    if (g.d == 64) { LH_SPREAD_GROUP(__nv_bfloat16, 64); } else { LH_SPREAD_GROUP(__nv_bfloat16, 128); }
+  } else {
+    if (g.d == 64) { LH_SPREAD_GROUP(float, 64); } else { LH_SPREAD_GROUP(float, 128); }
+  }
+#undef LH_SPREAD_GROUP
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace lh

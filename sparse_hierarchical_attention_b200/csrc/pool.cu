@@ -52,7 +52,23 @@ struct PoolArgs {
   int wdiv[8];        // W / p^l for l = 1..A: level-l cells per stream
   int p, L, W, A2, U;
   int do_pyr, do_score;
+  // Pyramid: the nx tensors streamed, and what the score of a cell is:
+  //   0: |x[0]| + |x[1]| (q, k: each query head has its own key head);
+  //   1: |x[0]| (grouped heads, key/value pass: the max-pooled key norms);
+  //   2: |x[0]| + partner row of the key head (grouped heads, query pass).
+  int nx, score_mode;
+  const float* partner;  // mode 2: [B Hkv, N+R] max-pooled key norms
+  int H, grp;            // mode 2: query heads per batch, query heads per key/value head
 };
+
+// Mode 2's partner row: the key/value head of query head bh (b H + h -> b Hkv + h / grp).
+__device__ inline const float* partner_row(const PoolArgs& a, int64_t bh) {
+  return a.partner + ((bh / a.H) * (a.H / a.grp) + (bh % a.H) / a.grp) * (a.N + a.R);
+}
+// A cell's score from the query-side and key-side maxima (see score_mode); rid its row id.
+__device__ inline float cell_score(const PoolArgs& a, const float* prow, float sq, float sk, int64_t rid) {
+  return a.score_mode == 0 ? __fadd_rn(sq, sk) : a.score_mode == 1 ? sq : __fadd_rn(sq, prow[rid]);
+}
 
 // fp32 l2 norm in that fixed order. Each lane of a row sums the squares of its 16-byte
 // group in ascending order (products rounded on their own) and leaves that partial in shared
@@ -120,8 +136,9 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
   const int64_t t_tile = (int64_t)blockIdx.x * tile;
   const int64_t tok0 = t_tile + (int64_t)s * W;
   const bool active = tok0 < a.N;
-  const int nx = MODE == MODE_PYRAMID ? (a.do_pyr ? 3 : 2) : 1;
+  const int nx = MODE == MODE_PYRAMID ? a.nx : 1;
   const int64_t NR = a.N + a.R;
+  const float* const prow = MODE == MODE_PYRAMID && a.score_mode == 2 ? partner_row(a, bh) : nullptr;
 
   // Span sums: map every selected cell of level <= A2 inside this tile to its subsequence row.
   // Map layout: level l occupies tile/p^l slots starting at moff(l).
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
     }
     const E* const X = static_cast<const E*>(a.x[xi]) + (bh * a.N + tok0) * D + col * VEC;
     E* const PX = static_cast<E*>(a.px[MODE == MODE_PYRAMID ? xi : 0]);
-    const bool norm_of = NORMS && a.do_score && xi < 2;  // Q and K rows feed the score
+    const bool norm_of = NORMS && a.do_score && xi < (a.score_mode == 0 ? 2 : 1);  // the scored rows
     // L2 prefetch ahead of the loads. The kernel waits mostly on load latency, and the rows a
     // warp holds in flight are capped by its registers (the span-sum kernel sits at the register
     // limit of 4 CTAs per SM). A bulk prefetch into L2 holds no registers: one lane of the group
@@ -287,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
       float* const lk = lev + (STREAMS + s) * 32;
       for (int r = col; r < W; r += LPR) {
         const float nq = tree_norm<LPR>(part + (s * 16 + r) * PSTR);
-        const float nk = tree_norm<LPR>(part + ((STREAMS + s) * 16 + r) * PSTR);
-        if (active) a.score[bh * NR + tok0 + r] = __fadd_rn(nq, nk);
+        const float nk = a.score_mode == 0 ? tree_norm<LPR>(part + ((STREAMS + s) * 16 + r) * PSTR) : 0.f;
+        if (active) a.score[bh * NR + tok0 + r] = cell_score(a, prow, nq, nk, tok0 + r);
         lq[r] = nq;
         lk[r] = nk;
       }
@@ -306,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
           }
           lq[base + n + c] = mq;
           lk[base + n + c] = mk;
-          if (active) a.score[bh * NR + a.off[l] + first + c] = __fadd_rn(mq, mk);
+          if (active) a.score[bh * NR + a.off[l] + first + c] = cell_score(a, prow, mq, mk, a.off[l] + first + c);
         }
         base += n;
         n = nc;
@@ -325,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
     const int lvl = A + u;
     const int nc = cells / p;
     pw *= p;
-    const int nitems = NX * nc * D;
+    const int nitems = nx * nc * D;
     float v[(NX * STREAMS * D + kThreads - 1) / kThreads];
     float vmax[2] = {0.f, 0.f};
     int n = 0;
@@ -363,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
       smax[1][tid] = vmax[1];
       const int64_t j = t_tile / pw + tid;
       if (MODE == MODE_PYRAMID && a.do_score && j * pw < a.N)
-        a.score[bh * NR + a.off[lvl] + j] = __fadd_rn(vmax[0], vmax[1]);
+        a.score[bh * NR + a.off[lvl] + j] = cell_score(a, prow, vmax[0], vmax[1], a.off[lvl] + j);
     }
     __syncthreads();
     cells = nc;
@@ -372,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, (ctas_per_sm<MODE, A>())) pool_tile_
   // Hand the level-A2 sums to the coarse kernel.
   if (a.A2 < a.L - 1) {
     const int64_t n_a2 = a.N / pw;  // cells of level A2 per (b,h)
-    for (int it = tid; it < NX * cells * D; it += kThreads) {
+    for (int it = tid; it < nx * cells * D; it += kThreads) {
       const int xi = it / (cells * D), rem = it % (cells * D), c = rem / D, dd = rem % D;
       const int64_t j = t_tile / pw + c;
       if (j < n_a2) a.tmp[((bh * n_a2 + j) * NX + xi) * D + dd] = stage[xi][c][dd];
@@ -435,7 +452,7 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
   }
 
   constexpr int kBatch = 8;
-  if (tid < NX * D) {
+  if (tid < (MODE == MODE_PYRAMID ? a.nx : 1) * D) {
     const int xi = tid / D, dd = tid % D;
     const float* src = a.tmp + ((bh * n_a2 + first) * NX + xi) * D + dd;  // cell c at c NX D
     float acc[16];
@@ -470,6 +487,7 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
   }
   if (MODE == MODE_PYRAMID && a.do_score && tid == NX * D) {
     const float* mx = a.tmp + (int64_t)gridDim.y * n_a2 * NX * D + (bh * n_a2 + first) * 2;
+    const float* const prow = a.score_mode == 2 ? partner_row(a, bh) : nullptr;
     float q[16], k[16];
     for (int u = 0; u < 16; ++u) { q[u] = 0.f; k[u] = 0.f; }
     for (int64_t c0 = 0; c0 < ncell; c0 += kBatch) {
@@ -489,7 +507,7 @@ __global__ void pool_coarse_kernel(const PoolArgs a, int D, int NX) {
           if ((c + 1) % pw != 0) break;
           const int lvl = a.A2 + 1 + u;
           const int64_t j = (first + c + 1) / pw - 1;
-          a.score[bh * (a.N + a.R) + a.off[lvl] + j] = __fadd_rn(q[u], k[u]);
+          a.score[bh * (a.N + a.R) + a.off[lvl] + j] = cell_score(a, prow, q[u], k[u], a.off[lvl] + j);
           if (u + 1 < nlev) { q[u + 1] = fmaxf(q[u + 1], q[u]); k[u + 1] = fmaxf(k[u + 1], k[u]); }
           q[u] = 0.f; k[u] = 0.f;
         }
@@ -549,8 +567,9 @@ cudaError_t launch_tile(const Plan& pl, const PoolArgs& a, int64_t BH, cudaStrea
   }
 }
 
+// heads: the (b,h) rows of the streamed tensors (B H, or B Hkv for the key/value pass)
 template <int MODE>
-cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
+cudaError_t run_pool(const Geo& g, PoolArgs& a, int64_t heads, cudaStream_t st) {
   const Plan pl = make_plan(g, MODE == MODE_SPANSUM ? kWMaxSpan : kWMaxPyr);
   a.N = g.N; a.R = g.R; a.S = g.S; a.T = g.T; a.m = g.m; a.C = g.C; a.G = g.G;
   a.p = g.p; a.L = g.L; a.W = pl.W; a.A2 = pl.A2; a.U = pl.U;
@@ -567,12 +586,12 @@ cudaError_t run_pool(const Geo& g, PoolArgs& a, cudaStream_t st) {
   cudaError_t e;
   const bool bf = g.dtype == LH_BF16;
   if (g.d == 64)
-    e = bf ? launch_tile<__nv_bfloat16, 64, MODE>(pl, a, g.BH, st) : launch_tile<float, 64, MODE>(pl, a, g.BH, st);
+    e = bf ? launch_tile<__nv_bfloat16, 64, MODE>(pl, a, heads, st) : launch_tile<float, 64, MODE>(pl, a, heads, st);
   else
-    e = bf ? launch_tile<__nv_bfloat16, 128, MODE>(pl, a, g.BH, st) : launch_tile<float, 128, MODE>(pl, a, g.BH, st);
+    e = bf ? launch_tile<__nv_bfloat16, 128, MODE>(pl, a, heads, st) : launch_tile<float, 128, MODE>(pl, a, heads, st);
   if (e != cudaSuccess || pl.A2 >= g.L - 1) return e;
   const int nx = MODE == MODE_PYRAMID ? 3 : 1;
-  dim3 grid((unsigned)g.C, (unsigned)g.BH);
+  dim3 grid((unsigned)g.C, (unsigned)heads);
   const int threads = ((nx * g.d + (MODE == MODE_PYRAMID ? 1 : 0) + 31) / 32) * 32;  // + the score thread
   // span sums: one map slot per cell of the levels above A2 inside a chunk
   size_t smem = 0;
@@ -598,20 +617,53 @@ size_t tmp_bytes(const Geo& g, int nx, int wmax) {
 }  // namespace
 
 size_t pyramid_tmp_bytes(const Geo& g) { return tmp_bytes(g, 3, kWMaxPyr); }
-int pool_launches(const Geo& g) { return make_plan(g, kWMaxPyr).A2 >= g.L - 1 ? 1 : 2; }
+int pool_launches(const Geo& g) {
+  return (make_plan(g, kWMaxPyr).A2 >= g.L - 1 ? 1 : 2) * (g.grp > 1 ? 2 : 1);
+}
 size_t span_sum_tmp_bytes(const Geo& g) { return tmp_bytes(g, 1, kWMaxSpan); }
 int span_sum_launches(const Geo& g) { return make_plan(g, kWMaxSpan).A2 >= g.L - 1 ? 1 : 2; }
 
 cudaError_t launch_pyramid(const Geo& g, const void* q, const void* k, const void* v, void* pq,
-                           void* pk, void* pv, float* score, void* tmp, cudaStream_t st) {
+                           void* pk, void* pv, float* score, void* tmp, float* kscore,
+                           cudaStream_t st) {
+  if (g.grp == 1) {  // q, k, v of each head in one pass; score = |q| + |k|
+    PoolArgs a{};
+    a.x[0] = q; a.x[1] = k; a.x[2] = v;
+    a.px[0] = pq; a.px[1] = pk; a.px[2] = pv;
+    a.score = score;
+    a.tmp = static_cast<float*>(tmp);
+    a.do_pyr = pq != nullptr;
+    a.do_score = score != nullptr;
+    a.nx = a.do_pyr ? 3 : 2;
+    a.score_mode = 0;
+    return run_pool<MODE_PYRAMID>(g, a, g.BH, st);
+  }
+  // Grouped heads: the key/value heads first (K and V pooled, the max-pooled |k| of every cell
+  // into kscore), then the query heads (Q pooled, score = |q| + the kscore row of the head's
+  // key/value head, the same fp32 sum as in one pass).
   PoolArgs a{};
-  a.x[0] = q; a.x[1] = k; a.x[2] = v;
-  a.px[0] = pq; a.px[1] = pk; a.px[2] = pv;
-  a.score = score;
+  a.x[0] = k; a.x[1] = v;
+  a.px[0] = pk; a.px[1] = pv;
+  a.score = score ? kscore : nullptr;
   a.tmp = static_cast<float*>(tmp);
   a.do_pyr = pq != nullptr;
   a.do_score = score != nullptr;
-  return run_pool<MODE_PYRAMID>(g, a, st);
+  a.nx = a.do_pyr ? 2 : 1;
+  a.score_mode = 1;
+  cudaError_t e = run_pool<MODE_PYRAMID>(g, a, g.BHkv, st);
+  if (e != cudaSuccess) return e;
+  PoolArgs b{};
+  b.x[0] = q;
+  b.px[0] = pq;
+  b.score = score;
+  b.tmp = static_cast<float*>(tmp);
+  b.do_pyr = pq != nullptr;
+  b.do_score = score != nullptr;
+  b.nx = 1;
+  b.score_mode = 2;
+  b.partner = kscore;
+  b.H = g.H; b.grp = g.grp;
+  return run_pool<MODE_PYRAMID>(g, b, g.BH, st);
 }
 
 cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, void* do_sub,
@@ -623,7 +675,7 @@ cudaError_t launch_span_sum(const Geo& g, const int32_t* idx, const void* d_o, v
   a.status = status;
   a.tmp = static_cast<float*>(tmp);
   a.do_pyr = 1;
-  return run_pool<MODE_SPANSUM>(g, a, st);
+  return run_pool<MODE_SPANSUM>(g, a, g.BH, st);
 }
 
 }  // namespace lh

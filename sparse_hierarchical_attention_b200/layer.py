@@ -48,9 +48,11 @@ class LighthouseLayer:
         return o, saved
 
     def backward(self, saved, d_o, dq=None, dk=None, dv=None):
+        s = self.shape
+        kv = (s.B, s.kv_heads, s.N, s.d)  # K and V have the key/value heads
         dq = torch.empty_like(d_o) if dq is None else dq
-        dk = torch.empty_like(d_o) if dk is None else dk
-        dv = torch.empty_like(d_o) if dv is None else dv
+        dk = torch.empty(kv, dtype=d_o.dtype, device=d_o.device) if dk is None else dk
+        dv = torch.empty(kv, dtype=d_o.dtype, device=d_o.device) if dv is None else dv
         _lib.lh_layer_bwd(self.shape, saved, d_o, dq, dk, dv, self.ws)
         return dq, dk, dv
 
@@ -77,7 +79,9 @@ class _Fn(torch.autograd.Function):
 class LighthouseAttention(torch.nn.Module):
     """Drop-in replacement of causal SDPA on [B, H, N, d] tensors during pre-training.
 
-    deterministic=True makes the backward bit-reproducible (no atomics; slower at d = 128)."""
+    k and v may have fewer heads than q (grouped-query heads, [B, Hkv, N, d] with H a multiple
+    of Hkv). deterministic=True makes the backward bit-reproducible (no atomics; slower at
+    d = 128)."""
 
     def __init__(self, p: int, L: int, S: int, deterministic: bool = False):
         super().__init__()
@@ -86,7 +90,9 @@ class LighthouseAttention(torch.nn.Module):
 
     def forward(self, q, k, v):
         B, H, N, d = q.shape
-        shape = Shape(B, H, N, d, self.p, self.L, self.S, q.dtype, self.deterministic)
+        Hkv = k.shape[1]
+        shape = Shape(B, H, N, d, self.p, self.L, self.S, q.dtype, self.deterministic,
+                      0 if Hkv == H else Hkv)
         key = (shape, q.device)
         if key not in self._layers:
             self._layers[key] = LighthouseLayer(shape, q.device)

@@ -40,6 +40,9 @@ def test_sizes(N, p, L, S, want):
     Shape(1, 2, 4096, 128, 4, 3, 256 * 22),  # m = 22 > M + 1 = 21
     Shape(0, 2, 4096, 128, 4, 3, 256),     # empty batch
     Shape(1, 2, 4096, 128, 1, 3, 256),     # p < 2
+    Shape(1, 6, 4096, 128, 4, 3, 256, Hkv=4),  # 6 query heads do not split over 4 key heads
+    Shape(1, 2, 4096, 128, 4, 3, 256, Hkv=4),  # more key/value heads than query heads
+    Shape(1, 2, 4096, 128, 4, 3, 256, Hkv=-1),
 ])
 def test_invalid_shapes(bad):
     assert _lib.lh_validate_status(bad) == 1
@@ -84,6 +87,20 @@ def test_workspace_and_saved_sizes_grow_with_shape():
     assert 0 < lh.lh_saved_bytes(a) < lh.lh_saved_bytes(b)
     offs = lh.lh_saved_offsets(a)
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+
+
+def test_grouped_heads_workspace_and_launches():
+    """Hkv = 0 is Hkv = H; with fewer key/value heads the key and value pyramids shrink and the
+    key-score scratch appears; the saved context (per query head) is unchanged."""
+    plain = Shape(1, 8, 4096, 128, 4, 3, 1024)
+    assert lh.lh_workspace_bytes(plain) == lh.lh_workspace_bytes(Shape(1, 8, 4096, 128, 4, 3, 1024, Hkv=8))
+    grouped = Shape(1, 8, 4096, 128, 4, 3, 1024, Hkv=2)
+    assert lh.lh_validate(grouped)["C"] == 256
+    assert lh.lh_saved_bytes(grouped) == lh.lh_saved_bytes(plain)
+    assert lh.lh_workspace_bytes(grouped) <= lh.lh_workspace_bytes(plain)  # the larger region wins
+    f1, b1 = lh.lh_launches(plain)
+    f2, b2 = lh.lh_launches(grouped)
+    assert f2 > f1 and b2 == b1 + 1  # a key/value pooling pass; a second spread
 
 
 def test_launch_plan():
