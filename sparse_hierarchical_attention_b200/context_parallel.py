@@ -146,7 +146,9 @@ class GpuOps:
     """One rank's stages on its GPU, every step a liblh kernel: the shard's pyramid, scores,
     top-K, gather, scatter-back and their backward through the single-GPU entry points on the
     shard's shape (N/W tokens, budget S/W), and the attention through lh_attn_fwd_cp /
-    lh_attn_bwd_cp, which take the rank's query rows at a global offset. bf16, d = 128."""
+    lh_attn_bwd_cp, which take the rank's query rows at a global offset. bf16, d = 128.
+    With grouped heads (shape.Hkv) k, v and their pyramid levels and gradients have the
+    key/value heads; the subsequence and the exchanges stay per query head."""
 
     def __init__(self, shape, device="cuda"):
         from . import _lib
@@ -162,15 +164,15 @@ class GpuOps:
             if not t.is_contiguous():
                 raise ValueError("context-parallel operands must be contiguous [B, H, rows, d]")
 
-    def _e(self, rows, dtype=None):
+    def _e(self, rows, dtype=None, heads=None):
         s = self.shape
-        return torch.empty(s.B, s.H, rows, s.d, dtype=dtype or s.dtype, device=self.dev)
+        return torch.empty(s.B, heads or s.H, rows, s.d, dtype=dtype or s.dtype, device=self.dev)
 
     def local_fwd(self, q, k, v):
         s, L = self.shape, self.lib
         self._dense(q, k, v)
-        R = max(self.R, 1)
-        pq, pk, pv = self._e(R), self._e(R), self._e(R)
+        R, kv = max(self.R, 1), s.kv_heads
+        pq, pk, pv = self._e(R), self._e(R, heads=kv), self._e(R, heads=kv)
         score = torch.empty(s.B, s.H, s.N + self.R, dtype=torch.float32, device=self.dev)
         idx = torch.empty(s.B, s.H, s.S, dtype=torch.int32, device=self.dev)
         L.lh_build_pyramid(s, q, k, v, pq, pk, pv, score, self.ws)
@@ -208,7 +210,8 @@ class GpuOps:
         return dq_sub, dk_seen, dv_seen
 
     def gather_bwd(self, idx, dq_sub, dk_sub, dv_sub):
-        out = [self._e(self.shape.N) for _ in range(3)]
+        kv = self.shape.kv_heads
+        out = [self._e(self.shape.N), self._e(self.shape.N, heads=kv), self._e(self.shape.N, heads=kv)]
         self.lib.lh_gather_bwd(self.shape, idx, dq_sub, dk_sub.contiguous(), dv_sub.contiguous(), *out)
         return tuple(out)
 

@@ -32,7 +32,10 @@ class OracleOps:
         O, geo = self.O, self.geo
         q, k, v = (x.numpy() for x in (q, k, v))
         idx = O.select_topk(O.score(q, k, geo, 4), geo)
-        subs = [O.gather(x, O.build_pyramid(x, geo), idx) for x in (q, k, v)]
+        hmap = O.kv_head_of(q.shape[1], k.shape[1])  # grouped heads: a query head's key head
+        subs = [O.gather(q, O.build_pyramid(q, geo), idx)]
+        subs += [O.gather(x[:, hmap], O.build_pyramid(x, geo)[:, hmap], idx) for x in (k, v)]
+        self.heads = (q.shape[1], k.shape[1])
         return (idx, *(torch.from_numpy(s) for s in subs), idx)
 
     @staticmethod
@@ -60,13 +63,19 @@ class OracleOps:
         return torch.from_numpy(dq[:, :, row0:]), torch.from_numpy(dk), torch.from_numpy(dv)
 
     def gather_bwd(self, idx, dq, dk, dv):
-        return tuple(torch.from_numpy(self.O.gather_bwd(idx, x.numpy(), self.geo)) for x in (dq, dk, dv))
+        H, Hkv = self.heads
+        out = [self.O.gather_bwd(idx, x.numpy(), self.geo) for x in (dq, dk, dv)]
+        for i in (1, 2):  # a key/value head sums its query heads' gradients
+            B, _, N, d = out[i].shape
+            out[i] = out[i].reshape(B, Hkv, H // Hkv, N, d).sum(axis=2)
+        return tuple(torch.from_numpy(x) for x in out)
 
 
-CASES = [  # (N, p, L, S): strata of G chunks, whole strata per rank
-    (64, 2, 3, 24),    # C = 16, G = 2: 8 strata of 3 rows
-    (128, 4, 3, 40),   # C = 8, G = 1: 8 chunks of 5 rows
-    (96, 2, 3, 26),    # C = 24, G = 12: 2 strata of 13 rows (one per rank)
+CASES = [  # (N, p, L, S, Hkv): strata of G chunks, whole strata per rank; H = 2
+    (64, 2, 3, 24, 2),    # C = 16, G = 2: 8 strata of 3 rows
+    (128, 4, 3, 40, 2),   # C = 8, G = 1: 8 chunks of 5 rows
+    (96, 2, 3, 26, 2),    # C = 24, G = 12: 2 strata of 13 rows (one per rank)
+    (64, 2, 3, 24, 1),    # both query heads on one key/value head
 ]
 
 
@@ -81,10 +90,11 @@ def _worker(rank, world, port, case, out):
     import oracle as O
     from sparse_hierarchical_attention_b200.context_parallel import ContextParallelLayer
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
-    N, p, L, S = case
+    N, p, L, S, Hkv = case
     B, H, d = 1, 2, 8
     g = torch.Generator().manual_seed(11)
-    q, k, v, d_o = (torch.randn(B, H, N, d, generator=g, dtype=torch.float64) for _ in range(4))
+    q, d_o = (torch.randn(B, H, N, d, generator=g, dtype=torch.float64) for _ in range(2))
+    k, v = (torch.randn(B, Hkv, N, d, generator=g, dtype=torch.float64) for _ in range(2))
     layer = ContextParallelLayer(N, p, L, S, OracleOps(N // world, p, L, S // world))
     pl = layer.plan
     sl = slice(pl.tok0, pl.tok0 + pl.n_local)

@@ -18,21 +18,23 @@ if torch.cuda.is_available():
 from gpu_util import assert_close, np64
 
 
-@pytest.mark.parametrize("N,p,L,S", [
-    (8192, 4, 5, 32 * 32),       # strata of one chunk: 16 per rank, 512 rows each
-    (16384, 2, 3, 4096 + 256),   # the p = 2, L = 3 ablation's strata (G = 16, 17 rows): 128 per rank
+@pytest.mark.parametrize("N,p,L,S,Hkv", [
+    (8192, 4, 5, 32 * 32, 2),       # strata of one chunk: 16 per rank, 512 rows each
+    (16384, 2, 3, 4096 + 256, 2),   # the p = 2, L = 3 ablation's strata (G = 16, 17 rows): 128 per rank
+    (8192, 4, 5, 32 * 32, 1),       # grouped heads: both query heads on one key/value head
 ])
-def test_two_ranks_equal_the_whole_sequence(N, p, L, S):
+def test_two_ranks_equal_the_whole_sequence(N, p, L, S, Hkv):
     W, B, H, d = 2, 1, 2, 128
     g = torch.Generator(device="cuda").manual_seed(N + S)
-    q, k, v, d_o = (torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(4))
-    whole = LighthouseLayer(Shape(B, H, N, d, p, L, S))
+    q, d_o = (torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn(B, Hkv, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(2))
+    whole = LighthouseLayer(Shape(B, H, N, d, p, L, S, Hkv=Hkv))
     o_ref, saved = whole.forward(q, k, v)
     dq_ref, dk_ref, dv_ref = whole.backward(saved, d_o)
     whole.check()
 
     plans = [plan(N, p, L, S, W, r) for r in range(W)]
-    ops = [GpuOps(Shape(B, H, N // W, d, p, L, S // W)) for _ in range(W)]
+    ops = [GpuOps(Shape(B, H, N // W, d, p, L, S // W, Hkv=Hkv)) for _ in range(W)]
     tok = [slice(pl.tok0, pl.tok0 + pl.n_local) for pl in plans]
     shard = lambda x, r: x[:, :, tok[r]].contiguous()  # what rank r holds  # noqa: E731
     local = [ops[r].local_fwd(shard(q, r), shard(k, r), shard(v, r)) for r in range(W)]
@@ -65,11 +67,13 @@ def test_two_ranks_equal_the_whole_sequence(N, p, L, S):
     grads = [torch.cat(x, dim=2) for x in grads]
 
     geo = O.Geometry(N, p, L, S).check()
-    h = (slice(0, 1), slice(1, 2))  # the oracle checks one head whole
-    wo, sv = O.layer_fwd(np64(q[h]), np64(k[h]), np64(v[h]), geo, 8, store="bf16")
+    # the oracle checks one head whole; a shared key/value head needs every query head of it
+    h = (slice(0, 1), slice(1, 2)) if Hkv == H else (slice(0, 1), slice(0, H))
+    hk = h if Hkv == H else (slice(0, 1), slice(0, Hkv))
+    wo, sv = O.layer_fwd(np64(q[h]), np64(k[hk]), np64(v[hk]), geo, 8, store="bf16")
     want = O.layer_bwd(sv, np64(d_o[h]))
-    for got, ref, w_, n in zip(grads, (dq_ref, dk_ref, dv_ref), want, ("dQ", "dK", "dV")):
-        assert_close(np64(got[h]), w_, torch.bfloat16, n)
+    for got, ref, w_, n, hh in zip(grads, (dq_ref, dk_ref, dv_ref), want, ("dQ", "dK", "dV"), (h, hk, hk)):
+        assert_close(np64(got[hh]), w_, torch.bfloat16, n)
         x, y = got.float(), ref.float()  # and the whole-sequence GPU layer, to rounding
         rms = y.pow(2).mean().sqrt()
         assert ((x - y).abs() / torch.maximum(y.abs(), rms)).max().item() <= 2.0 ** -6, n
