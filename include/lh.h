@@ -72,8 +72,8 @@ typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
  * key/value head h / (H / Hkv). K, V, their pyramid levels and dK, dV have Hkv heads; Q, O,
  * the scores, the selection, the subsequence (q_sub, k_sub, v_sub) and dQ have H: every
  * query head selects its own cells, and its k_sub / v_sub rows come from its key/value head.
- * A key/value head's dK and dV add the terms of its H / Hkv query heads, in ascending head
- * order. */
+ * A key/value head's dK and dV add the terms of its H / Hkv query heads (coarsest level
+ * first, ascending heads within a level). */
 typedef struct {
   int B, H, N, d, p, L, S;
   int dtype; /* lh_dtype */
@@ -202,8 +202,8 @@ int lh_scatter_bwd(const lh_shape* shape, const int32_t* idx, const void* d_o, v
 
 /* Backward of steps 1+4: dx[t] = sum over rows i covering t of dx_sub[i] / p^level(i), for
  * x in q, k, v. dx_sub are float [B,H,S,d]; dq, dk, dv are [B,H,N,d] in shape.dtype. With
- * grouped heads dk, dv are [B,Hkv,N,d]: each adds the terms of its query heads in ascending
- * order, each head's from the coarsest level down, in one fp32 sum (two launches). */
+ * grouped heads dk, dv are [B,Hkv,N,d]: each adds the terms of its query heads in one fp32
+ * sum, from the coarsest level down and within a level in ascending head order (two launches). */
 int lh_gather_bwd(const lh_shape* shape, const int32_t* idx, const float* dq_sub,
                   const float* dk_sub, const float* dv_sub, void* dq, void* dk, void* dv,
                   void* stream);

@@ -172,10 +172,11 @@ __global__ void __launch_bounds__(kThreads) spread_kernel(const SpreadArgs a) {
 }
 
 // Gather backward of K and V with grouped heads. One CTA per (b, key/value head, chunk). It maps
-// the chunk's rows for each of the head's grp query heads (as spread_kernel does for one), then
-// each stream takes tokens one at a time: for query head h of the group in ascending order, and
-// within it from the coarsest level down, it adds the covering row of that head, scaled by
-// 1/p^level, into one fp32 sum per element.
+// the chunk's rows for each of the head's grp query heads (as spread_kernel does for one). The
+// sums then take spread_kernel's top-down form, with the query heads inside each level: a stream
+// takes a group of p^A tokens, adds the level L-1..A rows of every query head (levels in
+// descending order, heads ascending within a level) once for the group, the level-1 rows once
+// per p tokens, then each token's level-0 rows. With grp = 1 this is spread_kernel's order.
 template <typename E, typename SRC, int D>
 __global__ void __launch_bounds__(kThreads) spread_group_kernel(const SpreadArgs a) {
   constexpr int VEC = 16 / sizeof(E), LPR = D / VEC, STREAMS = kThreads / LPR;
@@ -211,29 +212,49 @@ __global__ void __launch_bounds__(kThreads) spread_group_kernel(const SpreadArgs
   }
   __syncthreads();
 
+  const int A = L >= 3 ? 2 : L - 1;  // levels handled inside a group
+  const int G = A == 2 ? p * p : (A == 1 ? p : 1);
+  const int ngroups = (int)(a.T / G);
   for (int xi = 0; xi < a.ntensor; ++xi) {
+    const SRC* src0 = static_cast<const SRC*>(a.src[xi]) + bh0 * a.S * D;  // head hm at + hm S D
     E* dst = static_cast<E*>(a.dst[xi]) + (bk * a.N + c * a.T) * D + col * VEC;
-    for (int64_t t = stream; t < a.T; t += STREAMS) {
-      float out[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) out[e] = 0.f;
+    // adds the (level l, cell) row of every query head of the group, scaled by 1/p^l
+    auto add_level = [&](float (&acc)[VEC], int l, int cell) {
       for (int hm = 0; hm < grp; ++hm) {
-        const SRC* src = static_cast<const SRC*>(a.src[xi]) + (bh0 + hm) * a.S * D;
-        int64_t cell = t;
-        int cells_of[16];
-        for (int l = 0; l < L; ++l) { cells_of[l] = (int)cell; cell /= p; }
-        for (int l = L - 1; l >= 0; --l) {
-          const int r = cmap[hm * tot + base[l] + cells_of[l]];
-          if (r >= 0) {
-            float x[VEC];
-            load_row<E, SRC, D>(src, r, col, x);
-            const float w = a.inv[l];
+        const int r = cmap[hm * tot + base[l] + cell];
+        if (r >= 0) {
+          float x[VEC];
+          load_row<E, SRC, D>(src0 + (int64_t)hm * a.S * D, r, col, x);
+          const float w = a.inv[l];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(x[e], w));
-          }
+          for (int e = 0; e < VEC; ++e) acc[e] = __fadd_rn(acc[e], __fmul_rn(x[e], w));
         }
       }
-      stg16_stream(dst + t * D, Vec<E>::pack(out));
+    };
+    for (int g = stream; g < ngroups; g += STREAMS) {
+      float coarse[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) coarse[e] = 0.f;
+      int cells[16];
+      cells[A] = g;
+      for (int l = A + 1; l < L; ++l) cells[l] = cells[l - 1] / p;
+      for (int l = L - 1; l >= A; --l) add_level(coarse, l, cells[l]);
+      const int n0 = A >= 1 ? p : 1;  // tokens per level-1 cell (per token with A = 1)
+      for (int c1 = 0; c1 < (A == 2 ? p : 1); ++c1) {
+        float part[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) part[e] = coarse[e];
+        if (A == 2) add_level(part, 1, g * p + c1);
+        const int t0 = A == 2 ? (g * p + c1) * p : g * G;
+        for (int c0 = 0; c0 < (A == 0 ? 1 : n0); ++c0) {
+          const int t = t0 + c0;
+          float out[VEC];
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) out[e] = part[e];
+          if (A >= 1) add_level(out, 0, t);  // with L = 1 the token is the coarsest level, in `coarse`
+          stg16_stream(dst + (int64_t)t * D, Vec<E>::pack(out));
+        }
+      }
     }
   }
 }
