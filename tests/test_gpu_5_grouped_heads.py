@@ -175,3 +175,21 @@ def test_autograd_module_takes_fewer_key_heads():
     o.float().sum().backward()
     assert o.shape == q.shape and k.grad.shape == k.shape and v.grad.shape == v.shape
     assert torch.isfinite(k.grad.float()).all() and torch.isfinite(q.grad.float()).all()
+
+
+def test_grouped_bad_ids_are_flagged_not_faulted():
+    """A corrupted selection reaching the grouped backward (span sums, the dQ spread and the
+    key/value group spread) sets status bit 1 instead of faulting."""
+    B, H, Hkv, N, d, p, L, S = 1, 4, 2, 1024, 64, 4, 3, 256
+    shape = Shape(B, H, N, d, p, L, S, torch.bfloat16, Hkv=Hkv)
+    q, k, v = heads(B, H, Hkv, N, d, torch.bfloat16, seed=5)
+    layer = LighthouseLayer(shape)
+    o, saved = layer.forward(q, k, v)
+    layer.check()
+    idx = saved_views(shape, saved)["idx"]
+    idx[0, 3, 5] = N + 10_000_000  # beyond the pyramid
+    idx[0, 1, 9] = -3
+    layer.backward(saved, torch.randn_like(q))
+    rc, flags = lh.lh_check(layer.ws)
+    assert rc != 0 and flags & 1
+    assert lh.lh_check(layer.ws) == (0, 0)  # cleared by the read
