@@ -3,7 +3,9 @@
 // MODE_PYRAMID: the symmetric average-pooling pyramid over Q, K, V and the l2 rank score of
 //   every cell, in one pass over the inputs ("Long Context Pre-Training with Lighthouse
 //   Attention", technical summary 2.A and 2.B; the Nous Research article's four-stage
-//   paragraph: Theta(N) pyramid, two scalar scores per cell, max-pooled upward).
+//   paragraph: Theta(N) pyramid, two scalar scores per cell, max-pooled upward). With grouped
+//   query heads (fewer key/value heads) it takes two passes: K and V over their heads, leaving
+//   the max-pooled key norms in scratch, then Q, whose scores add its key head's norms.
 // MODE_SPANSUM: dO_sub[i] = sum of dO over span(i) for the selected cells only, the backward
 //   of the scatter-back (technical summary 2.B: gradients flow through scatter-back).
 //
