@@ -62,11 +62,11 @@ typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
 /* One layer call. Names follow the pages: N tokens, H heads, d = d_head, pooling factor p,
  * L levels, S = subsequence length (the top-K budget plus the kept coarsest cells).
  * The softmax scale is fixed to 1/sqrt(d).
- * flags: 0 or LH_DETERMINISTIC. At d = 128 the default attention backward computes dK, dV and
- * dQ in one pass over the key blocks and adds the per-block dQ terms into dq_sub with fp32
- * atomic adds, whose order varies from run to run (so do the last bits of dQ). With
- * LH_DETERMINISTIC it runs a second pass for dQ instead (no atomics; slower). Everything else
- * is deterministic either way.
+ * flags: 0 or LH_DETERMINISTIC. The default attention backward computes dK, dV and dQ in one
+ * pass over the key blocks and adds the per-block dQ terms into dq_sub with fp32 reductions
+ * (atomic adds at d = 128, copy-engine tensor reductions at d = 64), whose order varies from
+ * run to run (so do the last bits of dQ). With LH_DETERMINISTIC it runs a second pass for dQ
+ * instead (no atomics; slower). Everything else is deterministic either way.
  * Hkv: key/value heads (grouped-query attention; the pages state no such model, this is a
  * reading). 0 means Hkv = H. Otherwise H must be a multiple of Hkv: query head h then uses
  * key/value head h / (H / Hkv). K, V, their pyramid levels and dK, dV have Hkv heads; Q, O,

@@ -5,8 +5,9 @@
 // dK_j = s sum_i dS_ij Q_i, with s = 1/sqrt(d).
 //
 // Two ways to run it:
-//   fused (d = 128, the default): one CTA per 128-key block steps through the 64-row query blocks
-//     that can see the keys:
+//   fused (the default; the d = 64 form, with 128-row query blocks and dQ added by the copy
+//     engine, is described above its kernel below): at d = 128 one CTA per 128-key block steps
+//     through the 64-row query blocks that can see the keys:
 //       S^T = K Q^T and dP^T = V dO^T;
 //       P^T = exp2(S^T c - lse2) and dS^T = P^T (dP^T - D) in fp32 registers;
 //       dV += P^T dO and dK += dS^T Q (accumulated in tensor memory over the whole block), and
@@ -17,7 +18,7 @@
 //     the MN-major B operand of dQ^T; K^T is the CTA's K tile read MN-major. So each step's S and
 //     dP are computed once for all three gradients. dV and dK are deterministic; the order in
 //     which the key blocks' dQ terms reach a dq_sub row varies from run to run.
-//   deterministic (LH_DETERMINISTIC, and every d = 64 call): two kernels without atomics:
+//   deterministic (LH_DETERMINISTIC): two kernels without atomics:
 //     dkdv: the fused kernel's dV/dK part, with dS^T in tensor memory;
 //     dq:   one CTA per 128-query block steps through the 64-row key blocks it sees:
 //           S = Q K^T and dP = dO V^T, dS as above, dQ += dS K (dS from tensor memory).
@@ -50,6 +51,8 @@
 namespace lh {
 
 bool make_tmap_rows_box(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows);
+// fp32 [rows][D] with 128-byte-swizzled boxes of 32 columns x box_rows rows (reductions into dq_sub)
+bool make_tmap_f32_box(CUtensorMap* map, const void* base, int64_t rows, int D, int box_rows);
 
 namespace {
 
@@ -599,6 +602,378 @@ attn_bwd_fused_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
+// P^T of one thread's 16 queries for its key kj: exp2(S^T c - lse log2 e), zero where the key
+// comes after the query (only on steps that reach the diagonal). Query pairs, lower in the low lane.
+__device__ inline void p_elements(const uint32_t (&st)[16], const float* lse, float scale_log2, int kj,
+                                  int q0, bool diag, uint64_t (&p2)[8]) {
+  const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4) {
+    const float4 lv = reinterpret_cast<const float4*>(lse)[c4];
+    const uint64_t nla[2] = {f2_pack(-(lv.x * kLog2e), -(lv.y * kLog2e)),
+                             f2_pack(-(lv.z * kLog2e), -(lv.w * kLog2e))};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = c4 * 2 + e;
+      float a0, a1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(st[2 * h]), __uint_as_float(st[2 * h + 1])), c2, nla[e]), a0, a1);
+      p2[h] = f2_pack(ex2(a0), ex2(a1));
+    }
+  }
+  if (diag) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float x0, x1;
+      f2_unpack(p2[h], x0, x1);
+      if (kj > q0 + 2 * h) x0 = 0.f;
+      if (kj > q0 + 2 * h + 1) x1 = 0.f;
+      p2[h] = f2_pack(x0, x1);
+    }
+  }
+}
+
+// dS^T = P^T (dP^T - D) for the same 16 queries, zero where the key comes after the query.
+__device__ inline void ds_elements(const uint64_t (&p2)[8], const uint32_t (&dpt)[16], const float* dlt,
+                                   int kj, int q0, bool diag, uint64_t (&ds2)[8]) {
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4) {
+    const float4 dv = reinterpret_cast<const float4*>(dlt)[c4];
+    const uint64_t da[2] = {f2_pack(dv.x, dv.y), f2_pack(dv.z, dv.w)};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = c4 * 2 + e;
+      ds2[h] = f2_mul(p2[h], f2_sub(f2_pack(__uint_as_float(dpt[2 * h]), __uint_as_float(dpt[2 * h + 1])), da[e]));
+    }
+  }
+  if (diag) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float y0, y1;
+      f2_unpack(ds2[h], y0, y1);
+      if (kj > q0 + 2 * h) y0 = 0.f;
+      if (kj > q0 + 2 * h + 1) y1 = 0.f;
+      ds2[h] = f2_pack(y0, y1);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------ fused, d = 64
+// One pass at d = 64: one CTA per 128-key block steps through the 128-row query blocks that see it.
+//   S^T = K Q^T and dP^T = V dO^T (N = 128 queries); P^T = exp2(S^T c - lse2) written over S^T in
+//   tensor memory; dS^T = P^T (dP^T - D) into a shared-memory tile;
+//   dV += P^T dO and dK += dS^T Q (N = d = 64, accumulated over the block);
+//   dQ = dS K for the step's 128 queries (M = 128 queries, so no 64-row MMA), into one of two
+//   tensor-memory buffers; the warps stage sigma dQ in shared memory (128-byte swizzled fp32
+//   boxes of 32 columns) and one thread adds it into dq_sub with two TMA tensor reductions
+//   (cp.reduce.async.bulk.tensor .add), so the atomic traffic runs in the copy engine while the
+//   warps go on. dq_sub is zeroed by the D kernel first; the order of the key blocks' terms in a
+//   dq_sub row varies from run to run, as in the d = 128 one-pass kernel.
+template <int D>
+struct LayFused64 {
+  static constexpr int K = 0;                 // [128 keys][64]
+  static constexpr int V = K + T128;          // [128 keys][64]
+  static constexpr int ST = V + T128;         // two stages of Q [128][64], dO [128][64]
+  static constexpr int DS = ST + 4 * T128;    // dS^T hi, then lo: [128 keys][128 queries] each
+  static constexpr int STG = DS + 4 * T128;   // sigma dQ staging: two [128 rows][32 fp32] boxes
+  static constexpr int VEC = STG + 2 * T128;  // two stages of lse[128], D[128]
+  static constexpr int BAR = VEC + 2 * 1024;
+  static constexpr int BYTES = BAR + 256;
+};
+static_assert(LayFused64<64>::BYTES + 1024 <= 232448, "d = 64 one-pass backward shared memory");
+
+__device__ inline void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y) : "memory");
+}
+__device__ inline void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ inline void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ inline void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ inline void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory"); }
+
+// bars: 0 K+V | 1-2 stages loaded | 3-4 stages free | 5 S^T done | 6 dP^T done | 7 P^T written
+//       | 8 dS^T written | 9-10 dQ buffer done | 11-12 dQ buffer read | 13 dV done | 14 dK done
+//       | 15 drain of the MMA issuer
+// TMEM columns: S^T 0-127 (P^T written over it: 16 queries per 16 columns, hi then lo), dP^T
+// 128-255, dV 256-319, dK 320-383, dQ buffers 384 and 448 (lanes = queries, columns = d).
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_fused64_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                    const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                    const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
+                    const float* __restrict__ delta, float* __restrict__ dK, float* __restrict__ dV,
+                    int S, int BH, float sigma, float scale_log2, uint32_t* status, uint64_t wait_ns) {
+  static_assert(D == 64, "the d = 64 one-pass kernel");
+  using Ly = LayFused64<D>;
+  constexpr int kBars = 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Ly::BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + kBars) + 1;
+  uint64_t* const bar_kv = bar;
+  uint64_t* const bar_st = bar + 1;      // + stage
+  uint64_t* const bar_stfree = bar + 3;  // + stage
+  uint64_t* const bar_s = bar + 5;
+  uint64_t* const bar_dp = bar + 6;
+  uint64_t* const bar_p = bar + 7;
+  uint64_t* const bar_ds = bar + 8;
+  uint64_t* const bar_dq = bar + 9;      // + buffer
+  uint64_t* const bar_dqr = bar + 11;    // + buffer
+  uint64_t* const bar_vdone = bar + 13;
+  uint64_t* const bar_kdone = bar + 14;
+  uint64_t* const bar_drain = bar + 15;
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int kb = blockIdx.y;  // low key blocks see the most queries: heaviest first in a group
+  const int bh = (int)blockIdx.z * kHeadGroup + (int)blockIdx.x;
+  if (bh >= BH) return;  // the last group may be partial
+  const int g0 = bh * S;         // first row of this (b,h)
+  const int k0 = kb * 128;       // first key of the block; its first query block too
+  const int nit = (S - k0) / 128;
+
+  if (tid == 0) {
+    for (int i = 0; i < kBars; ++i) {
+      uint64_t* b = bar + i;
+      mbar_init(b, (b == bar_p || b == bar_ds || b == bar_dqr || b == bar_dqr + 1) ? kCompute / 32 : 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t t_s = tbase, t_dp = tbase + 128, t_dv = tbase + 256, t_dk = tbase + 320;
+  const uint32_t t_dq = tbase + 384;  // + 64 * buffer
+  constexpr uint32_t kLo = (2 * T128) >> 4;  // dS^T lo tile, in descriptor units
+
+  if (warp == kCompute / 32) {
+    // ------------------------------------------------------------------ TMA: K, V, then Q/dO stages
+    if ((tid % 32) == 0) {
+      prefetch_tmap(&tk); prefetch_tmap(&tv); prefetch_tmap(&tq); prefetch_tmap(&tdo);
+      mbar_expect_tx(bar_kv, 2 * T128);
+      tma_load_2d(sm + Ly::K, &tk, 0, g0 + k0, bar_kv);
+      tma_load_2d(sm + Ly::V, &tv, 0, g0 + k0, bar_kv);
+      int issued = 0;
+      for (int j = 0; j < nit; ++j) {  // step j into stage j % 2 once dK(j - 2) is done
+        if (j >= 2 && !mbar_wait(bar_stfree + (j & 1), ((j - 2) >> 1) & 1, abort_flag, status, wait_ns)) break;
+        uint64_t* b = bar_st + (j & 1);
+        uint8_t* stg = sm + Ly::ST + (j & 1) * 2 * T128;
+        mbar_expect_tx(b, 2 * T128 + 1024);
+        tma_load_2d(stg, &tq, 0, g0 + k0 + j * 128, b);
+        tma_load_2d(stg + T128, &tdo, 0, g0 + k0 + j * 128, b);
+        bulk_load(sm + Ly::VEC + (j & 1) * 1024, lse + g0 + k0 + j * 128, 512, b);
+        bulk_load(sm + Ly::VEC + (j & 1) * 1024 + 512, delta + g0 + k0 + j * 128, 512, b);
+        ++issued;
+      }
+      mbar_drain(bar_kv, 0, status);
+      drain_ring(bar_st, 2, issued, status);
+    }
+  } else if (warp == kCompute / 32 + 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if ((tid % 32) == 0) {
+      const uint32_t s_k = smem_u32(sm + Ly::K), s_v = smem_u32(sm + Ly::V);
+      const uint32_t s_st = smem_u32(sm + Ly::ST), s_ds = smem_u32(sm + Ly::DS);
+      // K-major: LBO 16, SBO 1024. MN-major: LBO = the distance between 64-element halves of the
+      // M or N extent (one [128][64] sub-tile), SBO = 1024 between 8-row groups along K.
+      const uint64_t aK = desc_base(16, 1024) + (s_k >> 4), aV = desc_base(16, 1024) + (s_v >> 4);
+      const uint64_t bKm = desc_base(T128, 1024) + (s_k >> 4);  // K as B of dQ (N = d), MN-major
+      const uint64_t bStK = desc_base(16, 1024) + (s_st >> 4);   // Q, dO as B of S^T, dP^T
+      const uint64_t bStM = desc_base(T128, 1024) + (s_st >> 4); // Q, dO as B of dK, dV (N = d)
+      const uint64_t aSk = desc_base(16, 1024) + (s_ds >> 4);    // dS^T as A of dK, K-major
+      const uint64_t aSm = desc_base(T128, 1024) + (s_ds >> 4);  // dS as A of dQ (M = queries), MN-major
+      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t IDESC_ACC = idesc_bf16(128, D, false, true);
+      constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, true, true);
+      auto stage = [](int j, int which) { return (uint32_t)(((j & 1) * 2 + which) * T128) >> 4; };
+      auto issue_s = [&](int j) {  // S^T = K Q^T
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(t_s, aK + ks * 2, bStK + stage(j, 0) + ks * 2, IDESC_S, ks > 0);  // + ks * 32 bytes
+        mma_commit(bar_s);
+      };
+      auto issue_dp = [&](int j) {  // dP^T = V dO^T
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(t_dp, aV + ks * 2, bStK + stage(j, 1) + ks * 2, IDESC_S, ks > 0);
+        mma_commit(bar_dp);
+      };
+      auto issue_dv = [&](int j) {  // dV += (P^T_hi + P^T_lo) dO, 16 queries per MMA
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t b = bStM + stage(j, 1) + ks * 128;  // + ks * 2048 bytes: 16 query rows
+          mma_ts(t_dv, t_s + ks * 16, b, IDESC_ACC, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(t_dv, t_s + ks * 16 + 8, b, IDESC_ACC, 1u);
+        }
+        mma_commit(bar_vdone);  // P^T's columns are free once this completes
+      };
+      auto issue_dq = [&](int j) {  // dQ = (dS_hi + dS_lo) K, 16 keys per MMA, fresh each step
+        const uint32_t t = t_dq + (j & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = aSm + kk * 128, b = bKm + kk * 128;  // + kk * 2048 bytes: 16 keys
+          mma_ss(t, a, b, IDESC_DQ, kk > 0 ? 1u : 0u);
+          mma_ss(t, a + kLo, b, IDESC_DQ, 1u);
+        }
+        mma_commit(bar_dq + (j & 1));
+      };
+      auto issue_dk = [&](int j) {  // dK += (dS^T_hi + dS^T_lo) Q
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t b = bStM + stage(j, 0) + ks * 128;
+          const uint32_t offA = ((ks / 4) * T128 + (ks % 4) * 32) >> 4;
+          mma_ss(t_dk, aSk + offA, b, IDESC_ACC, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(t_dk, aSk + offA + kLo, b, IDESC_ACC, 1u);
+        }
+        mma_commit(bar_stfree + (j & 1));  // the stage of step j is free once this completes
+        mma_commit(bar_kdone);
+      };
+      // Per step j: dV(j); S^T(j+1) once dV(j) has read P^T(j); dP^T(j+1) once the warps have
+      // read dP^T(j); then dQ(j) and dK(j), which fill the pipe while the warps start step j+1.
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, status, wait_ns) &&
+                mbar_wait(bar_st, 0, abort_flag, status, wait_ns);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int j = 0; j < nit && ok; ++j) {
+        if (!mbar_wait(bar_p, j & 1, abort_flag, status, wait_ns)) break;
+        tc_fence_after();
+        issue_dv(j);
+        if (j + 1 < nit) {
+          if (!mbar_wait(bar_st + ((j + 1) & 1), ((j + 1) >> 1) & 1, abort_flag, status, wait_ns) ||
+              !mbar_wait(bar_vdone, j & 1, abort_flag, status, wait_ns))
+            break;
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (!mbar_wait(bar_ds, j & 1, abort_flag, status, wait_ns)) break;  // dS^T(j); dP^T(j) read
+        tc_fence_after();
+        if (j + 1 < nit) issue_dp(j + 1);
+        if (j >= 2 && !mbar_wait(bar_dqr + (j & 1), ((j - 2) >> 1) & 1, abort_flag, status, wait_ns)) break;
+        tc_fence_after();
+        issue_dq(j);
+        issue_dk(j);
+      }
+      mma_drain(bar_drain, status);
+    }
+  } else if (warp < kCompute / 32) {
+    // ------------------------------------------------------------------ compute warps
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;  // this warp's lane quarter
+    const int row = (warp % 4) * 32 + (tid % 32);  // key row of S^T; query row of dQ
+    const int qtr = warp / 4;                       // this thread's 32 of the step's 128 queries
+    const int kj = k0 + row;
+    uint8_t* const ds_row = sm + Ly::DS + (qtr >> 1) * T128 + (row >> 3) * 1024 + (row & 7) * 128;
+    const int cb = (qtr & 1) * 4;
+    // this thread's 16 columns of sigma dQ in the staging box qtr / 2 (32 fp32 per 128-byte row)
+    uint8_t* const stg_row = sm + Ly::STG + (qtr >> 1) * T128 + row * 128;
+    auto wait_all = [&](uint64_t* b, uint32_t parity) {
+      bool w = mbar_wait(b, parity, abort_flag, status, wait_ns);
+      return __all_sync(0xffffffffu, w);
+    };
+    // dQ of step i: read it, stage sigma dQ, and add it into dq_sub rows with the copy engine.
+    // Every compute warp reaches both barriers whatever `ok` is, so none waits alone.
+    auto flush_dq = [&](int i, bool& ok) {
+      uint32_t r[16];
+      ok = ok && wait_all(bar_dq + (i & 1), (i >> 1) & 1);
+      tc_fence_after();
+      if (ok) {
+        tmem_ld16(t_dq + (i & 1) * 64 + lane_off + qtr * 16, r);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_dqr + (i & 1));
+      if (tid == 0) bulk_wait_read_all();  // the previous reduction has read the staging
+      compute_sync();
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int ch = (cb + c) ^ (row & 7);
+          *reinterpret_cast<float4*>(stg_row + ch * 16) =
+              make_float4(__uint_as_float(r[4 * c]) * sigma, __uint_as_float(r[4 * c + 1]) * sigma,
+                          __uint_as_float(r[4 * c + 2]) * sigma, __uint_as_float(r[4 * c + 3]) * sigma);
+        }
+      }
+      fence_async_smem();  // the staging stores, visible to the copy engine
+      compute_sync();
+      if (ok && tid == 0) {
+        tma_reduce_add_2d(&tdq, sm + Ly::STG, 0, g0 + k0 + i * 128);
+        tma_reduce_add_2d(&tdq, sm + Ly::STG + T128, 32, g0 + k0 + i * 128);
+        bulk_commit();
+      }
+    };
+    bool ok = true;
+    for (int j = 0; j < nit; ++j) {
+      const int q0 = k0 + j * 128 + qtr * 32;  // query row of this thread's first column
+      const bool diag = j == 0;                // the first step holds the diagonal block
+      const float* vec = reinterpret_cast<const float*>(sm + Ly::VEC + (j & 1) * 1024);
+      // P^T, written over this thread's S^T columns
+      ok = ok && wait_all(bar_s, j & 1) && wait_all(bar_st + (j & 1), (j >> 1) & 1);
+      tc_fence_after();
+      uint64_t p2[2][8];
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[16];
+          tmem_ld16(t_s + lane_off + qtr * 32 + h * 16, r);
+          tmem_wait_ld();
+          p_elements(r, vec + qtr * 32 + h * 16, scale_log2, kj, q0 + h * 16, diag, p2[h]);
+          uint32_t wp[8], wq[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) split_bf16x2_f2(p2[h][e], wp[e], wq[e]);
+          tmem_st8(t_s + lane_off + (2 * qtr + h) * 16, wp);
+          tmem_st8(t_s + lane_off + (2 * qtr + h) * 16 + 8, wq);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_p);
+      // dS^T into shared memory, once dQ(j-1) and dK(j-1) have read the previous one
+      ok = ok && wait_all(bar_dp, j & 1) && (j == 0 || wait_all(bar_kdone, (j - 1) & 1));
+      tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[16];
+          tmem_ld16(t_dp + lane_off + qtr * 32 + h * 16, r);
+          tmem_wait_ld();
+          uint64_t ds2[8];
+          ds_elements(p2[h], r, vec + 128 + qtr * 32 + h * 16, kj, q0 + h * 16, diag, ds2);
+          uint32_t wh[8], wl[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) split_bf16x2_f2(ds2[e], wh[e], wl[e]);
+          const int c0 = ((cb + 2 * h) ^ (row & 7)) * 16, c1 = ((cb + 2 * h + 1) ^ (row & 7)) * 16;
+          *reinterpret_cast<uint4*>(ds_row + c0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(ds_row + c1) = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+          *reinterpret_cast<uint4*>(ds_row + 2 * T128 + c0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          *reinterpret_cast<uint4*>(ds_row + 2 * T128 + c1) = make_uint4(wl[4], wl[5], wl[6], wl[7]);
+        }
+      }
+      fence_async_smem();  // the dS^T stores, visible to the MMAs that read them
+      tc_fence_before();
+      __syncwarp();
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_ds);
+      if (j > 0) flush_dq(j - 1, ok);
+    }
+    flush_dq(nit - 1, ok);
+    // ---- epilogue: dV, dK rows (dK(nit-1) is the CTA's last MMA)
+    ok = ok && !*abort_flag && wait_all(bar_kdone, (nit - 1) & 1);
+    tc_fence_after();
+    if (ok)
+      store_dkdv<D>(dV + (size_t)(g0 + kj) * D, dK + (size_t)(g0 + kj) * D, t_dv, t_dk, lane_off, qtr, sigma);
+    if (tid == 0) bulk_wait_all();  // every reduction has finished reading the staging
+  }
+  // every role has drained its own loads and MMAs: nothing still writes shared or tensor memory
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
 // ------------------------------------------------------------------------------------ dQ
 constexpr int kStK = 4;  // K/V stages of the dQ kernel
 
@@ -853,7 +1228,7 @@ template <int D>
 cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs, const float* os,
                     const float* lse, const void* dos, float* dq, float* dk, float* dv, float* delta,
                     uint32_t* status, cudaStream_t st) {
-  const bool fused = D == 128 && !(g.flags & LH_DETERMINISTIC);
+  const bool fused = !(g.flags & LH_DETERMINISTIC);
   const int64_t rows = g.BH * g.S;
   CUtensorMap q64, do64, k128, v128;
   if (!make_tmap_rows_box(&q64, qs, rows, D, 64) || !make_tmap_rows_box(&do64, dos, rows, D, 64) ||
@@ -867,6 +1242,21 @@ cudaError_t run_bwd(const Geo& g, const void* qs, const void* ks, const void* vs
   const float scale_log2 = sigma * kLog2e;
   const dim3 grid((unsigned)(g.BH < kHeadGroup ? g.BH : kHeadGroup), (unsigned)(g.S / 128),
                   (unsigned)((g.BH + kHeadGroup - 1) / kHeadGroup));
+  if constexpr (D == 64) {
+    if (fused) {
+      CUtensorMap q128f, do128f, dq32;
+      if (!make_tmap_rows_box(&q128f, qs, rows, D, 128) || !make_tmap_rows_box(&do128f, dos, rows, D, 128) ||
+          !make_tmap_f32_box(&dq32, dq, rows, D, 128))
+        return cudaErrorInvalidValue;
+      const int smem = padded_smem(LayFused64<D>::BYTES);
+      e = cudaFuncSetAttribute(attn_bwd_fused64_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      attn_bwd_fused64_tc<D><<<grid, kThreads, smem, st>>>(k128, v128, q128f, do128f, dq32, lse, delta, dk, dv,
+                                                            g.S, (int)g.BH, sigma, scale_log2, status,
+                                                            g.wait_ns);
+      return cudaGetLastError();
+    }
+  }
   if constexpr (D == 128) {
     if (fused) {
       const int smem = padded_smem(LayFused<D>::BYTES);
@@ -926,7 +1316,7 @@ cudaError_t launch_attn_bwd_tc_rows(const Geo& g, int kb0, int Sk, const void* q
 }
 
 bool attn_bwd_fused(const Geo& g) {
-  return attn_tc_eligible(g) && g.d == 128 && !(g.flags & LH_DETERMINISTIC);
+  return attn_tc_eligible(g) && !(g.flags & LH_DETERMINISTIC);
 }
 
 cudaError_t launch_attn_bwd_tc(const Geo& g, const void* qs, const void* ks, const void* vs,

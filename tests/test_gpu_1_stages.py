@@ -196,12 +196,14 @@ def test_out_of_range_ids_are_flagged_not_faulted():
     assert lh.lh_check(ws) == (0, 0)  # cleared by the read
 
 
-@pytest.mark.parametrize("B,H,S", [(1, 2, 4096), (1, 9, 1024), (2, 3, 384)])
-def test_fused_backward_matches_the_deterministic_one(B, H, S):
+@pytest.mark.parametrize("B,H,S,d", [(1, 2, 4096, 128), (1, 9, 1024, 128), (2, 3, 384, 128),
+                                     (1, 2, 4096, 64), (1, 9, 1024, 64), (2, 3, 384, 64)])
+def test_fused_backward_matches_the_deterministic_one(B, H, S, d):
     """The one-pass backward computes dK and dV exactly as the two-pass one (the same MMAs
     accumulate in the same order), so they agree bit for bit. Its dQ adds fp32 partial sums per
-    128-key block in a varying order: it agrees to fp32 rounding of those sums."""
-    d, dtype = 128, torch.bfloat16
+    128-key block in a varying order (atomic adds at d = 128, copy-engine reductions at d = 64):
+    it agrees to fp32 rounding of those sums."""
+    dtype = torch.bfloat16
     qs, ks, vs, dos = rand_sub(B, H, S, d, dtype, seed=S + 1)
     out = {}
     for det in (False, True):
