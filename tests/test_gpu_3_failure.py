@@ -24,12 +24,14 @@ def _inputs(shape, seed):
             for _ in range(4)]
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("det", [False, True])
 @pytest.mark.parametrize("S", [128, 512])
-def test_wait_timeout_is_reported_and_the_next_call_is_correct(S, det):
+def test_wait_timeout_is_reported_and_the_next_call_is_correct(S, det, d):
     """One CTA per attention kernel at S = 128 (several at 512): the forward, and the one-pass
-    (det=False) or two-pass (det=True) backward, all run out of their waits."""
-    shape = Shape(1, 1, S, 128, 4, 1, S, torch.bfloat16, det)  # L = 1: dense causal attention
+    (det=False) or two-pass (det=True) backward, all run out of their waits. At d = 64 the
+    one-pass kernel's compute warps still meet at the barriers around the dQ staging."""
+    shape = Shape(1, 1, S, d, 4, 1, S, torch.bfloat16, det)  # L = 1: dense causal attention
     q, k, v, d_o = _inputs(shape, S)
     layer = LighthouseLayer(shape)
     prev = lh.lh_set_wait_limit_ns(1)
