@@ -4,30 +4,33 @@
 // 2.C: dense causal attention on the S selected rows; row j visible to row i iff j <= i).
 //
 // One CTA = 128 query rows of one (b,h). Warp roles:
-//  - warps 0-7 (softmax): warps w and w+4 share the TMEM lanes 32(w%4)..+31 (query rows); warp w
-//    takes keys 0-63 of every block and warp w+4 keys 64-127, and the pair swaps row maxima
-//    through shared memory (a 64-thread named barrier) so that both halves use one max;
-//  - warp 8, one lane: TMA loads (Q once; K through a three-stage ring, V through two or three);
-//  - warp 9, one lane: the S MMAs; warp 10, one lane: the PV MMAs. Two issuers keep the tensor
-//    queue fed while either waits on its own barriers.
-// Tensor memory (512 columns) holds four disjoint regions, so that no MMA writes columns that
-// an earlier MMA may still read:
-//   S buffers at 0 and 128 (S_{j+1} = Q K_{j+1}^T runs while the softmax of S_j does),
-//   O at 256, P at 384 (hi in 384..447, lo in 448..511: 128 bf16 keys, two per column).
+//  - warps 0-15 (softmax), in two sets: set 0 (warps 0-7) takes the even key blocks, set 1
+//    (warps 8-15) the odd ones, so that one set's exponentials run while the other set loads its
+//    scores, takes its maxima and waits. Warps w, w+4, w+8, w+12 share the TMEM lanes
+//    32(w%4)..+31 (query rows); within a set, warp w takes keys 0-63 of its block and warp w+4
+//    keys 64-127;
+//  - warp 16, one lane: TMA loads (Q once; K through a three-stage ring, V through two or three,
+//    the two rings advancing independently);
+//  - warp 17, one lane: the S MMAs; warp 18, one lane: the PV MMAs.
+// Tensor memory (512 columns): three S/P buffers at 0, 128 and 256 and O at 384. S_j = Q K_j^T
+// goes to buffer j % 3; once the softmax warps hold S_j in registers they write P_j over it, and
+// PV_j reads P_j there. S_{j+3} waits for PV_j.
 //  - P_j = hi + lo with hi = bf16(P) and lo = bf16(P - hi), and O += hi V_j + lo V_j takes the
-//    A operand from tensor memory. The split keeps P to ~16 bits: the backward recomputes P
-//    exactly and forms D_i = dO_i . O_i, so an O made from bf16-rounded P would leave
-//    sum_j dS_ij off zero by dO . (O error), which is large on coarse rows whose dO sums
-//    thousands of tokens.
-//  - The running max is updated lazily: O and l are rescaled only when a row's max grows by more
-//    than 2^8, which keeps every exponent bounded and skips most TMEM round trips.
+//    A operand from tensor memory (hi of keys 16i..16i+15 in 8 columns, their lo in the next 8).
+//    The split keeps P to ~16 bits: the backward recomputes P exactly and forms
+//    D_i = dO_i . O_i, so an O made from bf16-rounded P would leave sum_j dS_ij off zero by
+//    dO . (O error), which is large on coarse rows whose dO sums thousands of tokens.
+//  - The running max is updated lazily: O is rescaled only when a row's max grows by more than
+//    2^8, which keeps every exponent bounded and skips most TMEM round trips. The max of block j
+//    goes from one set to the other through shared memory and a named barrier per set and lane
+//    quarter, on which the set of block j syncs and the set of block j - 1 arrives; the same
+//    barrier swaps the two halves' block maxima. Each warp keeps its own row sum, relative to
+//    the max it last used, and the four sums of a row meet in the epilogue.
 //  - The softmax warps are bound by instruction issue and the ex2 unit, so their arithmetic is
 //    counted: the row max is taken over the raw scores with three-input max (exact, as the scale is
 //    positive), the scale enters the exponent through one packed f32x2 FMA per pair of keys, and
 //    the row sums and the lo residuals are packed f32x2 adds and subtracts.
 //  - Key blocks above the diagonal are skipped; the diagonal block is masked.
-// Tensor-core order: S_0, S_1, PV_0, S_2, PV_1, ... The softmax of S_j therefore overlaps PV_{j-1}
-// and S_{j+1}; it writes P_j only after PV_{j-1} has finished reading P and O.
 // The output is fp32 O_sub and the natural-log lse. Shared memory per CTA: Q + 3 K + 2 V tiles of
 // 128 rows at d = 128 (192 KB; 3 V tiles at d = 64), one CTA per SM.
 #include <mutex>
@@ -40,8 +43,9 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kSoftmax = 256, kThreads = kSoftmax + 96;  // + the TMA warp and two MMA warps
+constexpr int kSoftmax = 512, kThreads = kSoftmax + 96;  // + the TMA warp and two MMA warps
 constexpr int kStages = 3;  // K ring
+constexpr int kSBuf = 3;    // S/P buffers in tensor memory
 template <int D> constexpr int v_stages() { return D == 128 ? 2 : 3; }
 constexpr int TILE = 128 * 128;  // bytes of one [128 rows][64 bf16] 128B-swizzled sub-tile
 
@@ -52,13 +56,18 @@ struct Layout {
   static constexpr int K = Q + KB * TILE;            // stage s at K + s * KB * TILE
   static constexpr int V = K + kStages * KB * TILE;  // stage s at V + s * KB * TILE
   static constexpr int BAR = V + v_stages<D>() * KB * TILE;
-  static constexpr int XCH = BAR + 256;              // [2 parities][2 halves][128 rows] floats
-  static constexpr int BYTES = XCH + 2 * 2 * 128 * 4;
+  // floats [.][128 rows]: XM [2] the max block j used, at j & 1; XC [4][2 halves] the halves'
+  // maxima of block j, at j & 3; XL, XE [4 warps] partial row sums and the max each is relative to
+  static constexpr int XM = BAR + 256;
+  static constexpr int XC = XM + 2 * 128 * 4;
+  static constexpr int XL = XC + 8 * 128 * 4;
+  static constexpr int XE = XL + 4 * 128 * 4;
+  static constexpr int BYTES = XE + 4 * 128 * 4;
 };
 
-// bars: 0 Q | 1-3 K loaded | 4-6 V loaded | 7-9 K free | 10-12 V free | 13-14 S ready
-//       | 15-16 S buffer read | 17 P written | 18 PV done | 19-20 drain of the two MMA issuers
-constexpr int kBars = 21;
+// bars: 0 Q | 1-3 K loaded | 4-6 V loaded | 7-9 K free | 10-12 V free | 13-15 S ready
+//       | 16-18 P written | 19-21 PV done | 22 last PV done | 23-24 drain of the two MMA issuers
+constexpr int kBars = 25;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -79,9 +88,9 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   uint64_t* const bar_kfree = bar + 7;
   uint64_t* const bar_vfree = bar + 10;
   uint64_t* const bar_s = bar + 13;
-  uint64_t* const bar_sfree = bar + 15;
-  uint64_t* const bar_p = bar + 17;
-  uint64_t* const bar_pv = bar + 18;
+  uint64_t* const bar_p = bar + 16;
+  uint64_t* const bar_pv = bar + 19;
+  uint64_t* const bar_fin = bar + 22;
 
   const int tid = threadIdx.x, warp = tid / 32;
   // S query rows and Sk key rows per (b,h); the queries are the global rows 128 kb0 .. of the
@@ -96,7 +105,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
   if (tid == 0) {
     for (int i = 0; i < kBars; ++i)
-      mbar_init(bar + i, (i == 15 || i == 16 || i == 17) ? kSoftmax / 32 : 1);  // one arrival per warp
+      mbar_init(bar + i, (i >= 16 && i <= 18) ? 8 : 1);  // P written: the eight warps of one set
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -105,7 +114,7 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t t_o = tbase + 256, t_p = tbase + 384;
+  const uint32_t t_o = tbase + kSBuf * 128;
 
   if (warp == kSoftmax / 32) {
     // ------------------------------------------------------------------ TMA warp
@@ -125,14 +134,30 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       };
       mbar_expect_tx(bar_q, KB * TILE);
       for (int c = 0; c < KB; ++c) tma_load_2d(sm + Ly::Q + c * TILE, &tq, c * 64, grow0 + qb * BM, bar_q);
+      // The two rings advance independently: K_j reuses the stage of K_{j-3} once S_{j-3} has read
+      // it, V_j that of V_{j-kStV} once PV_{j-kStV} has, and a K load never waits behind a V stage.
       int nk = 0, nv = 0;  // loads issued into each ring
-      for (int j = 0; j < nkb; ++j) {  // block j reuses the K stage of block j - 3, the V stage of j - kStV
-        if (j >= kStages && !mbar_wait(bar_kfree + j % kStages, ((j - kStages) / kStages) & 1, abort_flag, status, wait_ns)) break;
-        load_k(j);
-        ++nk;
-        if (j >= kStV && !mbar_wait(bar_vfree + j % kStV, ((j - kStV) / kStV) & 1, abort_flag, status, wait_ns)) break;
-        load_v(j);
-        ++nv;
+      uint64_t t_moved = globaltimer();
+      for (uint32_t it = 1; nk < nkb || nv < nkb; ++it) {
+        bool moved = false;
+        if (nk < nkb && (nk < kStages || mbar_try(bar_kfree + nk % kStages, ((nk - kStages) / kStages) & 1))) {
+          load_k(nk++);
+          moved = true;
+        }
+        if (nv < nk && (nv < kStV || mbar_try(bar_vfree + nv % kStV, ((nv - kStV) / kStV) & 1))) {
+          load_v(nv++);
+          moved = true;
+        }
+        if (moved) {
+          t_moved = globaltimer();
+        } else if ((it & 255) == 0) {  // no stage freed for wait_ns: the bound of every other wait
+          if (*abort_flag) break;
+          if (globaltimer() - t_moved > wait_ns) {
+            *abort_flag = 1;
+            raise_fault(status, kFaultTimeout);
+            break;
+          }
+        }
       }
       // every load issued has landed before this thread leaves (on the normal path they were
       // all consumed already, so these return at once)
@@ -149,88 +174,97 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       const uint64_t dV = desc_base(TILE, 1024) + (s_v >> 4);  // MN-major: LBO = one sub-tile
       constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
-      auto issue_s = [&](int j) {  // S_j = Q K_j^T into TMEM buffer j & 1
+      auto issue_s = [&](int j) {  // S_j = Q K_j^T into TMEM buffer j % 3
         const uint32_t sg = (uint32_t)((j % kStages) * KB * TILE) >> 4;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = ((ks / 4) * TILE + (ks % 4) * 32) >> 4;
-          mma_ss(tbase + (j & 1) * 128, dQ + off, dK + sg + off, IDESC_S, ks > 0);
+          mma_ss(tbase + (j % kSBuf) * 128, dQ + off, dK + sg + off, IDESC_S, ks > 0);
         }
-        mma_commit(bar_s + (j & 1));
+        mma_commit(bar_s + j % kSBuf);
         mma_commit(bar_kfree + j % kStages);
       };
-      auto issue_pv = [&](int j) {  // O += hi_j V_j + lo_j V_j
+      auto issue_pv = [&](int j) {  // O += hi_j V_j + lo_j V_j, P_j over S_j in buffer j % 3
         const uint32_t sg = (uint32_t)((j % kStV) * KB * TILE) >> 4;
+        const uint32_t tp = tbase + (j % kSBuf) * 128;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_ts(t_o, t_p + part * 64 + ks * 8, dV + sg + ks * (2048 >> 4), IDESC_PV,
+          for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: hi at column 16 ks, lo at 16 ks + 8
+            mma_ts(t_o, tp + ks * 16 + part * 8, dV + sg + ks * (2048 >> 4), IDESC_PV,
                    (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(bar_pv);
+        mma_commit(bar_pv + j % kSBuf);
         mma_commit(bar_vfree + j % kStV);
       };
       if (s_issuer) {
         bool ok = mbar_wait(bar_q, 0, abort_flag, status, wait_ns);
-        for (int n = 0; n < nkb && ok; ++n) {  // S_n into buffer n & 1 once the softmax has read S_{n-2}
+        for (int n = 0; n < nkb && ok; ++n) {  // S_n into buffer n % 3 once PV_{n-3} has read P_{n-3} there
           ok = mbar_wait(bar_k + n % kStages, (n / kStages) & 1, abort_flag, status, wait_ns);
-          if (ok && n >= 2) ok = mbar_wait(bar_sfree + (n & 1), ((n >> 1) - 1) & 1, abort_flag, status, wait_ns);
+          if (ok && n >= kSBuf) ok = mbar_wait(bar_pv + n % kSBuf, ((n / kSBuf) - 1) & 1, abort_flag, status, wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_s(n);
         }
-        mma_drain(bar + 19, status);
+        mma_drain(bar + 23, status);
       } else {
-        for (int j = 0; j < nkb; ++j) {
-          const bool ok = mbar_wait(bar_p, j & 1, abort_flag, status, wait_ns) &&
+        int j = 0;
+        for (; j < nkb; ++j) {
+          const bool ok = mbar_wait(bar_p + j % kSBuf, (j / kSBuf) & 1, abort_flag, status, wait_ns) &&
                           mbar_wait(bar_v + j % kStV, (j / kStV) & 1, abort_flag, status, wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_pv(j);
         }
-        mma_drain(bar + 20, status);
+        if (j == nkb) mma_commit(bar_fin);
+        mma_drain(bar + 24, status);
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    constexpr int DH = D / 2;  // O columns each half rescales and stores
-    const int q4 = warp % 4, half = warp / 4;
+    // Set 0 (warps 0-7) takes the even key blocks, set 1 (warps 8-15) the odd ones. Warps
+    // w, w + 4, w + 8, w + 12 own the same 32 query rows (TMEM lanes 32 (w % 4) ..); within a set,
+    // warp w + 4 h takes keys 64 h .. 64 h + 63 of the block. One set's exponentials thus overlap
+    // the other set's loads, maxima and waits.
+    constexpr int DQ = D / 4;  // O columns each of the four warps of a lane quarter stores
+    const int q4 = warp % 4, half = (warp / 4) & 1, set = warp / 8;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const int row = q4 * 32 + (tid % 32);  // query row within the tile = TMEM lane
-    float* const xch = reinterpret_cast<float*>(sm + Ly::XCH);
-    // Warps w and w+4 meet here every block, so both always reach it: a failed wait clears `ok`
-    // and the loop goes on without touching tensor memory.
-    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
-    // all lanes of a warp wait together, so that the warp stays converged for tcgen05.ld/st
-    auto wait_all = [&](uint64_t* b, uint32_t parity) {
+    float* const xm = reinterpret_cast<float*>(sm + Ly::XM);
+    float* const xc = reinterpret_cast<float*>(sm + Ly::XC);
+    float* const xl = reinterpret_cast<float*>(sm + Ly::XL);
+    float* const xe = reinterpret_cast<float*>(sm + Ly::XE);
+    // Block j meets on the named barrier of its set and lane quarter: the set's two warps sync,
+    // having stored their halves' maxima, and the other set's two warps arrive, having stored
+    // the max block j - 1 used (block 0 has no predecessor: its two warps alone). Every warp
+    // takes these steps for every block of its set whatever its waits returned, so a failed wait
+    // never strands another warp at a barrier.
+    const int bar_in = 1 + 4 * set + q4, bar_out = 1 + 4 * (set ^ 1) + q4;
+    auto wait_all = [&](uint64_t* b, uint32_t parity) {  // the whole warp waits, converged
       bool ok = mbar_wait(b, parity, abort_flag, status, wait_ns);
       return __all_sync(0xffffffffu, ok);
     };
-    float m_used = -INFINITY, l = 0.f;
+    float m_mine = -INFINITY, l = 0.f;  // this warp's partial row sum, relative to m_mine
     bool ok = true;
-    for (int j = 0; j < nkb; ++j) {
-      ok = ok && wait_all(bar_s + (j & 1), (j >> 1) & 1);
+    for (int j = set; j < nkb; j += 2) {
+      ok = ok && wait_all(bar_s + j % kSBuf, (j / kSBuf) & 1);
       tc_fence_after();
+      const uint32_t ts = tbase + (j % kSBuf) * 128 + half * 64 + lane_off;  // this warp's 64 keys
       float s[64];
       if (ok) {
         uint32_t r0[32], r1[32];
-        const uint32_t ts = tbase + (j & 1) * 128 + half * 64 + lane_off;
         tmem_ld32(ts, r0);
         tmem_ld32(ts + 32, r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(r0[e]);  // raw scores: the scale goes into the exponent's FMA
+        for (int e = 0; e < 32; ++e) {  // raw scores: the scale goes into the exponent's FMA
+          s[e] = __uint_as_float(r0[e]);
           s[32 + e] = __uint_as_float(r1[e]);
         }
       } else {
 #pragma unroll
         for (int e = 0; e < 64; ++e) s[e] = 0.f;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (ok && (tid % 32) == 0) mbar_arrive(bar_sfree + (j & 1));
       if (j == kb0 + qb) {  // diagonal block: key column > query row is invisible
 #pragma unroll
         for (int e = 0; e < 64; ++e)
@@ -245,37 +279,52 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         m4[c] = fmaxf(m4[c], s[16 * c + 15]);
       }
       const float mloc = max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;
-      xch[((j & 1) * 2 + half) * 128 + row] = mloc;
-      pair_sync();
-      const float mt = fmaxf(mloc, xch[((j & 1) * 2 + (half ^ 1)) * 128 + row]);
-      const bool grow = mt > m_used + 8.0f;
-      const float m_new = grow ? mt : m_used;
-      const float alpha = grow ? exp2f(m_used - m_new) : 1.0f;
+      xc[((j & 3) * 2 + half) * 128 + row] = mloc;
+      if (j == 0) asm volatile("bar.sync %0, 64;" ::"r"(bar_in) : "memory");
+      else asm volatile("bar.sync %0, 128;" ::"r"(bar_in) : "memory");
+      const float mt = fmaxf(mloc, xc[((j & 3) * 2 + (half ^ 1)) * 128 + row]);
+      const float m_prev = j > 0 ? xm[((j - 1) & 1) * 128 + row] : -INFINITY;  // the max block j - 1 used
+      const bool grow = mt > m_prev + 8.0f;
+      const float m_new = grow ? mt : m_prev;
+      if (j + 1 < nkb) {
+        if (half == 0) xm[(j & 1) * 128 + row] = m_new;
+        asm volatile("bar.arrive %0, 128;" ::"r"(bar_out) : "memory");
+      }
       const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
       uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-      uint32_t ph[32], pl[32];
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {  // p = 2^(s * scale - m), a pair per instruction
-        float a0, a1;
-        f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nm2), a0, a1);
-        const uint64_t x = f2_pack(ex2(a0), ex2(a1));
-        sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], x);
-        split_bf16x2_f2(x, ph[e / 2], pl[e / 2]);
+      for (int c = 0; c < 4; ++c) {  // keys 64 half + 16 c ..: P hi in columns 16 c .. + 7, lo in 16 c + 8 ..
+        uint32_t h[8], w[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {  // p = 2^(s * scale - m), a pair per instruction
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(s[16 * c + e], s[16 * c + e + 1]), c2, nm2), a0, a1);
+          const uint64_t x = f2_pack(ex2(a0), ex2(a1));
+          sum2[(e >> 1) & 1] = f2_add(sum2[(e >> 1) & 1], x);
+          split_bf16x2_f2(x, h[e / 2], w[e / 2]);
+        }
+        if (ok) {  // S_j of these columns is in registers already: P goes over it
+          tmem_st8(ts + 16 * c, h);
+          tmem_st8(ts + 16 * c + 8, w);
+        }
       }
       float sa0, sa1, sb0, sb1;
       f2_unpack(sum2[0], sa0, sa1);
       f2_unpack(sum2[1], sb0, sb1);
-      l = l * alpha + ((sa0 + sa1) + (sb0 + sb1));
-      m_used = m_new;
-      // PV_{j-1} must be done before P and O are touched again
-      if (j > 0) {
-        ok = ok && wait_all(bar_pv, (j - 1) & 1);
+      if (m_new != m_mine) l *= exp2f(m_mine - m_new);  // l = 0 before this warp's first block
+      l += (sa0 + sa1) + (sb0 + sb1);
+      m_mine = m_new;
+      // O holds sum_{i<j} P_i V_i relative to m_prev: rescale this warp's half of it once PV_{j-1}
+      // is done (both warps of the set see the same grow flags)
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        ok = ok && wait_all(bar_pv + (j - 1) % kSBuf, ((j - 1) / kSBuf) & 1);
         tc_fence_after();
-        if (ok && __any_sync(0xffffffffu, grow)) {  // rescale this warp's rows of its O half
+        if (ok) {
+          const float alpha = grow ? exp2f(m_prev - m_new) : 1.0f;
           uint32_t r[32];
 #pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            const uint32_t to = t_o + lane_off + half * DH + c * 32;
+          for (int c = 0; c < D / 64; ++c) {
+            const uint32_t to = t_o + lane_off + half * (D / 2) + c * 32;
             tmem_ld32(to, r);
             tmem_wait_ld();
 #pragma unroll
@@ -284,44 +333,50 @@ attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           }
         }
       }
-      if (ok) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {  // keys 64 half + 32c .. : 16 columns of packed pairs
-          uint32_t h[16], w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) { h[e] = ph[c * 16 + e]; w[e] = pl[c * 16 + e]; }
-          tmem_st16(t_p + lane_off + half * 32 + c * 16, h);
-          tmem_st16(t_p + lane_off + 64 + half * 32 + c * 16, w);
-        }
-        tmem_wait_st();
-      }
+      if (ok) tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (ok && (tid % 32) == 0) mbar_arrive(bar_p);
+      if (ok && (tid % 32) == 0) mbar_arrive(bar_p + j % kSBuf);
     }
-    // ---- epilogue: O / l and lse (the pair adds its two partial sums of l)
-    ok = ok && wait_all(bar_pv, (nkb - 1) & 1);
+    // ---- epilogue: O / l and lse (the four warps' partial sums brought to the last max)
+    ok = ok && wait_all(bar_fin, 0);
     tc_fence_after();
-    xch[((nkb & 1) * 2 + half) * 128 + row] = l;
-    pair_sync();
-    const float lo = xch[((nkb & 1) * 2 + (half ^ 1)) * 128 + row];
-    const float lt = half == 0 ? l + lo : lo + l;
+    const int k4 = set * 2 + half;
+    xl[k4 * 128 + row] = l;
+    xe[k4 * 128 + row] = m_mine;
+    asm volatile("bar.sync %0, 128;" ::"r"(9 + q4) : "memory");
+    float m_fin = xe[row];
+#pragma unroll
+    for (int k = 1; k < 4; ++k) m_fin = fmaxf(m_fin, xe[k * 128 + row]);
+    float lt = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lk = xl[k * 128 + row], mk = xe[k * 128 + row];
+      lt += mk == m_fin ? lk : lk * exp2f(mk - m_fin);
+    }
     if (ok) {
       const float inv = 1.0f / lt;
-      float* orow = O + (size_t)(grow0 + qb * BM + row) * D + half * DH;
-      uint32_t r[32];
-#pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        tmem_ld32(t_o + lane_off + half * DH + c * 32, r);
+      float* orow = O + (size_t)(grow0 + qb * BM + row) * D + k4 * DQ;
+      if constexpr (DQ == 32) {
+        uint32_t r[32];
+        tmem_ld32(t_o + lane_off + k4 * DQ, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 v = make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
-                                 __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
-          *reinterpret_cast<float4*>(orow + c * 32 + e) = v;
-        }
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(orow + e) =
+              make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
+                          __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+      } else {
+        uint32_t r[16];
+        tmem_ld16(t_o + lane_off + k4 * DQ, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(orow + e) =
+              make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
+                          __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
       }
-      if (half == 0) lse[grow0 + qb * BM + row] = (m_used + log2f(lt)) * 0.69314718055994531f;
+      if (k4 == 0) lse[grow0 + qb * BM + row] = (m_fin + log2f(lt)) * 0.69314718055994531f;
     }
   }
   // every role has drained its own loads and MMAs, so nothing still writes shared or tensor
