@@ -43,7 +43,7 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # (workload, stage) -> (bytes per call, source digest, how the bytes were obtained)
 MEASURED_TRAFFIC = {
     ("128k", "attn_bwd"): (
-        994826240, "9bd396dd863674f1",
+        996068352, "4e12501af0a2f120",
         "ncu dram__bytes_read.sum + dram__bytes_write.sum of the D and one-pass kernels at 16 of the "
         "32 heads (two of four head groups), x2; reads grow in proportion to head groups (8 -> 16 "
         "heads: 156 -> 312 MB), writes faster (51 -> 186 MB), so the write part is a lower bound"),
