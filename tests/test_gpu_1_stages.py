@@ -128,6 +128,48 @@ def test_attention_fwd_bwd(B, H, S, d, dt, det):
         assert_close(np64(got), want, dtype, n, mode="literal")
 
 
+@pytest.mark.parametrize("S,d", [(1024, 128), (1152, 128), (1024, 64), (1152, 64)])
+def test_attention_running_max_grows(S, d):
+    """The forward's lazy running max: O is rescaled only when a row's max grows by more than
+    2^8, after the previous block's PV. Key blocks are scaled up part-way through the sequence
+    (head 0 at odd blocks, head 1 at even ones), so that growth reaches both sets of softmax
+    warps. Every other query row is scaled down, so that within one warp some rows grow and
+    others do not. N(0,1) inputs never grow after the first block."""
+    B, H = 1, 2
+    dtype = torch.bfloat16
+    shape = Shape(B, H, S, d, 4, 1, S, dtype)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    nb = S // 128
+    grow_at = [(1, 3), (2, 4)]  # blocks where the key scale goes up 4x, per head
+    f = torch.ones(H, nb)
+    for h, blocks in enumerate(grow_at):
+        for b in blocks:
+            f[h, b:] *= 4.0
+    kscale = f.repeat_interleave(128, dim=1)[None, :, :, None].cuda()
+    qscale = torch.where(torch.arange(S) % 2 == 0, 1.0, 0.1)[None, None, :, None].cuda()
+    qs = (torch.randn(B, H, S, d, generator=g, device="cuda") * qscale).to(dtype)
+    ks = (torch.randn(B, H, S, d, generator=g, device="cuda") * kscale).to(dtype)
+    vs, dos = (torch.randn(B, H, S, d, generator=g, device="cuda").to(dtype) for _ in range(2))
+    os_ = torch.empty(B, H, S, d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
+    ws = ws_for(shape)
+    lh.lh_attn_fwd(shape, qs, ks, vs, os_, lse, ws)
+    dq, dk, dv = (torch.empty(B, H, S, d, dtype=torch.float32, device="cuda") for _ in range(3))
+    lh.lh_attn_bwd(shape, qs, ks, vs, os_, lse, dos, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    assert lh.lh_check(ws) == (0, 0)
+    want_o, want_lse = O.attn_fwd(np64(qs), np64(ks), np64(vs))
+    # the running max of an unscaled row that sees every block grows by more than 2^8
+    qr = np64(qs)[0, :, S - 2]
+    sc = np.einsum("hd,hjd->hj", qr, np64(ks)[0, :, :S - 1]) / np.sqrt(d)
+    assert ((sc.max(-1) - sc[:, :128].max(-1)) * np.log2(np.e) > 8).all()
+    assert_close(np64(os_), want_o, dtype, "o_sub", mode="literal")
+    np.testing.assert_allclose(np64(lse), want_lse, rtol=1e-5, atol=1e-5)
+    wq, wk, wv = O.attn_bwd(np64(qs), np64(ks), np64(vs), want_o, want_lse, np64(dos))
+    for got, want, n in ((dq, wq, "dq"), (dk, wk, "dk"), (dv, wv, "dv")):
+        assert_close(np64(got), want, dtype, n)
+
+
 def valid_idx(B, H, N, p, L, S, seed):
     geo = O.Geometry(N, p, L, S).check()
     r = np.random.default_rng(seed).random((B, H, N + geo.R)).astype(np.float32)
