@@ -57,7 +57,9 @@ struct Layout {
   static constexpr int V = K + kStages * KB * TILE;  // stage s at V + s * KB * TILE
   static constexpr int BAR = V + v_stages<D>() * KB * TILE;
   // floats [.][128 rows]: XM [2] the max block j used, at j & 1; XC [4][2 halves] the halves'
-  // maxima of block j, at j & 3; XL, XE [4 warps] partial row sums and the max each is relative to
+  // maxima of block j, at j & 3 (a warp can store block j + 2's maximum before its partner has
+  // read block j's, but not block j + 4's: that needs PV_{j+1}, after the partner's arrival);
+  // XL, XE [4 warps] partial row sums and the max each is relative to
   static constexpr int XM = BAR + 256;
   static constexpr int XC = XM + 2 * 128 * 4;
   static constexpr int XL = XC + 8 * 128 * 4;
