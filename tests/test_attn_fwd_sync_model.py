@@ -1,0 +1,216 @@
+"""A randomised model of the attention forward's synchronisation (csrc/attn_tc_fwd.cu), run on
+the CPU. It checks the protocol, not the kernel: every wait and barrier of the kernel's roles,
+for one lane quarter, with every interleaving a seeded scheduler picks.
+
+Modelled:
+  - mbarriers with phase-parity waits. A wait passes when the phase of the other parity is the
+    current one, exactly as the hardware test does. So a waiter two phases behind passes on a
+    stale phase, and the model reports that.
+  - The tensor core as one in-order queue, each commit arriving once the operations before it
+    are done, and TMA loads landing in issue order.
+  - Named barriers as phases of a fixed count. An arrival that joins an open phase with another
+    tag or count is an error, and so is a barrier that never completes (a deadlock).
+  - The shared-memory slots that carry the block maxima between warps.
+Roles: the TMA thread (independent K and V rings), the S and PV issuers, and two softmax sets
+(even and odd key blocks) of two warps each (the two key halves of a block).
+"""
+import random
+
+import pytest
+
+
+class MBar:
+    def __init__(self, count):
+        self.count, self.pending, self.phase = count, 0, 0  # phase = completed phases
+
+    def arrive(self):
+        self.pending += 1
+        assert self.pending <= self.count
+        if self.pending == self.count:
+            self.pending, self.phase = 0, self.phase + 1
+
+    def passes(self, parity):  # mbarrier.try_wait.parity
+        return (self.phase & 1) != parity
+
+
+class Named:
+    def __init__(self):
+        self.phase, self.n, self.tag, self.count = 0, 0, None, None
+
+    def join(self, tag, threads):
+        if self.n == 0:
+            self.tag, self.count = tag, threads
+        assert (self.tag, self.count) == (tag, threads), "arrival joins another phase"
+        self.n += 32
+        ph = self.phase
+        if self.n == self.count:
+            self.n, self.phase = 0, self.phase + 1
+        return ph
+
+
+class Protocol:
+    """One CTA of the forward at nkb key blocks. `xc_slots` and `epilogue_on_last_pv` select the
+    design (4 slots and a dedicated last-PV barrier) or a flawed alternative."""
+
+    def __init__(self, nkb, seed, kStV=2, xc_slots=4, epilogue_on_last_pv=True):
+        self.nkb, self.R, self.kStV = nkb, random.Random(seed), kStV
+        self.kStages = self.kSBuf = 3
+        self.xc_slots, self.fin_bar = xc_slots, epilogue_on_last_pv
+        self.q = MBar(1)
+        self.K = [MBar(1) for _ in range(3)]
+        self.V = [MBar(1) for _ in range(kStV)]
+        self.KF = [MBar(1) for _ in range(3)]
+        self.VF = [MBar(1) for _ in range(kStV)]
+        self.SB = [MBar(1) for _ in range(3)]
+        self.PB = [MBar(2) for _ in range(3)]  # the set's two warps of this lane quarter
+        self.PVB = [MBar(1) for _ in range(3)]
+        self.FIN = MBar(1)
+        self.named = [Named(), Named()]  # the incoming barrier of set 0 and of set 1
+        self.epi = Named()
+        self.xm, self.xc = {}, {}
+        self.tensor, self.tma = [], []
+        self.S_done, self.PV_done, self.P_written = set(), set(), {}
+
+    def seen(self, bar, phases):  # a wait that passed must see at least this many phases
+        assert bar.phase >= phases, "a wait passed on a stale phase"
+
+    def tma_thread(self):
+        yield lambda: True
+        self.tma.append(("q", 0))
+        nk = nv = 0
+        ks, kv = self.kStages, self.kStV
+        k_ok = lambda: nk < self.nkb and (nk < ks or self.KF[nk % ks].passes(((nk - ks) // ks) & 1))
+        v_ok = lambda: nv < nk and (nv < kv or self.VF[nv % kv].passes(((nv - kv) // kv) & 1))
+        while nk < self.nkb or nv < self.nkb:
+            if not (k_ok() or v_ok()):
+                yield lambda: k_ok() or v_ok()
+                continue
+            if k_ok():
+                if nk >= ks:
+                    self.seen(self.KF[nk % ks], (nk - ks) // ks + 1)
+                    assert nk - ks in self.S_done, "K stage reloaded before S read it"
+                self.tma.append(("k", nk))
+                nk += 1
+            if v_ok():
+                if nv >= kv:
+                    self.seen(self.VF[nv % kv], (nv - kv) // kv + 1)
+                    assert nv - kv in self.PV_done, "V stage reloaded before PV read it"
+                self.tma.append(("v", nv))
+                nv += 1
+            yield lambda: True
+
+    def s_issuer(self):
+        yield lambda: self.q.passes(0)
+        for n in range(self.nkb):
+            yield lambda n=n: self.K[n % 3].passes((n // 3) & 1)
+            self.seen(self.K[n % 3], n // 3 + 1)
+            if n >= 3:
+                yield lambda n=n: self.PVB[n % 3].passes(((n // 3) - 1) & 1)
+                self.seen(self.PVB[n % 3], n // 3)
+                assert n - 3 in self.PV_done, "S written over a P that PV has not read"
+            self.tensor += [("S", n), ("commit", self.SB[n % 3]), ("commit", self.KF[n % 3])]
+
+    def pv_issuer(self):
+        for j in range(self.nkb):
+            yield lambda j=j: self.PB[j % 3].passes((j // 3) & 1)
+            self.seen(self.PB[j % 3], j // 3 + 1)
+            assert self.P_written.get(j) == 2
+            yield lambda j=j: self.V[j % self.kStV].passes((j // self.kStV) & 1)
+            self.seen(self.V[j % self.kStV], j // self.kStV + 1)
+            self.tensor += [("PV", j), ("commit", self.PVB[j % 3]),
+                            ("commit", self.VF[j % self.kStV])]
+        self.tensor.append(("commit", self.FIN))
+
+    def softmax_warp(self, st, half):
+        for j in range(st, self.nkb, 2):
+            yield lambda j=j: self.SB[j % 3].passes((j // 3) & 1)
+            self.seen(self.SB[j % 3], j // 3 + 1)
+            assert j in self.S_done
+            yield lambda: True  # load S_j, take this half's max
+            self.xc[(j % self.xc_slots, half)] = j
+            ph = self.named[st].join(j, 64 if j == 0 else 128)
+            yield lambda ph=ph, st=st: self.named[st].phase > ph
+            assert self.xc[(j % self.xc_slots, half ^ 1)] == j, "the other half's max was overwritten"
+            if j > 0:
+                assert self.xm[(j - 1) & 1] == j - 1, "the max of block j - 1 was overwritten"
+            yield lambda: True
+            if j + 1 < self.nkb:
+                if half == 0:
+                    self.xm[j & 1] = j
+                self.named[st ^ 1].join(j + 1, 128)
+            if j > 0 and self.R.random() < 0.3:  # a row max grew: rescale O after PV_{j-1}
+                yield lambda j=j: self.PVB[(j - 1) % 3].passes(((j - 1) // 3) & 1)
+                self.seen(self.PVB[(j - 1) % 3], (j - 1) // 3 + 1)
+                assert j - 1 in self.PV_done and j not in self.PV_done
+            yield lambda: True
+            self.P_written[j] = self.P_written.get(j, 0) + 1
+            self.PB[j % 3].arrive()
+        if self.fin_bar:
+            yield lambda: self.FIN.passes(0)
+            self.seen(self.FIN, 1)
+        else:  # the flawed alternative: the last block's own PV barrier
+            last = self.nkb - 1
+            yield lambda: self.PVB[last % 3].passes((last // 3) & 1)
+            self.seen(self.PVB[last % 3], last // 3 + 1)
+        assert self.nkb - 1 in self.PV_done, "epilogue before the last PV"
+        ph = self.epi.join("epilogue", 128)
+        yield lambda ph=ph: self.epi.phase > ph
+
+    def run(self):
+        actors = [self.tma_thread(), self.s_issuer(), self.pv_issuer()] + [
+            self.softmax_warp(st, h) for st in (0, 1) for h in (0, 1)]
+        waiting = [next(a) for a in actors]
+        done = [False] * len(actors)
+        for _ in range(200000):
+            if all(done) and not self.tensor and not self.tma:
+                return
+            ready = [("actor", i) for i, a in enumerate(actors) if not done[i] and waiting[i]()]
+            if self.tensor:
+                ready.append(("tensor", 0))
+            if self.tma:
+                ready.append(("tma", 0))
+            assert ready, "deadlock"
+            kind, i = self.R.choice(ready)
+            if kind == "tensor":
+                op, x = self.tensor.pop(0)
+                if op == "S":
+                    self.S_done.add(x)
+                elif op == "PV":
+                    assert self.P_written.get(x) == 2
+                    self.PV_done.add(x)
+                else:
+                    x.arrive()
+            elif kind == "tma":
+                op, n = self.tma.pop(0)
+                {"q": lambda: self.q, "k": lambda: self.K[n % 3], "v": lambda: self.V[n % self.kStV]}[op]().arrive()
+            else:
+                try:
+                    waiting[i] = next(actors[i])
+                except StopIteration:
+                    done[i] = True
+        raise AssertionError("livelock")
+
+
+@pytest.mark.parametrize("kStV", [2, 3])  # V stages at d = 128 and d = 64
+@pytest.mark.parametrize("nkb", list(range(1, 12)) + [31, 64])
+def test_forward_protocol_never_deadlocks_or_reads_stale(nkb, kStV):
+    for seed in range(40):
+        Protocol(nkb, seed, kStV).run()
+
+
+def test_model_catches_the_epilogue_on_a_per_buffer_barrier():
+    """The set that does not own the last block can reach the epilogue while the last block's
+    PV barrier is two phases behind: its parity wait would pass at once."""
+    with pytest.raises(AssertionError, match="stale phase"):
+        for nkb in range(2, 12):
+            for seed in range(200):
+                Protocol(nkb, seed, epilogue_on_last_pv=False).run()
+
+
+def test_model_catches_two_slots_for_the_halves_maxima():
+    """With the halves' block maxima in two slots, a warp can store block j + 2's max before its
+    partner has read block j's."""
+    with pytest.raises(AssertionError, match="other half"):
+        for nkb in range(3, 16):
+            for seed in range(200):
+                Protocol(nkb, seed, xc_slots=2).run()
