@@ -1,0 +1,182 @@
+"""A randomised model of the synchronisation of the one-pass attention backward at d = 64
+(`attn_bwd_fused64_tc` in csrc/attn_tc_bwd.cu), run on the CPU. It checks the protocol, not the
+kernel: the TMA thread, the MMA issuer, the compute warps (two stand for all of them) and the
+copy engine that adds dQ, under random interleavings.
+
+Per 128-query step j the issuer runs dV(j), S^T(j+1), dP^T(j+1), dQ(j), dK(j) on one in-order
+tensor queue. Tensor memory holds S^T (then P^T over it), dP^T, and two dQ buffers; shared
+memory holds two Q/dO stages, one dS^T tile and one dQ staging tile. The model asserts that no
+MMA or warp overwrites one of them before its last reader is done, that every parity wait which
+passes sees the phase it means, and that every named barrier completes.
+"""
+import random
+
+import pytest
+
+from sync_model import MBar, Named, schedule
+
+WARPS = 2  # compute warps modelled; every per-warp barrier counts them
+
+
+class Fused64:
+    def __init__(self, nit, seed, staging_wait=True, dqr_wait=True):
+        self.nit, self.R = nit, random.Random(seed)
+        self.staging_wait, self.dqr_wait = staging_wait, dqr_wait
+        self.kv = MBar(1)
+        self.st = [MBar(1), MBar(1)]
+        self.stfree = [MBar(1), MBar(1)]
+        self.s, self.dp, self.vdone, self.kdone = MBar(1), MBar(1), MBar(1), MBar(1)
+        self.p, self.ds = MBar(WARPS), MBar(WARPS)
+        self.dq = [MBar(1), MBar(1)]
+        self.dqr = [MBar(WARPS), MBar(WARPS)]
+        self.sync = Named()  # the compute warps' named barrier around the staging
+        self.tensor, self.tma, self.copy = [], [], []
+        self.done = set()             # ("S", j), ("dP", j), ("dV", j), ("dQ", j), ("dK", j)
+        self.loaded = set()           # stages loaded, by step
+        self.s_cols = None            # what the S^T columns hold: ("S", j) or ("P", j)
+        self.p_read = {}              # warps that have read S^T(j) / dP^T(j) / dQ(j)
+        self.dp_read, self.dq_read = {}, {}
+        self.ds_tile = None           # the step whose dS^T the tile holds
+        self.staging = None           # the step whose sigma dQ the staging tile holds
+        self.staging_reads = 0        # reductions issued that have not read the staging yet
+        self.added = []               # steps the copy engine added, in order
+
+    # ---- roles
+    def tma_thread(self):
+        yield lambda: True
+        self.tma.append(("kv", 0))
+        for j in range(self.nit):
+            if j >= 2:
+                yield lambda j=j: self.stfree[j & 1].passes(((j - 2) >> 1) & 1)
+                assert self.stfree[j & 1].phase >= (j - 2) // 2 + 1, "stale stage-free pass"
+                assert ("dK", j - 2) in self.done, "stage reloaded under its readers"
+                assert self.dp_read.get(j - 2) == WARPS, "stage reloaded before the warps read its vectors"
+            self.tma.append(("st", j))
+
+    def issuer(self):
+        yield lambda: self.kv.passes(0) and self.st[0].passes(0)
+        self.tensor += [("S", 0), ("commit", self.s), ("dP", 0), ("commit", self.dp)]
+        for j in range(self.nit):
+            yield lambda j=j: self.p.passes(j & 1)
+            assert self.p.phase >= j + 1 and self.s_cols == ("P", j)
+            self.tensor += [("dV", j), ("commit", self.vdone)]
+            if j + 1 < self.nit:
+                n = j + 1
+                yield lambda n=n: self.st[n & 1].passes((n >> 1) & 1)
+                assert self.st[n & 1].phase >= n // 2 + 1
+                yield lambda j=j: self.vdone.passes(j & 1)
+                assert self.vdone.phase >= j + 1
+                self.tensor += [("S", n), ("commit", self.s)]
+            yield lambda j=j: self.ds.passes(j & 1)
+            assert self.ds.phase >= j + 1 and self.ds_tile == j
+            if j + 1 < self.nit:
+                self.tensor += [("dP", j + 1), ("commit", self.dp)]
+            if j >= 2 and self.dqr_wait:
+                yield lambda j=j: self.dqr[j & 1].passes(((j - 2) >> 1) & 1)
+                assert self.dqr[j & 1].phase >= (j - 2) // 2 + 1
+            self.tensor += [("dQ", j), ("commit", self.dq[j & 1]),
+                            ("dK", j), ("commit", self.stfree[j & 1]), ("commit", self.kdone)]
+
+    def compute_warp(self, w):
+        def flush(i):
+            yield lambda i=i: self.dq[i & 1].passes((i >> 1) & 1)
+            assert self.dq[i & 1].phase >= i // 2 + 1 and ("dQ", i) in self.done
+            self.dq_read[i] = self.dq_read.get(i, 0) + 1
+            self.dqr[i & 1].arrive()
+            if w == 0 and self.staging_wait:  # bulk_wait_read_all: the last reduction has read it
+                yield lambda: self.staging_reads == 0
+            ph = self.sync.join(("stage", i), 32 * WARPS)
+            yield lambda ph=ph: self.sync.phase > ph
+            assert self.staging_reads == 0, "staging overwritten before the copy engine read it"
+            self.staging = i
+            ph = self.sync.join(("issue", i), 32 * WARPS)
+            yield lambda ph=ph: self.sync.phase > ph
+            if w == 0:
+                self.staging_reads += 1
+                self.copy.append(i)
+
+        for j in range(self.nit):
+            yield lambda j=j: self.s.passes(j & 1) and self.st[j & 1].passes((j >> 1) & 1)
+            assert self.s.phase >= j + 1 and self.st[j & 1].phase >= j // 2 + 1
+            assert self.s_cols in (("S", j), ("P", j)) and j in self.loaded
+            self.p_read[j] = self.p_read.get(j, 0) + 1
+            if self.p_read[j] == WARPS:
+                self.s_cols = ("P", j)  # every warp's columns now hold P^T(j)
+            self.p.arrive()
+            yield lambda j=j: self.dp.passes(j & 1) and (j == 0 or self.kdone.passes((j - 1) & 1))
+            assert ("dP", j) in self.done and (j == 0 or ("dK", j - 1) in self.done)
+            assert ("dQ", j - 1) in self.done or j == 0, "dS^T overwritten under dQ"
+            self.dp_read[j] = self.dp_read.get(j, 0) + 1
+            self.ds_tile = j
+            self.ds.arrive()
+            if j > 0:
+                yield from flush(j - 1)
+        yield from flush(self.nit - 1)
+        yield lambda: self.kdone.passes((self.nit - 1) & 1)
+        assert ("dK", self.nit - 1) in self.done
+        if w == 0:  # bulk_wait_all
+            yield lambda: not self.copy
+
+    # ---- the units that complete work in order
+    def on_tensor(self, item):
+        op, x = item
+        if op == "commit":
+            x.arrive()
+            return
+        j = x
+        if op == "S":
+            assert j == 0 or ("dV", j - 1) in self.done, "S^T over a P^T that dV has not read"
+            assert j == 0 or self.p_read.get(j - 1) == WARPS
+            self.s_cols = ("S", j)
+        elif op == "dP":
+            assert j == 0 or self.dp_read.get(j - 1) == WARPS, "dP^T overwritten before the warps read it"
+        elif op == "dV":
+            assert self.s_cols == ("P", j)
+        elif op == "dQ":
+            assert self.ds_tile == j
+            assert j < 2 or self.dq_read.get(j - 2) == WARPS, "dQ buffer overwritten before the warps read it"
+        elif op == "dK":
+            assert self.ds_tile == j
+        self.done.add((op, j))
+
+    def on_tma(self, item):
+        op, j = item
+        if op == "kv":
+            self.kv.arrive()
+        else:
+            self.loaded.add(j)
+            self.st[j & 1].arrive()
+
+    def on_copy(self, i):
+        assert self.staging == i, "the copy engine read another step's staging"
+        self.staging_reads -= 1
+        self.added.append(i)
+
+    def run(self):
+        actors = [self.tma_thread(), self.issuer()] + [self.compute_warp(w) for w in range(WARPS)]
+        schedule(self.R, actors, [(self.tensor, self.on_tensor), (self.tma, self.on_tma),
+                                  (self.copy, self.on_copy)])
+        assert self.added == list(range(self.nit)), "a step's dQ was not added exactly once"
+
+
+@pytest.mark.parametrize("nit", list(range(1, 10)) + [24, 48])
+def test_fused64_protocol(nit):
+    for seed in range(60):
+        Fused64(nit, seed).run()
+
+
+def test_model_catches_a_staging_overwrite():
+    """Without the wait for the copy engine to have read the staging, a warp can overwrite it."""
+    with pytest.raises(AssertionError, match="staging"):
+        for nit in range(2, 10):
+            for seed in range(300):
+                Fused64(nit, seed, staging_wait=False).run()
+
+
+def test_dq_buffer_wait_is_implied_by_the_step_order():
+    """The issuer's wait for the warps to have read dQ(j - 2) before dQ(j) is a guard the step
+    order already implies: dQ(j) follows dS^T(j), which every warp writes only after its flush
+    of step j - 2 has read dQ(j - 2). Without the wait the model finds no overwrite."""
+    for nit in range(3, 10):
+        for seed in range(100):
+            Fused64(nit, seed, dqr_wait=False).run()

@@ -18,34 +18,7 @@ import random
 
 import pytest
 
-
-class MBar:
-    def __init__(self, count):
-        self.count, self.pending, self.phase = count, 0, 0  # phase = completed phases
-
-    def arrive(self):
-        self.pending += 1
-        assert self.pending <= self.count
-        if self.pending == self.count:
-            self.pending, self.phase = 0, self.phase + 1
-
-    def passes(self, parity):  # mbarrier.try_wait.parity
-        return (self.phase & 1) != parity
-
-
-class Named:
-    def __init__(self):
-        self.phase, self.n, self.tag, self.count = 0, 0, None, None
-
-    def join(self, tag, threads):
-        if self.n == 0:
-            self.tag, self.count = tag, threads
-        assert (self.tag, self.count) == (tag, threads), "arrival joins another phase"
-        self.n += 32
-        ph = self.phase
-        if self.n == self.count:
-            self.n, self.phase = 0, self.phase + 1
-        return ph
+from sync_model import MBar, Named, schedule
 
 
 class Protocol:
@@ -156,39 +129,24 @@ class Protocol:
         ph = self.epi.join("epilogue", 128)
         yield lambda ph=ph: self.epi.phase > ph
 
+    def on_tensor(self, item):
+        op, x = item
+        if op == "S":
+            self.S_done.add(x)
+        elif op == "PV":
+            assert self.P_written.get(x) == 2
+            self.PV_done.add(x)
+        else:
+            x.arrive()
+
+    def on_tma(self, item):
+        op, n = item
+        {"q": lambda: self.q, "k": lambda: self.K[n % 3], "v": lambda: self.V[n % self.kStV]}[op]().arrive()
+
     def run(self):
         actors = [self.tma_thread(), self.s_issuer(), self.pv_issuer()] + [
             self.softmax_warp(st, h) for st in (0, 1) for h in (0, 1)]
-        waiting = [next(a) for a in actors]
-        done = [False] * len(actors)
-        for _ in range(200000):
-            if all(done) and not self.tensor and not self.tma:
-                return
-            ready = [("actor", i) for i, a in enumerate(actors) if not done[i] and waiting[i]()]
-            if self.tensor:
-                ready.append(("tensor", 0))
-            if self.tma:
-                ready.append(("tma", 0))
-            assert ready, "deadlock"
-            kind, i = self.R.choice(ready)
-            if kind == "tensor":
-                op, x = self.tensor.pop(0)
-                if op == "S":
-                    self.S_done.add(x)
-                elif op == "PV":
-                    assert self.P_written.get(x) == 2
-                    self.PV_done.add(x)
-                else:
-                    x.arrive()
-            elif kind == "tma":
-                op, n = self.tma.pop(0)
-                {"q": lambda: self.q, "k": lambda: self.K[n % 3], "v": lambda: self.V[n % self.kStV]}[op]().arrive()
-            else:
-                try:
-                    waiting[i] = next(actors[i])
-                except StopIteration:
-                    done[i] = True
-        raise AssertionError("livelock")
+        schedule(self.R, actors, [(self.tensor, self.on_tensor), (self.tma, self.on_tma)])
 
 
 @pytest.mark.parametrize("kStV", [2, 3])  # V stages at d = 128 and d = 64
