@@ -1,13 +1,18 @@
-"""A randomised model of the synchronisation of the one-pass attention backward at d = 64
-(`attn_bwd_fused64_tc` in csrc/attn_tc_bwd.cu), run on the CPU. It checks the protocol, not the
-kernel: the TMA thread, the MMA issuer, the compute warps (two stand for all of them) and the
-copy engine that adds dQ, under random interleavings.
+"""Randomised models of the synchronisation of the one-pass attention backward kernels in
+csrc/attn_tc_bwd.cu, run on the CPU. They check the protocols, not the kernels: the TMA thread,
+the MMA issuers, the compute warps (two stand for all of them) and, at d = 64, the copy engine
+that adds dQ, under random interleavings.
 
-Per 128-query step j the issuer runs dV(j), S^T(j+1), dP^T(j+1), dQ(j), dK(j) on one in-order
+d = 64 (`attn_bwd_fused64_tc`):
+per 128-query step j the issuer runs dV(j), S^T(j+1), dP^T(j+1), dQ(j), dK(j) on one in-order
 tensor queue. Tensor memory holds S^T (then P^T over it), dP^T, and two dQ buffers; shared
 memory holds two Q/dO stages, one dS^T tile and one dQ staging tile. The model asserts that no
 MMA or warp overwrites one of them before its last reader is done, that every parity wait which
 passes sees the phase it means, and that every named barrier completes.
+
+d = 128 (`attn_bwd_fused_tc`): per 64-query step one issuer runs S^T and dP^T, the other the
+accumulations dV, dK and dQ^T, on the same in-order tensor queue. S^T/dP^T, P^T, dS^T and dQ^T
+are single buffers; the Q/dO stages form a ring of three.
 """
 import random
 
@@ -180,3 +185,108 @@ def test_dq_buffer_wait_is_implied_by_the_step_order():
     for nit in range(3, 10):
         for seed in range(100):
             Fused64(nit, seed, dqr_wait=False).run()
+
+
+class Fused128:
+    def __init__(self, nit, seed, stages=3, sfree_wait=True):
+        self.nit, self.R, self.ks = nit, random.Random(seed), stages
+        self.sfree_wait = sfree_wait
+        self.kv = MBar(1)
+        self.st = [MBar(1) for _ in range(stages)]
+        self.stfree = [MBar(1) for _ in range(stages)]
+        self.s, self.acc = MBar(1), MBar(1)
+        self.sfree, self.p = MBar(WARPS), MBar(WARPS)
+        self.tensor, self.tma = [], []
+        self.done, self.loaded = set(), set()
+        self.sdp = None          # the step whose S^T/dP^T the columns hold
+        self.sdp_read = {}       # warps that have read S^T/dP^T(n)
+        self.pds = None          # the step whose P^T and dS^T the warps last wrote
+        self.pds_writes = {}
+        self.dqt = None          # the step whose dQ^T the columns hold
+        self.dqt_read = {}
+
+    def tma_thread(self):
+        yield lambda: True
+        self.tma.append(("kv", 0))
+        for it in range(self.nit):
+            if it >= self.ks:
+                n = it - self.ks
+                yield lambda it=it, n=n: self.stfree[it % self.ks].passes((n // self.ks) & 1)
+                assert self.stfree[it % self.ks].phase >= n // self.ks + 1, "stale stage-free pass"
+                assert ("acc", n) in self.done and self.sdp_read.get(n) == WARPS
+            self.tma.append(("st", it))
+
+    def s_issuer(self):
+        yield lambda: self.kv.passes(0)
+        for n in range(self.nit):
+            yield lambda n=n: self.st[n % self.ks].passes((n // self.ks) & 1) and (
+                n == 0 or not self.sfree_wait or self.sfree.passes((n - 1) & 1))
+            assert self.st[n % self.ks].phase >= n // self.ks + 1 and n in self.loaded
+            assert n == 0 or not self.sfree_wait or self.sfree.phase >= n
+            self.tensor += [("S", n), ("commit", self.s)]
+
+    def acc_issuer(self):
+        for it in range(self.nit):
+            yield lambda it=it: self.p.passes(it & 1)
+            assert self.p.phase >= it + 1 and self.pds_writes.get(it) == WARPS
+            self.tensor += [("acc", it), ("commit", self.acc), ("commit", self.stfree[it % self.ks])]
+
+    def compute_warp(self, w):
+        for it in range(self.nit):
+            yield lambda it=it: self.s.passes(it & 1) and self.st[it % self.ks].passes((it // self.ks) & 1)
+            assert self.s.phase >= it + 1 and self.sdp == it and it in self.loaded
+            self.sdp_read[it] = self.sdp_read.get(it, 0) + 1
+            self.sfree.arrive()
+            if it > 0:
+                yield lambda it=it: self.acc.passes((it - 1) & 1)
+                assert self.acc.phase >= it and ("acc", it - 1) in self.done
+                assert self.dqt == it - 1
+                self.dqt_read[it - 1] = self.dqt_read.get(it - 1, 0) + 1
+            assert it == 0 or ("acc", it - 1) in self.done, "P^T or dS^T overwritten under its MMAs"
+            self.pds_writes[it] = self.pds_writes.get(it, 0) + 1
+            self.pds = it
+            self.p.arrive()
+        yield lambda: self.acc.passes((self.nit - 1) & 1)
+        assert ("acc", self.nit - 1) in self.done and self.dqt == self.nit - 1
+
+    def on_tensor(self, item):
+        op, x = item
+        if op == "commit":
+            x.arrive()
+            return
+        if op == "S":
+            assert x == 0 or self.sdp_read.get(x - 1) == WARPS, "S^T/dP^T overwritten before the warps read it"
+            self.sdp = x
+        else:
+            assert self.pds == x and self.pds_writes.get(x) == WARPS
+            assert x == 0 or self.dqt_read.get(x - 1) == WARPS, "dQ^T overwritten before the warps read it"
+            self.dqt = x
+        self.done.add((op, x))
+
+    def on_tma(self, item):
+        op, j = item
+        if op == "kv":
+            self.kv.arrive()
+        else:
+            self.loaded.add(j)
+            self.st[j % self.ks].arrive()
+
+    def run(self):
+        actors = [self.tma_thread(), self.s_issuer(), self.acc_issuer()] + [
+            self.compute_warp(w) for w in range(WARPS)]
+        schedule(self.R, actors, [(self.tensor, self.on_tensor), (self.tma, self.on_tma)])
+
+
+@pytest.mark.parametrize("nit", list(range(1, 10)) + [32, 128])
+def test_fused128_protocol(nit):
+    for seed in range(60):
+        Fused128(nit, seed).run()
+
+
+def test_model_catches_s_over_unread_scores():
+    """Without the S issuer's wait for the warps to have read S^T/dP^T(n - 1), S^T(n) can
+    overwrite them."""
+    with pytest.raises(AssertionError, match="before the warps read it"):
+        for nit in range(2, 10):
+            for seed in range(300):
+                Fused128(nit, seed, sfree_wait=False).run()
