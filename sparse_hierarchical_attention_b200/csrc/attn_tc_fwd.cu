@@ -22,8 +22,8 @@
 //    dO . (O error), which is large on coarse rows whose dO sums thousands of tokens.
 //  - The running max is updated lazily: O is rescaled only when a row's max grows by more than
 //    2^kGrow (2^32), which keeps every exponent bounded and skips most rescales, each of which
-//    waits for the previous PV. P <= 2^32, l <= 2^32 S and |O| <= 2^32 S max|V| stay far from
-//    the fp32 range for any S and |V| < 2^70. The max of block j
+//    waits for the previous PV. P <= 2^32, l <= 2^32 S and |O| <= 2^32 S max|V| stay inside the
+//    fp32 range while S max|V| < 2^96 (S = 2^20 rows leave |V| up to 2^76). The max of block j
 //    goes from one set to the other through shared memory and a named barrier per set and lane
 //    quarter, on which the set of block j syncs and the set of block j - 1 arrives; the same
 //    barrier swaps the two halves' block maxima. Each warp keeps its own row sum, relative to
