@@ -25,8 +25,11 @@ class Protocol:
     """One CTA of the forward at nkb key blocks. `xc_slots` and `epilogue_on_last_pv` select the
     design (4 slots and a dedicated last-PV barrier) or a flawed alternative."""
 
-    def __init__(self, nkb, seed, kStV=2, xc_slots=4, epilogue_on_last_pv=True):
+    def __init__(self, nkb, seed, kStV=2, xc_slots=4, epilogue_on_last_pv=True, abort_after=None):
         self.nkb, self.R, self.kStV = nkb, random.Random(seed), kStV
+        self.aborted = False
+        # a wait runs out after this many ticks of a clock the scheduler advances at random
+        self.clock = [None] * abort_after if abort_after else []
         self.kStages = self.kSBuf = 3
         self.xc_slots, self.fin_bar = xc_slots, epilogue_on_last_pv
         self.q = MBar(1)
@@ -47,6 +50,17 @@ class Protocol:
     def seen(self, bar, phases):  # a wait that passed must see at least this many phases
         assert bar.phase >= phases, "a wait passed on a stale phase"
 
+    def wait(self, cond):
+        """A bounded mbarrier wait: passes once cond() holds. After any wait has run out
+        (self.aborted) every wait returns at once, true only if its phase is already complete."""
+        yield lambda: cond() or self.aborted
+        return cond()
+
+    def drain(self):  # mma_drain: a commit of the issuer's own MMAs, then a wait for it
+        bar = MBar(1)
+        self.tensor.append(("commit", bar))
+        yield lambda: bar.phase >= 1
+
     def tma_thread(self):
         yield lambda: True
         self.tma.append(("q", 0))
@@ -56,7 +70,9 @@ class Protocol:
         v_ok = lambda: nv < nk and (nv < kv or self.VF[nv % kv].passes(((nv - kv) // kv) & 1))
         while nk < self.nkb or nv < self.nkb:
             if not (k_ok() or v_ok()):
-                yield lambda: k_ok() or v_ok()
+                yield lambda: k_ok() or v_ok() or self.aborted
+                if not (k_ok() or v_ok()):
+                    break  # no stage freed and the CTA has aborted
                 continue
             if k_ok():
                 if nk >= ks:
@@ -71,35 +87,53 @@ class Protocol:
                 self.tma.append(("v", nv))
                 nv += 1
             yield lambda: True
+        yield lambda: not self.tma  # every issued load lands before the thread leaves
 
     def s_issuer(self):
-        yield lambda: self.q.passes(0)
-        for n in range(self.nkb):
-            yield lambda n=n: self.K[n % 3].passes((n // 3) & 1)
-            self.seen(self.K[n % 3], n // 3 + 1)
-            if n >= 3:
-                yield lambda n=n: self.PVB[n % 3].passes(((n // 3) - 1) & 1)
-                self.seen(self.PVB[n % 3], n // 3)
-                assert n - 3 in self.PV_done, "S written over a P that PV has not read"
+        ok = yield from self.wait(lambda: self.q.passes(0))
+        n = 0
+        while n < self.nkb and ok:
+            ok = yield from self.wait(lambda n=n: self.K[n % 3].passes((n // 3) & 1))
+            if ok:
+                self.seen(self.K[n % 3], n // 3 + 1)
+            if ok and n >= 3:
+                ok = yield from self.wait(lambda n=n: self.PVB[n % 3].passes(((n // 3) - 1) & 1))
+                if ok:
+                    self.seen(self.PVB[n % 3], n // 3)
+                    assert n - 3 in self.PV_done, "S written over a P that PV has not read"
+            if not ok:
+                break
             self.tensor += [("S", n), ("commit", self.SB[n % 3]), ("commit", self.KF[n % 3])]
+            n += 1
+        yield from self.drain()
 
     def pv_issuer(self):
-        for j in range(self.nkb):
-            yield lambda j=j: self.PB[j % 3].passes((j // 3) & 1)
-            self.seen(self.PB[j % 3], j // 3 + 1)
-            assert self.P_written.get(j) == 2
-            yield lambda j=j: self.V[j % self.kStV].passes((j // self.kStV) & 1)
+        j = 0
+        while j < self.nkb:
+            ok = yield from self.wait(lambda j=j: self.PB[j % 3].passes((j // 3) & 1))
+            if ok:
+                self.seen(self.PB[j % 3], j // 3 + 1)
+                assert self.P_written.get(j) == 2
+                ok = yield from self.wait(lambda j=j: self.V[j % self.kStV].passes((j // self.kStV) & 1))
+            if not ok:
+                break
             self.seen(self.V[j % self.kStV], j // self.kStV + 1)
             self.tensor += [("PV", j), ("commit", self.PVB[j % 3]),
                             ("commit", self.VF[j % self.kStV])]
-        self.tensor.append(("commit", self.FIN))
+            j += 1
+        if j == self.nkb:
+            self.tensor.append(("commit", self.FIN))
+        yield from self.drain()
 
     def softmax_warp(self, st, half):
+        ok = True
         for j in range(st, self.nkb, 2):
-            yield lambda j=j: self.SB[j % 3].passes((j // 3) & 1)
-            self.seen(self.SB[j % 3], j // 3 + 1)
-            assert j in self.S_done
-            yield lambda: True  # load S_j, take this half's max
+            if ok:
+                ok = yield from self.wait(lambda j=j: self.SB[j % 3].passes((j // 3) & 1))
+                if ok:
+                    self.seen(self.SB[j % 3], j // 3 + 1)
+                    assert j in self.S_done
+            yield lambda: True  # load S_j (when ok), take this half's max
             self.xc[(j % self.xc_slots, half)] = j
             ph = self.named[st].join(j, 64 if j == 0 else 128)
             yield lambda ph=ph, st=st: self.named[st].phase > ph
@@ -111,21 +145,27 @@ class Protocol:
                 if half == 0:
                     self.xm[j & 1] = j
                 self.named[st ^ 1].join(j + 1, 128)
-            if j > 0 and self.R.random() < 0.3:  # a row max grew: rescale O after PV_{j-1}
-                yield lambda j=j: self.PVB[(j - 1) % 3].passes(((j - 1) // 3) & 1)
-                self.seen(self.PVB[(j - 1) % 3], (j - 1) // 3 + 1)
-                assert j - 1 in self.PV_done and j not in self.PV_done
+            if j > 0 and self.R.random() < 0.3 and ok:  # a row max grew: rescale O after PV_{j-1}
+                ok = yield from self.wait(lambda j=j: self.PVB[(j - 1) % 3].passes(((j - 1) // 3) & 1))
+                if ok:
+                    self.seen(self.PVB[(j - 1) % 3], (j - 1) // 3 + 1)
+                    assert j - 1 in self.PV_done and j not in self.PV_done
             yield lambda: True
-            self.P_written[j] = self.P_written.get(j, 0) + 1
-            self.PB[j % 3].arrive()
-        if self.fin_bar:
-            yield lambda: self.FIN.passes(0)
-            self.seen(self.FIN, 1)
-        else:  # the flawed alternative: the last block's own PV barrier
-            last = self.nkb - 1
-            yield lambda: self.PVB[last % 3].passes((last // 3) & 1)
-            self.seen(self.PVB[last % 3], last // 3 + 1)
-        assert self.nkb - 1 in self.PV_done, "epilogue before the last PV"
+            if ok:
+                self.P_written[j] = self.P_written.get(j, 0) + 1
+                self.PB[j % 3].arrive()
+        if ok:
+            if self.fin_bar:
+                ok = yield from self.wait(lambda: self.FIN.passes(0))
+                if ok:
+                    self.seen(self.FIN, 1)
+            else:  # the flawed alternative: the last block's own PV barrier
+                last = self.nkb - 1
+                ok = yield from self.wait(lambda: self.PVB[last % 3].passes((last // 3) & 1))
+                if ok:
+                    self.seen(self.PVB[last % 3], last // 3 + 1)
+            if ok:
+                assert self.nkb - 1 in self.PV_done, "epilogue before the last PV"
         ph = self.epi.join("epilogue", 128)
         yield lambda ph=ph: self.epi.phase > ph
 
@@ -146,7 +186,12 @@ class Protocol:
     def run(self):
         actors = [self.tma_thread(), self.s_issuer(), self.pv_issuer()] + [
             self.softmax_warp(st, h) for st in (0, 1) for h in (0, 1)]
-        schedule(self.R, actors, [(self.tensor, self.on_tensor), (self.tma, self.on_tma)])
+        schedule(self.R, actors, [(self.tensor, self.on_tensor), (self.tma, self.on_tma),
+                                  (self.clock, self.on_tick)])
+
+    def on_tick(self, _):
+        if not self.clock:
+            self.aborted = True
 
 
 @pytest.mark.parametrize("kStV", [2, 3])  # V stages at d = 128 and d = 64
@@ -154,6 +199,16 @@ class Protocol:
 def test_forward_protocol_never_deadlocks_or_reads_stale(nkb, kStV):
     for seed in range(40):
         Protocol(nkb, seed, kStV).run()
+
+
+@pytest.mark.parametrize("nkb", [1, 2, 3, 5, 8, 13, 31])
+def test_forward_abort_at_any_point_ends_every_role(nkb):
+    """A wait that runs out at a random moment: every role takes its abort path (issuers and the
+    TMA thread stop, softmax warps keep meeting at their named barriers without touching tensor
+    memory) and every one of them ends, with its issued loads and MMAs drained."""
+    rng = random.Random(nkb)
+    for seed in range(80):
+        Protocol(nkb, seed, abort_after=rng.randint(1, 8 * nkb)).run()
 
 
 def test_model_catches_the_epilogue_on_a_per_buffer_barrier():
